@@ -1,0 +1,498 @@
+"""Pins of the fp64 oracle against values the pages and the mathematics fix.
+
+Every pin is written as a `check_*` function over the oracle module so that the
+mutation tests at the bottom can plant a plausible mistake in the oracle (on the
+CPU) and confirm that at least one pin catches it.
+"""
+import itertools
+import math
+
+import numpy as np
+import pytest
+import scipy.special
+import torch
+
+from oracle import moe_oracle as orc
+from tests.conftest import read_sections
+
+RNG = np.random.default_rng(1234)
+
+
+# --------------------------------------------------------------------------
+# capacity
+# --------------------------------------------------------------------------
+
+def check_capacity_worked_example(o=orc):
+    # "负载均衡策略：MoE训练稳定性保障", section "专家容量裁剪": 1024 tokens, 8 experts,
+    # ideal 128; factor 1.25 -> 160.
+    for row in read_sections("capacity_worked_example.txt")[""]:
+        T, N, k, cf, cap = int(row[0]), int(row[1]), int(row[2]), float(row[3]), int(row[4])
+        assert o.capacity(cf, T, k, N) == cap, (row, o.capacity(cf, T, k, N))
+
+
+def check_capacity_closed_forms(o=orc):
+    # C = ceil(cf * T * k / N) for the five workload shapes (exact integers) and
+    # for products that are not integers (ceiling, not floor or round).
+    assert o.capacity(1.25, 256, 2, 8) == 80
+    assert o.capacity(1.25, 4096, 2, 8) == 1280
+    assert o.capacity(1.0, 8192, 8, 128) == 512
+    assert o.capacity(1.25, 8192, 8, 256) == 320
+    assert o.capacity(1.25, 16384, 2, 8) == 5120
+    assert o.capacity(1.5, 7, 1, 2) == 6          # 5.25 -> 6
+    assert o.capacity(1.0, 10, 1, 4) == 3         # 2.5 -> 3
+    assert o.capacity(1.0, 0, 2, 8) == 0
+
+
+def test_capacity_worked_example():
+    check_capacity_worked_example()
+
+
+def test_capacity_closed_forms():
+    check_capacity_closed_forms()
+
+
+# --------------------------------------------------------------------------
+# softmax
+# --------------------------------------------------------------------------
+
+def check_softmax_library(o=orc):
+    # special case that reduces to a library routine: scipy's softmax
+    g = RNG.normal(size=(64, 16)) * 4.0
+    np.testing.assert_allclose(o.softmax(g), scipy.special.softmax(g, axis=1), rtol=1e-13, atol=0)
+    # large logits: exp would overflow without the max subtraction
+    big = np.array([[1000.0, 999.0, 0.0], [-1000.0, -1001.0, -1002.0]])
+    np.testing.assert_allclose(o.softmax(big), scipy.special.softmax(big, axis=1), rtol=1e-13)
+    assert np.all(np.isfinite(o.softmax(big)))
+
+
+def test_softmax_library():
+    check_softmax_library()
+
+
+# --------------------------------------------------------------------------
+# top-k selection and weights
+# --------------------------------------------------------------------------
+
+def _brute_topk(g_row, k):
+    """The unique k-subset whose members all precede every non-member under the
+    order 'larger logit first, then lower index', listed in that order."""
+    N = len(g_row)
+    key = lambda i: (-g_row[i], i)  # noqa: E731
+    hits = []
+    for S in itertools.combinations(range(N), k):
+        rest = [j for j in range(N) if j not in S]
+        if all(key(i) < key(j) for i in S for j in rest):
+            hits.append(sorted(S, key=key))
+    assert len(hits) == 1
+    return hits[0]
+
+
+def check_topk_bruteforce(o=orc):
+    rng = np.random.default_rng(7)
+    for N in (1, 2, 3, 5, 8):
+        for k in range(1, N + 1):
+            # small integers force many exact ties
+            g = rng.integers(-2, 3, size=(40, N)).astype(np.float64)
+            idx = o.topk(g, k)
+            for t in range(g.shape[0]):
+                assert list(idx[t]) == _brute_topk(list(g[t]), k), (N, k, g[t], idx[t])
+
+
+def check_topk_argmax(o=orc):
+    # k = 1 is argmax; numpy's argmax returns the first (lowest) index on ties
+    g = np.random.default_rng(3).integers(-3, 4, size=(200, 8)).astype(np.float64)
+    np.testing.assert_array_equal(o.topk(g, 1)[:, 0], np.argmax(g, axis=1))
+
+
+def check_weights(o=orc):
+    rng = np.random.default_rng(11)
+    g = rng.normal(size=(50, 8)) * 2
+    s = o.softmax(g)
+    for k in (1, 2, 3, 8):
+        idx = o.topk(g, k)
+        w = o.topk_weights(s, idx)
+        np.testing.assert_allclose(w.sum(axis=1), 1.0, rtol=0, atol=1e-12)
+        if k == 1:
+            np.testing.assert_allclose(w, 1.0, rtol=0, atol=1e-15)
+        if k == 8:   # k = N: the renormalised weights are the softmax itself
+            np.testing.assert_allclose(w, np.take_along_axis(s, idx.astype(np.int64), 1),
+                                       rtol=1e-13)
+    # N = 2, k = 2 closed form: the weight of the larger logit a vs b is
+    # 1 / (1 + exp(b - a))
+    a, b = 0.7, -0.4
+    w = o.topk_weights(o.softmax(np.array([[b, a]])), o.topk(np.array([[b, a]]), 2))
+    assert abs(w[0, 0] - 1.0 / (1.0 + math.exp(b - a))) < 1e-15
+
+
+def test_topk_bruteforce():
+    check_topk_bruteforce()
+
+
+def test_topk_argmax():
+    check_topk_argmax()
+
+
+def test_weights():
+    check_weights()
+
+
+# --------------------------------------------------------------------------
+# capacity clip and permutation
+# --------------------------------------------------------------------------
+
+def check_dispatch_hand(o=orc):
+    sec = read_sections("dispatch_hand.txt")
+    for name in ("A", "B"):
+        kv = {r[0]: [int(v) for v in r[1:]] for r in sec[name]}
+        T, N, k, C, align = kv["T"][0], kv["N"][0], kv["k"][0], kv["C"][0], kv["align"][0]
+        idx = np.array(kv["idx"], dtype=np.int32).reshape(T, k)
+        dp = o.dispatch(idx, N, C, align)
+        np.testing.assert_array_equal(dp.counts, kv["counts"])
+        np.testing.assert_array_equal(dp.kept, kv["kept"])
+        np.testing.assert_array_equal(dp.seg_off, kv["seg_off"])
+        np.testing.assert_array_equal(dp.row_map.reshape(-1), kv["row_map"])
+        assert dp.num_dropped == kv["dropped"][0]
+
+
+def check_dispatch_invariants(o=orc):
+    rng = np.random.default_rng(5)
+    for (T, N, k, C, align) in [(300, 8, 2, 40, 128), (257, 16, 4, 70, 32),
+                                (100, 5, 5, 100, 1), (64, 4, 1, 0, 8), (50, 3, 2, 1000, 16)]:
+        g = rng.normal(size=(T, N)) + np.linspace(1.5, -1.5, N)[None, :]
+        idx = o.topk(g, k)
+        dp = o.dispatch(idx, N, C, align)
+        np.testing.assert_array_equal(dp.counts, np.bincount(idx.reshape(-1), minlength=N))
+        np.testing.assert_array_equal(dp.kept, np.minimum(dp.counts, C))
+        assert int(dp.kept.sum()) == T * k - dp.num_dropped
+        assert np.all(dp.seg_off % align == 0)
+        kept_rows = dp.row_map[dp.row_map >= 0]
+        assert len(np.unique(kept_rows)) == len(kept_rows)           # injective
+        for e in range(N):
+            tok, slot = np.nonzero(idx == e)                          # token order
+            order = np.argsort(tok, kind="stable")
+            tok, slot = tok[order], slot[order]
+            rows = dp.row_map[tok, slot]
+            # the first min(count, C) tokens are kept, in order, at consecutive rows
+            n_keep = min(len(tok), C)
+            np.testing.assert_array_equal(rows[:n_keep], dp.seg_off[e] + np.arange(n_keep))
+            assert np.all(rows[n_keep:] == -1)
+            assert dp.seg_off[e + 1] - dp.seg_off[e] >= n_keep
+
+
+def test_dispatch_hand():
+    check_dispatch_hand()
+
+
+def test_dispatch_invariants():
+    check_dispatch_invariants()
+
+
+def test_permuted_rows_are_copies():
+    x = np.arange(24, dtype=np.float32).reshape(6, 4)
+    idx = np.array([[0], [0], [1], [0], [2], [0]], dtype=np.int32)
+    dp = orc.dispatch(idx, 3, 2, 4)
+    rows = orc.permuted_rows(x, dp)
+    assert sorted(rows) == [0, 1, 4, 8]
+    for r, t in ((0, 0), (1, 1), (4, 2), (8, 4)):
+        np.testing.assert_array_equal(rows[r], x[t])
+
+
+# --------------------------------------------------------------------------
+# FFN and combine
+# --------------------------------------------------------------------------
+
+def _py_matvec(xrow, W):
+    """Plain-Python x . W for a row x and a matrix W[d][f] (lists)."""
+    d, f = len(W), len(W[0])
+    return [sum(xrow[c] * W[c][j] for c in range(d)) for j in range(f)]
+
+
+def _py_swiglu(xrow, W1, W3, W2):
+    g = _py_matvec(xrow, W1)
+    u = _py_matvec(xrow, W3)
+    h = [gi / (1.0 + math.exp(-gi)) * ui for gi, ui in zip(g, u)]
+    return _py_matvec(h, W2)
+
+
+def _tiny_weights(rng, N, d, f):
+    w1 = rng.normal(size=(N, d, f)).astype(np.float32)
+    w3 = rng.normal(size=(N, d, f)).astype(np.float32)
+    w2 = rng.normal(size=(N, f, d)).astype(np.float32)
+    return w1, w3, w2
+
+
+def check_dense_mlp(o=orc):
+    # N = 1, k = 1, capacity >= T: the layer is one dense SwiGLU MLP
+    rng = np.random.default_rng(21)
+    T, d, f = 3, 4, 5
+    x = rng.normal(size=(T, d)).astype(np.float32)
+    wr = rng.normal(size=(d, 1)).astype(np.float32)
+    w1, w3, w2 = _tiny_weights(rng, 1, d, f)
+    res = o.layer_forward(x, wr, None, w1, w3, w2, k=1, cap=T, bf16=False, align=1)
+    for t in range(T):
+        want = _py_swiglu([float(v) for v in x[t]], w1[0].tolist(), w3[0].tolist(), w2[0].tolist())
+        np.testing.assert_allclose(res.y[t], want, rtol=1e-12, atol=1e-12)
+
+
+def check_dense_mixture(o=orc):
+    # k = N and capacity >= T: y = sum_i softmax_i(g) * Expert_i(x)
+    rng = np.random.default_rng(22)
+    T, d, f, N = 4, 3, 4, 3
+    x = rng.normal(size=(T, d)).astype(np.float32)
+    wr = rng.normal(size=(d, N)).astype(np.float32)
+    w1, w3, w2 = _tiny_weights(rng, N, d, f)
+    res = o.layer_forward(x, wr, None, w1, w3, w2, k=N, cap=T, bf16=False, align=1)
+    for t in range(T):
+        xr = [float(v) for v in x[t]]
+        g = [sum(xr[c] * float(wr[c, i]) for c in range(d)) for i in range(N)]
+        m = max(g)
+        ex = [math.exp(v - m) for v in g]
+        s = [v / sum(ex) for v in ex]
+        want = [0.0] * d
+        for i in range(N):
+            oi = _py_swiglu(xr, w1[i].tolist(), w3[i].tolist(), w2[i].tolist())
+            want = [a + s[i] * b for a, b in zip(want, oi)]
+        np.testing.assert_allclose(res.y[t], want, rtol=1e-12, atol=1e-12)
+
+
+def check_dropped_slots_contribute_zero(o=orc):
+    # capacity 0: every assignment is dropped, the routed output is exactly zero
+    rng = np.random.default_rng(23)
+    T, d, f, N = 5, 4, 4, 3
+    x = rng.normal(size=(T, d)).astype(np.float32)
+    wr = rng.normal(size=(d, N)).astype(np.float32)
+    w1, w3, w2 = _tiny_weights(rng, N, d, f)
+    res = o.layer_forward(x, wr, None, w1, w3, w2, k=2, cap=0, bf16=False, align=1)
+    assert np.all(res.y == 0.0)
+    # capacity 1 with k=1, N=1: only token 0 is kept and nothing is renormalised
+    wr1 = rng.normal(size=(d, 1)).astype(np.float32)
+    res = o.layer_forward(x, wr1, None, w1[:1], w3[:1], w2[:1], k=1, cap=1, bf16=False, align=1)
+    assert np.any(res.y[0] != 0.0) and np.all(res.y[1:] == 0.0)
+
+
+def check_shared_expert_added(o=orc):
+    # a shared expert is added with weight 1 on top of the routed sum
+    rng = np.random.default_rng(24)
+    T, d, f, N = 4, 3, 4, 2
+    x = rng.normal(size=(T, d)).astype(np.float32)
+    wr = rng.normal(size=(d, N)).astype(np.float32)
+    w1, w3, w2 = _tiny_weights(rng, N, d, f)
+    s1, s3, s2 = _tiny_weights(rng, 1, d, f)
+    base = o.layer_forward(x, wr, None, w1, w3, w2, k=1, cap=T, bf16=False, align=1)
+    both = o.layer_forward(x, wr, None, w1, w3, w2, k=1, cap=T, bf16=False, align=1,
+                           ws1=s1[0], ws3=s3[0], ws2=s2[0])
+    for t in range(T):
+        sh = _py_swiglu([float(v) for v in x[t]], s1[0].tolist(), s3[0].tolist(), s2[0].tolist())
+        np.testing.assert_allclose(both.y[t] - base.y[t], sh, rtol=1e-11, atol=1e-12)
+
+
+def test_dense_mlp():
+    check_dense_mlp()
+
+
+def test_dense_mixture():
+    check_dense_mixture()
+
+
+def test_dropped_slots_contribute_zero():
+    check_dropped_slots_contribute_zero()
+
+
+def test_shared_expert_added():
+    check_shared_expert_added()
+
+
+# --------------------------------------------------------------------------
+# load-balance statistics
+# --------------------------------------------------------------------------
+
+def check_aux_hand(o=orc):
+    sec = read_sections("aux_loss_4x4.txt")
+    p = np.array([[float(v) for v in r] for r in sec["probs"]])
+    g = np.log(p)
+    idx = o.topk(g, 1)
+    np.testing.assert_array_equal(idx[:, 0], [int(v) for v in sec["top1"][0]])
+    st = o.aux_stats(idx, o.softmax(g), 4)
+    np.testing.assert_allclose(st.y_frac, [float(v) for v in sec["y"][0]], rtol=0, atol=1e-15)
+    np.testing.assert_allclose(st.z_mean, [float(v) for v in sec["z"][0]], rtol=0, atol=1e-15)
+    assert abs(st.l_aux_p3 - float(sec["l_aux_p3"][0][0])) < 1e-14
+    assert abs(st.l_aux_switch - float(sec["l_aux_switch"][0][0])) < 1e-14
+
+
+def check_aux_uniform(o=orc):
+    # circulant logits: every expert sees the same score distribution and the same
+    # number of tokens, so f_i = P_i = 1/N and the Switch loss is exactly 1
+    N, k, reps = 8, 2, 5
+    c = np.array([3.0, 1.0, 0.5, 0.2, 0.1, -0.3, -1.0, -2.0])
+    T = N * reps
+    g = np.array([[c[(i - t) % N] for i in range(N)] for t in range(T)])
+    st = o.aux_stats(o.topk(g, k), o.softmax(g), N)
+    np.testing.assert_allclose(st.y_frac, 1.0 / N, rtol=1e-14)
+    np.testing.assert_allclose(st.z_mean, 1.0 / N, rtol=1e-13)
+    assert abs(st.l_aux_switch - 1.0) < 1e-13
+    assert abs(st.l_aux_p3 - T / N**2) < 1e-12
+
+
+def test_aux_hand():
+    check_aux_hand()
+
+
+def test_aux_uniform():
+    check_aux_uniform()
+
+
+# --------------------------------------------------------------------------
+# number formats
+# --------------------------------------------------------------------------
+
+def check_bf16_rounding(o=orc):
+    one = 1.0
+    assert o.round_to_bf16(np.array([one + 2.0**-8]))[0] == 1.0              # tie -> even
+    assert o.round_to_bf16(np.array([one + 3 * 2.0**-8]))[0] == 1.0 + 2.0**-6  # tie -> even (up)
+    assert o.round_to_bf16(np.array([one + 2.0**-8 + 2.0**-30]))[0] == 1.0 + 2.0**-7
+    assert o.round_to_bf16(np.array([-3.0]))[0] == -3.0
+    # library special case: torch's fp32 -> bf16 conversion rounds to nearest even
+    v = np.random.default_rng(9).normal(size=4096).astype(np.float32) * 10
+    v = np.concatenate([v, np.float32(2.0**-130) * np.arange(1, 64, dtype=np.float32)])
+    want = torch.from_numpy(v).to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(o.round_to_bf16(v.astype(np.float64)), want)
+
+
+def check_bf16_decode(o=orc):
+    bits = np.random.default_rng(10).integers(0, 2**16, size=4096).astype(np.uint16)
+    bits = bits[((bits >> 7) & 0xFF) != 0xFF]                   # finite values only
+    want = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(o.bf16_bits_to_f64(bits), want)
+
+
+def test_bf16_rounding():
+    check_bf16_rounding()
+
+
+def test_bf16_decode():
+    check_bf16_decode()
+
+
+# --------------------------------------------------------------------------
+# mutation tests: plant a plausible mistake in the oracle, expect a pin to fail
+# --------------------------------------------------------------------------
+
+ALL_CHECKS = [check_capacity_worked_example, check_capacity_closed_forms, check_softmax_library,
+              check_topk_bruteforce, check_topk_argmax, check_weights, check_dispatch_hand,
+              check_dispatch_invariants, check_dense_mlp, check_dense_mixture,
+              check_dropped_slots_contribute_zero, check_shared_expert_added, check_aux_hand,
+              check_aux_uniform, check_bf16_rounding, check_bf16_decode]
+
+
+def _mut_topk_high_index_ties(g, k):
+    g = np.asarray(g, np.float64)
+    return np.argsort(g, axis=1, kind="stable")[:, ::-1][:, :k].astype(np.int32)
+
+
+def _mut_weights_no_renorm(s, idx):
+    return np.take_along_axis(s, idx.astype(np.int64), axis=1)
+
+
+def _mut_capacity_floor(cf, T, k, N):
+    from fractions import Fraction
+    return int(math.floor(Fraction(cf) * T * k / N))
+
+
+def _mut_capacity_no_k(cf, T, k, N):
+    from fractions import Fraction
+    return int(math.ceil(Fraction(cf) * T / N))
+
+
+def _mut_dispatch_drop_whole_expert(idx, N, C, align=128):
+    # the literal reading of the page's snippet: an over-full expert loses all tokens
+    d = orc.Dispatch.__new__(orc.Dispatch)
+    ref = _ORIG["dispatch"](idx, N, C, align)
+    rm = ref.row_map.copy()
+    for e in range(N):
+        if ref.counts[e] > C:
+            rm[idx == e] = -1
+    d.__dict__.update(ref.__dict__)
+    d.row_map = rm
+    return d
+
+
+def _mut_dispatch_keep_last(idx, N, C, align=128):
+    ref = _ORIG["dispatch"](idx[::-1].copy(), N, C, align)
+    d = orc.Dispatch.__new__(orc.Dispatch)
+    d.__dict__.update(ref.__dict__)
+    d.row_map = ref.row_map[::-1].copy()
+    return d
+
+
+def _mut_softmax_no_max(g):
+    with np.errstate(over="ignore", invalid="ignore"):
+        z = np.exp(np.asarray(g, np.float64))
+        return z / z.sum(axis=1, keepdims=True)
+
+
+def _mut_silu_sign(u):
+    with np.errstate(over="ignore"):
+        return u / (1.0 + np.exp(u))
+
+
+def _mut_swiglu_swap(x64, w1, w3, w2, round_h_bf16):
+    return _ORIG["swiglu_ffn"](x64, w3, w1, w2, round_h_bf16)
+
+
+def _mut_aux_z_topk(idx, s, N):
+    st = _ORIG["aux_stats"](idx, s, N)
+    w = orc.topk_weights(s, idx)
+    z = np.zeros(N)
+    np.add.at(z, idx.reshape(-1), w.reshape(-1))
+    z /= idx.shape[0]
+    st.z_mean = z
+    return st
+
+
+def _mut_aux_p3_inverted(idx, s, N):
+    st = _ORIG["aux_stats"](idx, s, N)
+    T = idx.shape[0]
+    st.l_aux_p3 = (N / T) * float(np.sum(st.y_frac * st.z_mean))
+    return st
+
+
+def _mut_bf16_truncate(v):
+    v = np.asarray(v, np.float64).astype(np.float32)
+    u = v.view(np.uint32) & np.uint32(0xFFFF0000)
+    return u.view(np.float32).astype(np.float64)
+
+
+def _mut_bf16_decode_low_half(bits):
+    u32 = np.asarray(bits, dtype=np.uint16).astype(np.uint32)
+    return u32.view(np.float32).astype(np.float64)
+
+
+_ORIG = {n: getattr(orc, n) for n in ("dispatch", "swiglu_ffn", "aux_stats")}
+
+MUTANTS = [
+    ("topk", _mut_topk_high_index_ties),
+    ("topk_weights", _mut_weights_no_renorm),
+    ("capacity", _mut_capacity_floor),
+    ("capacity", _mut_capacity_no_k),
+    ("dispatch", _mut_dispatch_drop_whole_expert),
+    ("dispatch", _mut_dispatch_keep_last),
+    ("softmax", _mut_softmax_no_max),
+    ("silu", _mut_silu_sign),
+    ("swiglu_ffn", _mut_swiglu_swap),
+    ("aux_stats", _mut_aux_z_topk),
+    ("aux_stats", _mut_aux_p3_inverted),
+    ("round_to_bf16", _mut_bf16_truncate),
+    ("bf16_bits_to_f64", _mut_bf16_decode_low_half),
+]
+
+
+@pytest.mark.parametrize("name,mutant", MUTANTS, ids=[f"{n}:{m.__name__}" for n, m in MUTANTS])
+def test_mutant_is_caught(monkeypatch, name, mutant):
+    monkeypatch.setattr(orc, name, mutant)
+    caught = []
+    for chk in ALL_CHECKS:
+        try:
+            chk(orc)
+        except (AssertionError, ValueError, FloatingPointError, IndexError):
+            caught.append(chk.__name__)
+    assert caught, f"no pin caught the planted mistake in {name}"
