@@ -1,0 +1,465 @@
+"""Benchmark of the MoE-layer forward pass on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config qwen3] [--impl ours|reference]
+
+A step is one forward pass of the whole layer (router GEMM + softmax + top-k +
+statistics, capacity clip + permutation, grouped SwiGLU GEMMs, combine) over one
+synthetic batch of the named workload, through the C ABI of libmoe.so.
+
+  value     tokens/s of moe_layer_fwd with inputs resident in HBM (K steps,
+            CUDA events, max over ranks; every rank runs an independent replica,
+            so the work per GPU is fixed: weak scaling)
+  e2e       the same call with the batch copied in from pinned host memory and
+            the output copied back inside the timed region
+  kernels   per-stage times from CUDA events recorded between the C-ABI steps
+            (moe_route, moe_dispatch, moe_expert_ffn, moe_combine) of a second
+            timed region, with each stage's algorithmic work and roofline
+  roofline  the dominant kernel (the grouped GEMM pair of moe_expert_ffn)
+  cpu_baseline  the fp64 oracle on the host cores, on a bounded sample
+
+--impl reference times the fp64 oracle (the reference of this method) on the
+host cores instead, on the same workload and metric.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from expert_router_gemm_b200 import configs, synth  # noqa: E402
+
+METRIC = "MoE-layer fwd tokens/s on 1 B200; grouped-GEMM % bf16 TC peak; permute GB/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# fp32 FFMA peak of a B200: 148 SMs x 128 FP32 lanes x 2 flop x 1.965 GHz (max SM clock)
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def traffic_record(kernel_file: str):
+    """DRAM bytes per launch from the committed ncu summary, or None when the
+    kernel source changed since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    src = os.path.join(ROOT, "expert_router_gemm_b200", "csrc", kernel_file)
+    if not (os.path.exists(path) and os.path.exists(src)):
+        return None
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    out = {}
+    for line in open(path):
+        parts = line.split()
+        if len(parts) >= 4 and not line.startswith("#") and parts[1] == sha:
+            out[parts[0]] = float(parts[2]) + float(parts[3])
+    return out or None
+
+
+# ----------------------------------------------------------------- clocks (NVML, read only)
+class ClockSampler:
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, torch_dev: int, period_s: float = 0.02):
+        self.ok = False
+        self.samples = []
+        self.period = period_s
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(torch_dev)
+            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+            self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # pragma: no cover - depends on the box
+            self.err = repr(e)
+
+    def _reasons(self):
+        nv = self.nv
+        fn = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        return fn(self.h)
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append((nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM),
+                                     nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0,
+                                     self._reasons()))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._stop = threading.Event()
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        mhz = [s[0] for s in self.samples]
+        bits = 0
+        for s in self.samples:
+            bits |= s[2]
+        reasons = [n for b, n in self.REASONS.items() if bits & b and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(mhz), "power_w_max": round(max(s[1] for s in self.samples), 1)}
+
+
+# ----------------------------------------------------------------- oracle timing (CPU)
+def oracle_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max([i.get("num_threads", 1) for i in info if i.get("user_api") == "blas"] or [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_expert_steps(w, inp, n_steps=None, budget_s=None):
+    """Time the fp64 oracle on a bounded sample of the workload: the routing of
+    all T tokens once, then one expert per step (its kept rows through the SwiGLU
+    FFN and their weighted contributions to the combine).  Returns a list of
+    (token_equivalents, seconds) per step and the routing time."""
+    from oracle import moe_oracle as orc
+    t0 = time.perf_counter()
+    g = orc.router_logits(inp.x, inp.w_router, inp.bias)
+    s = orc.softmax(g)
+    idx = orc.topk(g, w.k)
+    wts = orc.topk_weights(s, idx)
+    cap = orc.capacity(w.capacity_factor, w.T, w.k, w.N)
+    disp = orc.dispatch(idx, w.N, cap, 128)
+    orc.aux_stats(idx, s, w.N)
+    t_route = time.perf_counter() - t0
+    bf16 = w.dtype == "bf16"
+    y = np.zeros((w.T, w.d))
+    steps = []
+    order = np.argsort(-disp.kept, kind="stable")   # busiest experts first: fixed order
+    i = 0
+    start = time.perf_counter()
+    while True:
+        if n_steps is not None and i >= n_steps:
+            break
+        if budget_s is not None and time.perf_counter() - start >= budget_s and i > 0:
+            break
+        e = int(order[i % w.N])
+        ts = time.perf_counter()
+        ti, tj = np.nonzero((idx == e) & (disp.row_map >= 0))
+        if len(ti):
+            o = orc.swiglu_ffn(orc.as_f64(inp.x[ti]), inp.w1[e], inp.w3[e], inp.w2[e], bf16)
+            np.add.at(y, ti, wts[ti, tj][:, None] * o)
+        steps.append((len(ti) / w.k, time.perf_counter() - ts))
+        i += 1
+    return steps, t_route
+
+
+def cpu_rate(steps, t_route, T):
+    tok = sum(s[0] for s in steps)
+    sec = sum(s[1] for s in steps) + t_route * tok / T   # routing amortised per token
+    return tok / sec if sec > 0 else 0.0, tok, sec
+
+
+def run_reference(args, w, rank, world):
+    """--impl reference: the fp64 oracle on the host cores (rank 0 only)."""
+    if rank != 0:
+        return
+    inp = synth.make_inputs(w)
+    warm, _ = oracle_expert_steps(w, inp, n_steps=args.warmup)
+    steps, t_route = oracle_expert_steps(w, inp, n_steps=args.steps)
+    rate, tok, sec = cpu_rate(steps, t_route, w.T)
+    cores = oracle_threads()
+    sample = (f"fp64 oracle: routing of all {w.T} tokens once (time amortised per token), "
+              f"then per step the kept rows of one expert through the SwiGLU FFN and the "
+              f"combine; {args.steps} steps = {tok:.0f} token-equivalents")
+    line = {"impl": "reference", "metric": METRIC, "value": round(rate, 3), "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1e3 * sec / max(1, len(steps)), 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(w),
+            "cpu_baseline": {"value": round(rate, 3), "unit": "tokens/s", "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(rate, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w):
+    return {"workload": w.name, "T": w.T, "d": w.d, "N": w.N, "k": w.k, "f": w.f,
+            "f_shared": w.f_shared, "capacity_factor": w.capacity_factor,
+            "capacity": int(np.ceil(w.capacity_factor * w.T * w.k / w.N)),
+            "act_dtype": w.dtype, "router_dtype": "f32", "seed": w.seed}
+
+
+# ----------------------------------------------------------------- our arm
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--config", default="qwen3")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work")
+    ap.add_argument("--quick", action="store_true", help="layer loop only (profiling runs)")
+    args = ap.parse_args()
+    if args.warmup < 3 and not args.quick:
+        ap.error("--warmup must be >= 3")
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    w = configs.get(args.config)
+
+    if args.impl == "reference":
+        run_reference(args, w, rank, world)
+        return
+
+    import torch
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    from expert_router_gemm_b200 import moe
+
+    inp = synth.make_inputs(w)
+    cfg = moe.config_from_workload(w)
+    dl = moe.to_device(inp, cfg)
+    act = moe.act_dtype(cfg)
+    elem = 2 if w.dtype == "bf16" else 4
+    lb, ob, max_rows = moe.moe_workspace_size(cfg)
+    ws = torch.empty(lb, dtype=torch.uint8, device="cuda")
+    y = torch.empty((w.T, w.d), dtype=act, device="cuda")
+    sbuf = dict(y_frac=torch.empty(w.N, device="cuda"), z_mean=torch.empty(w.N, device="cuda"),
+                l_aux_p3=torch.empty(1, device="cuda"), l_aux_switch=torch.empty(1, device="cuda"),
+                counts=torch.empty(w.N, dtype=torch.int32, device="cuda"),
+                kept=torch.empty(w.N, dtype=torch.int32, device="cuda"),
+                num_dropped=torch.empty(1, dtype=torch.int32, device="cuda"))
+    stats = moe.make_stats(**sbuf)
+    weights = dl.weights()
+    stream = torch.cuda.current_stream()
+
+    def layer():
+        moe.moe_layer_fwd(cfg, weights, dl.x, y, stats, ws, stream)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if dist is None:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        layer()
+    torch.cuda.synchronize()
+    flags = moe.moe_read_flags(ws)
+    dropped = int(sbuf["num_dropped"].item())
+    a_kept = w.T * w.k - dropped
+
+    # ------------------------------------------------ region A: the layer call
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize()
+    with sampler:
+        ev0.record(stream)
+        for _ in range(args.steps):
+            layer()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    ms = max_over_ranks(ev0.elapsed_time(ev1)) / args.steps
+    value = world * w.T / (ms / 1e3)
+    clocks = sampler.summary()
+
+    per_step_launches = 1 + 1 + 3 + 2 + (2 if w.f_shared else 0) + 1
+    line = {"metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+            "data": "synthetic",
+            "config": dict(workload_config(w), parallelism=f"replicas x{world}",
+                           l2="inputs larger than L2: the expert weights read every step "
+                              f"({(inp.w1.nbytes + inp.w3.nbytes + inp.w2.nbytes) / 1e9:.2f} GB) "
+                              "exceed the 126 MB L2; no flush"),
+            "gpu_launches": per_step_launches * args.steps, "clocks": clocks,
+            "device_flags": flags, "dropped": dropped}
+
+    if not args.quick:
+        # -------------------------------------------- region B: per-stage events
+        T, N, k, d, f = w.T, w.N, w.k, w.d, w.f
+        ws_op = torch.empty(ob, dtype=torch.uint8, device="cuda")
+        idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+        wt = torch.empty((T, k), dtype=torch.float32, device="cuda")
+        row_map = torch.empty((T, k), dtype=torch.int32, device="cuda")
+        seg_off = torch.empty(N + 1, dtype=torch.int32, device="cuda")
+        seg_count = torch.empty(N, dtype=torch.int32, device="cuda")
+        xp = torch.empty((max_rows, d), dtype=act, device="cuda")
+        h = torch.empty((max_rows, f), dtype=act, device="cuda")
+        hs = torch.empty((T, w.f_shared), dtype=act, device="cuda") if w.f_shared else None
+        sh = torch.empty((T, d), dtype=act, device="cuda") if w.f_shared else None
+        names = ["route", "dispatch", "expert_ffn", "shared_ffn", "combine"]
+
+        def staged(evs):
+            evs[0].record(stream)
+            moe.moe_route(cfg, dl.x, dl.w_router, dl.bias, None, idx, wt, stats, ws_op, stream)
+            evs[1].record(stream)
+            moe.moe_dispatch(cfg, dl.x, idx, row_map, seg_off, seg_count, xp, stats, ws_op, stream)
+            evs[2].record(stream)
+            moe.moe_expert_ffn(cfg, xp, seg_off, seg_count, weights, h, xp, ws_op, stream)
+            evs[3].record(stream)
+            if w.f_shared:
+                moe.moe_shared_expert_ffn(cfg, dl.x, weights, hs, sh, ws_op, stream)
+            evs[4].record(stream)
+            moe.moe_combine(cfg, xp, row_map, wt, sh, y, ws_op, stream)
+            evs[5].record(stream)
+
+        for _ in range(3):
+            staged([torch.cuda.Event(enable_timing=True) for _ in range(6)])
+        all_evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+        barrier()
+        torch.cuda.synchronize()
+        for evs in all_evs:
+            staged(evs)
+        torch.cuda.synchronize()
+        stage_ms = {n: 0.0 for n in names}
+        for evs in all_evs:
+            for i, n in enumerate(names):
+                stage_ms[n] += evs[i].elapsed_time(evs[i + 1])
+        stage_ms = {n: max_over_ranks(v) / args.steps for n, v in stage_ms.items()}
+
+        peaks, peak_src = load_peaks()
+        hbm = peaks["hbm_gbs"]
+        tc_peak = peaks["bf16_tflops_sustained"]
+        x_bytes = T * d * elem
+        route_bytes = x_bytes + d * N * 4 + T * k * 8
+        route_flops = 2.0 * T * d * N
+        disp_bytes = x_bytes + a_kept * d * elem + T * k * 8
+        ffn_flops = 6.0 * d * f * a_kept
+        ffn_wbytes = 3.0 * N * d * f * elem
+        comb_bytes = a_kept * d * elem + T * k * 8 + x_bytes + (x_bytes if w.f_shared else 0)
+        sh_flops = 6.0 * T * d * w.f_shared
+
+        def gbs(b, ms_):
+            return b / (ms_ / 1e3) / 1e9 if ms_ > 0 else None
+
+        def tfs(fl, ms_):
+            return fl / (ms_ / 1e3) / 1e12 if ms_ > 0 else None
+
+        kern = {
+            "route": {"ms": round(stage_ms["route"], 4), "bytes": route_bytes, "flops": route_flops,
+                      "GB/s": round(gbs(route_bytes, stage_ms["route"]), 1),
+                      "frac_hbm": round(gbs(route_bytes, stage_ms["route"]) / hbm, 4),
+                      "TFLOP/s_fp32": round(tfs(route_flops, stage_ms["route"]), 2),
+                      "frac_fp32_alu": round(tfs(route_flops, stage_ms["route"]) / FP32_ALU_TFLOPS, 4)},
+            "dispatch": {"ms": round(stage_ms["dispatch"], 4), "bytes": disp_bytes,
+                         "GB/s": round(gbs(disp_bytes, stage_ms["dispatch"]), 1),
+                         "frac_hbm": round(gbs(disp_bytes, stage_ms["dispatch"]) / hbm, 4)},
+            "expert_ffn": {"ms": round(stage_ms["expert_ffn"], 4), "flops": ffn_flops,
+                           "TFLOP/s": round(tfs(ffn_flops, stage_ms["expert_ffn"]), 1),
+                           "frac_tensor": round(tfs(ffn_flops, stage_ms["expert_ffn"]) / tc_peak, 4),
+                           "weight_bytes": ffn_wbytes,
+                           "weight_GB/s": round(gbs(ffn_wbytes, stage_ms["expert_ffn"]), 1)},
+            "combine": {"ms": round(stage_ms["combine"], 4), "bytes": comb_bytes,
+                        "GB/s": round(gbs(comb_bytes, stage_ms["combine"]), 1),
+                        "frac_hbm": round(gbs(comb_bytes, stage_ms["combine"]) / hbm, 4)},
+        }
+        if w.f_shared:
+            kern["shared_ffn"] = {"ms": round(stage_ms["shared_ffn"], 4), "flops": sh_flops,
+                                  "TFLOP/s": round(tfs(sh_flops, stage_ms["shared_ffn"]), 1)}
+        line["kernels"] = kern
+        line["stage_sum_ms"] = round(sum(stage_ms.values()), 4)
+        ffn_tf = tfs(ffn_flops, stage_ms["expert_ffn"])
+        tr = traffic_record("ffn_tc.cu")
+        line["roofline"] = {
+            "kernel": "tc_ffn_gemm_kernel (grouped SwiGLU GEMM + down GEMM, the two launches of "
+                      "moe_expert_ffn)",
+            "bound": "tensor", "achieved": round(ffn_tf, 1), "peak": tc_peak, "unit": "TFLOP/s",
+            "frac": round(ffn_tf / tc_peak, 4),
+            "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a seconds-long loop)",
+            "frac_of_burst_peak": round(ffn_tf / peaks["bf16_tflops"], 4),
+            "algorithmic_flops_per_step": ffn_flops,
+            "traffic": (tr["expert_ffn_per_step"] * 1.0 if tr and "expert_ffn_per_step" in tr else None)}
+
+        # -------------------------------------------- e2e: host buffers through the C ABI
+        x_host = torch.empty_like(dl.x, device="cpu").pin_memory()
+        x_host.copy_(dl.x.cpu())
+        y_host = torch.empty((T, d), dtype=act).pin_memory()
+        x_in = torch.empty_like(dl.x)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+        def e2e_step():
+            x_in.copy_(x_host, non_blocking=True)
+            moe.moe_layer_fwd(cfg, weights, x_in, y, stats, ws, stream)
+            y_host.copy_(y, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / args.steps
+        line["e2e"] = {"value": round(world * T / (e2e_ms / 1e3), 1), "unit": "tokens/s",
+                       "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
+                       "d2h_bytes_per_step": y_host.numel() * y_host.element_size(),
+                       "ms_per_step": round(e2e_ms, 4)}
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.quick:
+        steps, t_route = oracle_expert_steps(w, inp, budget_s=args.cpu_budget)
+        rate, tok, sec = cpu_rate(steps, t_route, w.T)
+        line["cpu_baseline"] = {
+            "value": round(rate, 3), "unit": "tokens/s", "cores": oracle_threads(), "kind": "oracle",
+            "sample": f"fp64 oracle: routing of all {w.T} tokens ({t_route:.2f} s, amortised per "
+                      f"token) + the kept rows of the {len(steps)} busiest experts through SwiGLU "
+                      f"and combine = {tok:.0f} token-equivalents in {sec:.1f} s"}
+
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

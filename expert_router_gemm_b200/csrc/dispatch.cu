@@ -1,0 +1,179 @@
+// Capacity clip and permutation into expert-contiguous rows.
+//
+// "负载均衡策略：MoE训练稳定性保障", section "专家容量裁剪": each expert processes at
+// most C = ceil(capacity_factor * T * k / N) tokens and the overflow is dropped;
+// the drop order here is token order (the earliest C assignments of an expert
+// are kept).  "ETP专家并行加速MoE模型", section "动态路由下的高效通信": the tokens
+// are re-shuffled to their experts; on one GPU that is a stable scatter into one
+// buffer with a contiguous segment per expert.
+//
+// Three kernels, no atomics whose order matters and no spin waits:
+//   1. mask:    per block of 32 tokens, a 32-bit token mask per expert
+//               (bit t set iff token t of the block chose the expert);
+//   2. scan:    per expert, exclusive prefix of popcount(mask) over the blocks
+//               (-> rank base of every block) and the total count; the last block
+//               to finish (ticket counter, no waiting) turns the counts into
+//               kept = min(count, C) and the aligned segment offsets;
+//   3. scatter: rank of (t, e) = base[block][e] + popcount of the mask bits below
+//               t, kept iff rank < C; row = seg_off[e] + rank; one warp per token
+//               copies x[t] with 16-byte vectors to each of its kept rows.
+#include "device_utils.cuh"
+#include "internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int kMaskThreads = 256;
+constexpr int kScatterThreads = 32 * kDispatchTokens;  // one warp per token
+constexpr int kCopyUnroll = 4;
+
+// true iff slot j of token t holds a valid expert index not used by an earlier slot
+__device__ __forceinline__ bool slot_valid(const int32_t* idx_row, int j, int e, int N) {
+  if (e < 0 || e >= N) return false;
+  for (int j2 = 0; j2 < j; ++j2)
+    if (idx_row[j2] == e) return false;
+  return true;
+}
+
+__global__ void __launch_bounds__(kMaskThreads) dispatch_mask_kernel(const DispatchArgs a) {
+  __shared__ uint32_t m[256];
+  const int tid = threadIdx.x;
+  const int N = a.N, k = a.k;
+  for (int e = tid; e < N; e += kMaskThreads) m[e] = 0u;
+  if (blockIdx.x == 0 && tid == 0) *a.ticket = 0u;
+  __syncthreads();
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kDispatchTokens;
+  for (int s = tid; s < kDispatchTokens * k; s += kMaskThreads) {
+    const int tl = s / k, j = s % k;
+    const int64_t t = t0 + tl;
+    if (t >= a.T) continue;
+    const int32_t* row = a.topk_idx + t * k;
+    const int e = row[j];
+    if (!slot_valid(row, j, e, N)) {
+      atomicOr(a.flags, kFlagBadIndex);
+      continue;
+    }
+    atomicOr(&m[e], 1u << tl);
+  }
+  __syncthreads();
+  for (int e = tid; e < N; e += kMaskThreads)
+    a.mask[static_cast<int64_t>(blockIdx.x) * N + e] = m[e];
+}
+
+// grid: ceil(N / 32) blocks of 32 warps; lane = expert, warp = a run of blocks
+__global__ void __launch_bounds__(1024) dispatch_scan_kernel(const DispatchArgs a, int blocks) {
+  __shared__ int part[32][33];
+  __shared__ int is_last;
+  __shared__ int kept_s[256];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int N = a.N;
+  const int e = blockIdx.x * 32 + lane;
+  const int chunk = (blocks + 31) / 32;
+  const int b_lo = min(blocks, warp * chunk), b_hi = min(blocks, b_lo + chunk);
+
+  int s = 0;
+  if (e < N)
+    for (int b = b_lo; b < b_hi; ++b) s += __popc(a.mask[static_cast<int64_t>(b) * N + e]);
+  part[warp][lane] = s;
+  __syncthreads();
+  int excl = 0;
+  for (int w = 0; w < warp; ++w) excl += part[w][lane];
+  if (e < N) {
+    int run = excl;
+    for (int b = b_lo; b < b_hi; ++b) {
+      a.base[static_cast<int64_t>(b) * N + e] = run;
+      run += __popc(a.mask[static_cast<int64_t>(b) * N + e]);
+    }
+    if (warp == 31) a.counts[e] = run;
+  }
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) is_last = (atomicAdd(a.ticket, 1u) == gridDim.x - 1);
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+
+  // last block: kept counts, aligned segment offsets, statistics
+  long long dropped = 0;
+  for (int x = threadIdx.x; x < N; x += blockDim.x) {
+    const int c = __ldcg(a.counts + x);
+    const int kept = min(c, a.capacity);
+    kept_s[x] = kept;
+    a.seg_count[x] = kept;
+    if (a.stats.counts) a.stats.counts[x] = c;
+    if (a.stats.kept) a.stats.kept[x] = kept;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    long long off = 0;
+    for (int x = 0; x < N; ++x) {
+      a.seg_off[x] = static_cast<int32_t>(off);
+      off += (kept_s[x] + a.align - 1) / a.align * static_cast<long long>(a.align);
+      dropped += __ldcg(a.counts + x) - kept_s[x];
+    }
+    a.seg_off[N] = static_cast<int32_t>(off);
+    if (a.stats.num_dropped) a.stats.num_dropped[0] = static_cast<int32_t>(dropped);
+  }
+}
+
+__global__ void __launch_bounds__(kScatterThreads) dispatch_scatter_kernel(const DispatchArgs a) {
+  __shared__ uint32_t m[256];
+  __shared__ int base_s[256];
+  __shared__ int off_s[256];
+  __shared__ int rows_s[kDispatchTokens][32];
+  const int N = a.N, k = a.k;
+  const int64_t blk = blockIdx.x;
+  for (int e = threadIdx.x; e < N; e += kScatterThreads) {
+    m[e] = a.mask[blk * N + e];
+    base_s[e] = a.base[blk * N + e];
+    off_s[e] = a.seg_off[e];
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t t = blk * kDispatchTokens + warp;
+  if (t >= a.T) return;
+
+  if (lane < k) {
+    const int32_t* row = a.topk_idx + t * k;
+    const int e = row[lane];
+    int r = -1;
+    if (slot_valid(row, lane, e, N)) {
+      const int rank = base_s[e] + __popc(m[e] & ((1u << warp) - 1u));
+      if (rank < a.capacity) r = off_s[e] + rank;
+    }
+    a.row_map[t * k + lane] = r;
+    rows_s[warp][lane] = r;
+  }
+  __syncwarp();
+
+  // copy the row once from HBM, write it to each kept slot (16-byte vectors)
+  const int64_t nvec = static_cast<int64_t>(a.d) * a.elem_bytes / 16;
+  const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(a.x) + t * nvec * 16);
+  uint4* dst = static_cast<uint4*>(a.xp);
+  for (int64_t c = lane; c < nvec; c += 32 * kCopyUnroll) {
+    uint4 v[kCopyUnroll];
+#pragma unroll
+    for (int u = 0; u < kCopyUnroll; ++u)
+      if (c + 32 * u < nvec) v[u] = src[c + 32 * u];
+    for (int j = 0; j < k; ++j) {
+      const int r = rows_s[warp][j];
+      if (r < 0) continue;
+      uint4* drow = dst + static_cast<int64_t>(r) * nvec;
+#pragma unroll
+      for (int u = 0; u < kCopyUnroll; ++u)
+        if (c + 32 * u < nvec) drow[c + 32 * u] = v[u];
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t s) {
+  const int blocks = static_cast<int>((a.T + kDispatchTokens - 1) / kDispatchTokens);
+  dispatch_mask_kernel<<<blocks, kMaskThreads, 0, s>>>(a);
+  dispatch_scan_kernel<<<(a.N + 31) / 32, 1024, 0, s>>>(a, blocks);
+  dispatch_scatter_kernel<<<blocks, kScatterThreads, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

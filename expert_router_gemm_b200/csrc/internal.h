@@ -1,0 +1,117 @@
+// Internal declarations shared by the host entry points (moe_api.cu) and the
+// kernel translation units.  Not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "moe.h"
+
+namespace moe {
+
+// ---------------------------------------------------------------- routing
+// The router kernel is instantiated for a padded expert count NP (a power of
+// two >= 8, >= N); experts N..NP-1 are masked.  Each block handles route_bt(NP)
+// tokens with 256 threads.
+constexpr int kRouteThreads = 256;
+
+inline constexpr int route_np(int N) {
+  return N <= 8 ? 8 : N <= 16 ? 16 : N <= 32 ? 32 : N <= 64 ? 64 : N <= 128 ? 128 : 256;
+}
+inline constexpr int route_bt(int np) {
+  return np == 8 ? 256 : np == 16 ? 256 : np == 32 ? 128 : np == 64 ? 128 : np == 128 ? 64 : 32;
+}
+
+struct RouteArgs {
+  int64_t T;
+  int d, N, k;
+  int x_is_bf16;            // 1: x holds bf16 bits, 0: fp32
+  const void* x;            // [T, d] (GEMM mode) or nullptr
+  const float* w_router;    // [d, N]
+  const float* bias;        // [N] or nullptr
+  const float* logits_in;   // [T, N] (logits mode) or nullptr
+  float* logits_out;        // [T, N] or nullptr
+  int32_t* topk_idx;        // [T, k]
+  float* topk_w;            // [T, k]
+  int32_t* hist;            // [blocks, N]
+  float* zpart;             // [blocks, N]
+  uint32_t* flags;
+};
+cudaError_t launch_route(const RouteArgs& a, cudaStream_t s);
+
+struct RouteStatsArgs {
+  int64_t T;
+  int N, k, blocks;
+  const int32_t* hist;
+  const float* zpart;
+  moe_stats_t stats;        // device pointers, each may be null
+};
+cudaError_t launch_route_stats(const RouteStatsArgs& a, cudaStream_t s);
+
+// --------------------------------------------------------------- dispatch
+constexpr int kDispatchTokens = 32;   // tokens per dispatch block (one bit each)
+
+struct DispatchArgs {
+  int64_t T;
+  int d, N, k, capacity, align, elem_bytes;
+  const void* x;
+  const int32_t* topk_idx;
+  int32_t* row_map;
+  int32_t* seg_off;
+  int32_t* seg_count;
+  void* xp;
+  uint32_t* mask;           // [blocks, N] scratch
+  int32_t* base;            // [blocks, N] scratch
+  int32_t* counts;          // [N] scratch
+  uint32_t* ticket;         // [1] scratch
+  moe_stats_t stats;
+  uint32_t* flags;
+};
+cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t s);
+
+// ------------------------------------------------------------ expert FFN
+// One grouped SwiGLU FFN over G groups of rows.  Group g owns rows
+// [row0_g, row0_g + count_g) of `a` / `h` / `out`, where row0_g = seg_off[g]
+// and count_g = seg_count[g]; with seg_off == nullptr there is one group of
+// `dense_rows` rows starting at row 0.
+struct FfnArgs {
+  int G;
+  int dense_rows;
+  int max_count;            // upper bound of count_g (grid sizing of the fp32 path)
+  int64_t max_rows;         // rows of a / h / out buffers
+  int d, f;
+  const int32_t* seg_off;
+  const int32_t* seg_count;
+  const void* a;            // [rows, d]
+  const void* w1;           // [G][d][f]
+  const void* w3;           // [G][d][f]
+  const void* w2;           // [G][f][d]
+  void* h;                  // [rows, f]
+  void* out;                // [rows, d]
+  uint32_t* flags;
+};
+cudaError_t launch_ffn_bf16(const FfnArgs& a, cudaStream_t s);
+cudaError_t launch_ffn_f32(const FfnArgs& a, cudaStream_t s);
+
+// ---------------------------------------------------------------- combine
+struct CombineArgs {
+  int64_t T;
+  int d, k, is_bf16;
+  const void* out_rows;
+  const int32_t* row_map;
+  const float* topk_w;
+  const void* shared_out;   // or nullptr
+  void* y;
+};
+cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s);
+
+// flags word bits used by kernels (mirror of the public MOE_FLAG_* values)
+constexpr uint32_t kFlagNonfinite = MOE_FLAG_NONFINITE_LOGITS;
+constexpr uint32_t kFlagBadIndex = MOE_FLAG_BAD_EXPERT_INDEX;
+constexpr uint32_t kFlagTimeout = MOE_FLAG_WAIT_TIMEOUT;
+
+int device_sm_count();    // cached per device
+
+}  // namespace moe

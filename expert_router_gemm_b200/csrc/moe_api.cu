@@ -1,0 +1,469 @@
+// Host side of libmoe.so: argument validation, the exact capacity formula, the
+// workspace layout and the C-ABI entry points declared in include/moe.h.
+// Everything here runs on the host; every step of the computation runs in the
+// CUDA kernels of route.cu, dispatch.cu, ffn_tc.cu, ffn_f32.cu and combine.cu.
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+
+#include "internal.h"
+
+namespace moe {
+
+int device_sm_count() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  int& c = cache[dev & 63];
+  if (c == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+    c = v;
+  }
+  return c;
+}
+
+}  // namespace moe
+
+namespace {
+
+using namespace moe;
+
+thread_local char g_last_cuda_error[256] = "";
+
+moe_status_t cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return MOE_OK;
+  std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s: %s", cudaGetErrorName(e),
+                cudaGetErrorString(e));
+  return MOE_ERR_CUDA;
+}
+
+constexpr size_t kAlign = 256;
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Validated, derived sizes of one configuration.
+struct Dims {
+  int64_t T;
+  int d, N, k, f, fs, C, align, elem;
+  bool bf16;
+  int64_t max_rows;    // rows of xp / h / out buffers
+  int64_t max_count;   // upper bound of one expert's kept rows: min(C, T)
+};
+
+// C = ceil(cf * T * k / N) evaluated exactly on the double cf = m * 2^e.
+moe_status_t exact_capacity(double cf, int64_t T, int k, int N, int32_t* out) {
+  if (!std::isfinite(cf) || cf < 0.0) return MOE_ERR_INVALID_ARG;
+  using u128 = unsigned __int128;
+  if (cf == 0.0 || T == 0) {
+    *out = 0;
+    return MOE_OK;
+  }
+  int ex = 0;
+  const double fr = std::frexp(cf, &ex);                       // cf = fr * 2^ex, fr in [0.5, 1)
+  const uint64_t m = static_cast<uint64_t>(std::ldexp(fr, 53));  // exact 53-bit integer
+  const int e = ex - 53;                                       // cf = m * 2^e
+  const u128 P = static_cast<u128>(m) * static_cast<u128>(T) * static_cast<u128>(k);
+  u128 c;
+  if (e >= 0) {
+    if (e > 40) return MOE_ERR_INVALID_ARG;                    // >= 2^40 / 256: beyond int32
+    const u128 num = P << e;
+    c = (num + static_cast<u128>(N) - 1) / static_cast<u128>(N);
+  } else if (-e > 110) {
+    c = 1;                                                     // 0 < value < 1
+  } else {
+    const u128 den = static_cast<u128>(N) << (-e);
+    c = (P + den - 1) / den;
+  }
+  if (c > static_cast<u128>(INT32_MAX)) return MOE_ERR_INVALID_ARG;
+  *out = static_cast<int32_t>(c);
+  return MOE_OK;
+}
+
+moe_status_t derive(const moe_config_t* cfg, Dims* D) {
+  if (cfg == nullptr) return MOE_ERR_INVALID_ARG;
+  if (cfg->T < 0 || cfg->d < 1 || cfg->N < 1 || cfg->k < 1 || cfg->f < 1 || cfg->f_shared < 0 ||
+      cfg->seg_align < 0)
+    return MOE_ERR_INVALID_ARG;
+  if (cfg->k > cfg->N) return MOE_ERR_INVALID_ARG;
+  if (cfg->act_dtype != MOE_F32 && cfg->act_dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+  if (cfg->N > 256 || cfg->k > 32 || cfg->seg_align > 4096) return MOE_ERR_UNSUPPORTED;
+  if (cfg->T * static_cast<int64_t>(cfg->k) >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED;
+  D->T = cfg->T;
+  D->d = cfg->d;
+  D->N = cfg->N;
+  D->k = cfg->k;
+  D->f = cfg->f;
+  D->fs = cfg->f_shared;
+  D->bf16 = cfg->act_dtype == MOE_BF16;
+  D->elem = D->bf16 ? 2 : 4;
+  D->align = cfg->seg_align == 0 ? 128 : cfg->seg_align;
+  if (D->bf16) {
+    if (D->d % 64 || D->f % 64 || D->fs % 64) return MOE_ERR_UNSUPPORTED;
+  } else {
+    if (D->d % 4) return MOE_ERR_UNSUPPORTED;  // rows are moved as 16-byte vectors
+  }
+  if (cfg->capacity >= 0) {
+    D->C = cfg->capacity;
+  } else {
+    moe_status_t s = exact_capacity(cfg->capacity_factor, cfg->T, cfg->k, cfg->N, &D->C);
+    if (s != MOE_OK) return s;
+  }
+  D->max_count = std::min<int64_t>(D->C, D->T);
+  const int64_t rows = std::min<int64_t>(D->T * D->k, static_cast<int64_t>(D->N) * D->max_count);
+  D->max_rows = rows + static_cast<int64_t>(D->N) * (D->align - 1);
+  if (D->max_rows >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+struct Layout {
+  size_t flags, rhist, rz, dmask, dbase, dcounts, dticket, op_end;
+  size_t idx, w, row_map, seg_off, seg_count, xp, h, hs, sh, layer_end;
+};
+
+Layout layout(const Dims& D) {
+  Layout L{};
+  const int64_t rb = (D.T + route_bt(route_np(D.N)) - 1) / route_bt(route_np(D.N));
+  const int64_t db = (D.T + kDispatchTokens - 1) / kDispatchTokens;
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o = round_up(o + bytes, kAlign);
+    return at;
+  };
+  L.flags = take(kAlign);
+  L.rhist = take(sizeof(int32_t) * rb * D.N);
+  L.rz = take(sizeof(float) * rb * D.N);
+  L.dmask = take(sizeof(uint32_t) * db * D.N);
+  L.dbase = take(sizeof(int32_t) * db * D.N);
+  L.dcounts = take(sizeof(int32_t) * D.N);
+  L.dticket = take(sizeof(uint32_t));
+  L.op_end = o;
+  L.idx = take(sizeof(int32_t) * D.T * D.k);
+  L.w = take(sizeof(float) * D.T * D.k);
+  L.row_map = take(sizeof(int32_t) * D.T * D.k);
+  L.seg_off = take(sizeof(int32_t) * (D.N + 1));
+  L.seg_count = take(sizeof(int32_t) * D.N);
+  L.xp = take(static_cast<size_t>(D.elem) * D.max_rows * D.d);  // permuted rows, then expert outputs
+  L.h = take(static_cast<size_t>(D.elem) * D.max_rows * D.f);
+  L.hs = take(static_cast<size_t>(D.elem) * (D.fs ? D.T * D.fs : 0));
+  L.sh = take(static_cast<size_t>(D.elem) * (D.fs ? D.T * D.d : 0));
+  L.layer_end = o;
+  return L;
+}
+
+template <typename P>
+P at(void* ws, size_t off) {
+  return reinterpret_cast<P>(static_cast<uint8_t*>(ws) + off);
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+moe_status_t check_ws(void* ws, size_t ws_bytes, size_t need) {
+  if (ws == nullptr || ws_bytes < need) return MOE_ERR_WORKSPACE;
+  if (!aligned16(ws)) return MOE_ERR_MISALIGNED;
+  return MOE_OK;
+}
+
+bool route_stats_requested(const moe_stats_t* s) {
+  return s != nullptr && (s->y_frac || s->z_mean || s->l_aux_p3 || s->l_aux_switch || s->counts);
+}
+
+moe_status_t do_route(const Dims& D, const void* x, const float* w_router, const float* bias,
+                      const float* logits_in, float* logits_out, int32_t* topk_idx, float* topk_w,
+                      const moe_stats_t* stats, void* ws, cudaStream_t st) {
+  const Layout L = layout(D);
+  cudaError_t e = cudaMemsetAsync(at<uint32_t*>(ws, L.flags), 0, sizeof(uint32_t), st);
+  if (e != cudaSuccess) return cuda_status(e);
+  RouteArgs a{};
+  a.T = D.T;
+  a.d = D.d;
+  a.N = D.N;
+  a.k = D.k;
+  a.x_is_bf16 = D.bf16 ? 1 : 0;
+  a.x = x;
+  a.w_router = w_router;
+  a.bias = bias;
+  a.logits_in = logits_in;
+  a.logits_out = logits_out;
+  a.topk_idx = topk_idx;
+  a.topk_w = topk_w;
+  a.hist = at<int32_t*>(ws, L.rhist);
+  a.zpart = at<float*>(ws, L.rz);
+  a.flags = at<uint32_t*>(ws, L.flags);
+  e = launch_route(a, st);
+  if (e != cudaSuccess) return cuda_status(e);
+  if (route_stats_requested(stats)) {
+    RouteStatsArgs s{};
+    s.T = D.T;
+    s.N = D.N;
+    s.k = D.k;
+    s.blocks = static_cast<int>((D.T + route_bt(route_np(D.N)) - 1) / route_bt(route_np(D.N)));
+    s.hist = a.hist;
+    s.zpart = a.zpart;
+    s.stats = *stats;
+    e = launch_route_stats(s, st);
+    if (e != cudaSuccess) return cuda_status(e);
+  }
+  return MOE_OK;
+}
+
+moe_status_t do_dispatch(const Dims& D, const void* x, const int32_t* topk_idx, int32_t* row_map,
+                         int32_t* seg_off, int32_t* seg_count, void* xp, const moe_stats_t* stats,
+                         void* ws, cudaStream_t st) {
+  const Layout L = layout(D);
+  if (D.T == 0) {
+    cudaError_t e = cudaMemsetAsync(seg_off, 0, sizeof(int32_t) * (D.N + 1), st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(seg_count, 0, sizeof(int32_t) * D.N, st);
+    if (e == cudaSuccess && stats && stats->counts) e = cudaMemsetAsync(stats->counts, 0, 4 * D.N, st);
+    if (e == cudaSuccess && stats && stats->kept) e = cudaMemsetAsync(stats->kept, 0, 4 * D.N, st);
+    if (e == cudaSuccess && stats && stats->num_dropped) e = cudaMemsetAsync(stats->num_dropped, 0, 4, st);
+    return cuda_status(e);
+  }
+  DispatchArgs a{};
+  a.T = D.T;
+  a.d = D.d;
+  a.N = D.N;
+  a.k = D.k;
+  a.capacity = D.C;
+  a.align = D.align;
+  a.elem_bytes = D.elem;
+  a.x = x;
+  a.topk_idx = topk_idx;
+  a.row_map = row_map;
+  a.seg_off = seg_off;
+  a.seg_count = seg_count;
+  a.xp = xp;
+  a.mask = at<uint32_t*>(ws, L.dmask);
+  a.base = at<int32_t*>(ws, L.dbase);
+  a.counts = at<int32_t*>(ws, L.dcounts);
+  a.ticket = at<uint32_t*>(ws, L.dticket);
+  if (stats) a.stats = *stats;
+  a.flags = at<uint32_t*>(ws, L.flags);
+  return cuda_status(launch_dispatch(a, st));
+}
+
+moe_status_t do_ffn(const Dims& D, const void* a_rows, const int32_t* seg_off, const int32_t* seg_count,
+                    const void* w1, const void* w3, const void* w2, int f, bool dense, void* h, void* out,
+                    void* ws, cudaStream_t st) {
+  const Layout L = layout(D);
+  FfnArgs a{};
+  a.G = dense ? 1 : D.N;
+  a.dense_rows = dense ? static_cast<int>(D.T) : 0;
+  a.max_count = dense ? static_cast<int>(D.T) : static_cast<int>(D.max_count);
+  a.max_rows = dense ? D.T : D.max_rows;
+  a.d = D.d;
+  a.f = f;
+  a.seg_off = dense ? nullptr : seg_off;
+  a.seg_count = dense ? nullptr : seg_count;
+  a.a = a_rows;
+  a.w1 = w1;
+  a.w3 = w3;
+  a.w2 = w2;
+  a.h = h;
+  a.out = out;
+  a.flags = at<uint32_t*>(ws, L.flags);
+  if (D.T == 0) return MOE_OK;
+  return cuda_status(D.bf16 ? launch_ffn_bf16(a, st) : launch_ffn_f32(a, st));
+}
+
+moe_status_t do_combine(const Dims& D, const void* out_rows, const int32_t* row_map, const float* topk_w,
+                        const void* shared_out, void* y, cudaStream_t st) {
+  CombineArgs a{};
+  a.T = D.T;
+  a.d = D.d;
+  a.k = D.k;
+  a.is_bf16 = D.bf16 ? 1 : 0;
+  a.out_rows = out_rows;
+  a.row_map = row_map;
+  a.topk_w = topk_w;
+  a.shared_out = shared_out;
+  a.y = y;
+  return cuda_status(launch_combine(a, st));
+}
+
+bool ffn_weights_ok(const moe_weights_t* w) {
+  return w != nullptr && w->w1 && w->w3 && w->w2 && aligned16(w->w1) && aligned16(w->w3) && aligned16(w->w2);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_string(moe_status_t s) {
+  switch (s) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+    case MOE_ERR_MISALIGNED: return "MOE_ERR_MISALIGNED";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_NONFINITE: return "MOE_ERR_NONFINITE";
+    case MOE_ERR_DEVICE: return "MOE_ERR_DEVICE";
+  }
+  return "MOE_ERR_UNKNOWN";
+}
+
+const char* moe_last_cuda_error(void) { return g_last_cuda_error; }
+
+const char* moe_version(void) { return "moe-b200 0.1 (sm_100a)"; }
+
+moe_status_t moe_capacity(const moe_config_t* cfg, int32_t* capacity) {
+  if (cfg == nullptr || capacity == nullptr) return MOE_ERR_INVALID_ARG;
+  if (cfg->T < 0 || cfg->N < 1 || cfg->k < 1) return MOE_ERR_INVALID_ARG;
+  if (cfg->capacity >= 0) {
+    *capacity = cfg->capacity;
+    return MOE_OK;
+  }
+  return exact_capacity(cfg->capacity_factor, cfg->T, cfg->k, cfg->N, capacity);
+}
+
+moe_status_t moe_workspace_size(const moe_config_t* cfg, size_t* layer_bytes, size_t* op_bytes,
+                                int64_t* max_rows) {
+  Dims D;
+  moe_status_t s = derive(cfg, &D);
+  if (s != MOE_OK) return s;
+  const Layout L = layout(D);
+  if (layer_bytes) *layer_bytes = L.layer_end;
+  if (op_bytes) *op_bytes = L.op_end;
+  if (max_rows) *max_rows = D.max_rows;
+  return MOE_OK;
+}
+
+moe_status_t moe_route(const moe_config_t* cfg, const void* x, const float* w_router, const float* router_bias,
+                       float* logits_out, int32_t* topk_idx, float* topk_w, moe_stats_t* stats, void* ws,
+                       size_t ws_bytes, moe_stream_t stream) {
+  Dims D;
+  moe_status_t s = derive(cfg, &D);
+  if (s != MOE_OK) return s;
+  if (D.T > 0 && (x == nullptr || w_router == nullptr || topk_idx == nullptr || topk_w == nullptr))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x)) return MOE_ERR_MISALIGNED;
+  if ((s = check_ws(ws, ws_bytes, layout(D).op_end)) != MOE_OK) return s;
+  return do_route(D, x, w_router, router_bias, nullptr, logits_out, topk_idx, topk_w, stats, ws,
+                  reinterpret_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_route_from_logits(const moe_config_t* cfg, const float* logits, int32_t* topk_idx, float* topk_w,
+                                   moe_stats_t* stats, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  Dims D;
+  moe_status_t s = derive(cfg, &D);
+  if (s != MOE_OK) return s;
+  if (D.T > 0 && (logits == nullptr || topk_idx == nullptr || topk_w == nullptr)) return MOE_ERR_INVALID_ARG;
+  if ((s = check_ws(ws, ws_bytes, layout(D).op_end)) != MOE_OK) return s;
+  return do_route(D, nullptr, nullptr, nullptr, logits, nullptr, topk_idx, topk_w, stats, ws,
+                  reinterpret_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* topk_idx, int32_t* row_map,
+                          int32_t* seg_off, int32_t* seg_count, void* xp, moe_stats_t* stats, void* ws,
+                          size_t ws_bytes, moe_stream_t stream) {
+  Dims D;
+  moe_status_t s = derive(cfg, &D);
+  if (s != MOE_OK) return s;
+  if (seg_off == nullptr || seg_count == nullptr) return MOE_ERR_INVALID_ARG;
+  if (D.T > 0 && (x == nullptr || topk_idx == nullptr || row_map == nullptr || xp == nullptr))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(xp)) return MOE_ERR_MISALIGNED;
+  if ((s = check_ws(ws, ws_bytes, layout(D).op_end)) != MOE_OK) return s;
+  return do_dispatch(D, x, topk_idx, row_map, seg_off, seg_count, xp, stats, ws,
+                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_expert_ffn(const moe_config_t* cfg, const void* xp, const int32_t* seg_off,
+                            const int32_t* seg_count, const moe_weights_t* weights, void* h, void* out_rows,
+                            void* ws, size_t ws_bytes, moe_stream_t stream) {
+  Dims D;
+  moe_status_t s = derive(cfg, &D);
+  if (s != MOE_OK) return s;
+  if (weights == nullptr || !weights->w1 || !weights->w3 || !weights->w2) return MOE_ERR_INVALID_ARG;
+  if (D.T > 0 && (xp == nullptr || seg_off == nullptr || seg_count == nullptr || h == nullptr || out_rows == nullptr))
+    return MOE_ERR_INVALID_ARG;
+  if (!ffn_weights_ok(weights) || !aligned16(xp) || !aligned16(h) || !aligned16(out_rows))
+    return MOE_ERR_MISALIGNED;
+  if ((s = check_ws(ws, ws_bytes, layout(D).op_end)) != MOE_OK) return s;
+  return do_ffn(D, xp, seg_off, seg_count, weights->w1, weights->w3, weights->w2, D.f, false, h, out_rows, ws,
+                reinterpret_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_shared_expert_ffn(const moe_config_t* cfg, const void* x, const moe_weights_t* weights,
+                                   void* h_shared, void* shared_out, void* ws, size_t ws_bytes,
+                                   moe_stream_t stream) {
+  Dims D;
+  moe_status_t s = derive(cfg, &D);
+  if (s != MOE_OK) return s;
+  if (D.fs == 0 || weights == nullptr || !weights->ws1 || !weights->ws3 || !weights->ws2) return MOE_ERR_INVALID_ARG;
+  if (D.T > 0 && (x == nullptr || h_shared == nullptr || shared_out == nullptr)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(weights->ws1) || !aligned16(weights->ws3) || !aligned16(weights->ws2) ||
+      !aligned16(h_shared) || !aligned16(shared_out))
+    return MOE_ERR_MISALIGNED;
+  if ((s = check_ws(ws, ws_bytes, layout(D).op_end)) != MOE_OK) return s;
+  return do_ffn(D, x, nullptr, nullptr, weights->ws1, weights->ws3, weights->ws2, D.fs, true, h_shared,
+                shared_out, ws, reinterpret_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_combine(const moe_config_t* cfg, const void* out_rows, const int32_t* row_map, const float* topk_w,
+                         const void* shared_out, void* y, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  Dims D;
+  moe_status_t s = derive(cfg, &D);
+  if (s != MOE_OK) return s;
+  if (D.T > 0 && (out_rows == nullptr || row_map == nullptr || topk_w == nullptr || y == nullptr))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(out_rows) || !aligned16(shared_out) || !aligned16(y)) return MOE_ERR_MISALIGNED;
+  if ((s = check_ws(ws, ws_bytes, layout(D).op_end)) != MOE_OK) return s;
+  return do_combine(D, out_rows, row_map, topk_w, shared_out, y, reinterpret_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_layer_fwd(const moe_config_t* cfg, const moe_weights_t* weights, const void* x, void* y,
+                           moe_stats_t* stats, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  Dims D;
+  moe_status_t s = derive(cfg, &D);
+  if (s != MOE_OK) return s;
+  if (weights == nullptr || weights->w_router == nullptr || !weights->w1 || !weights->w3 || !weights->w2 ||
+      (D.T > 0 && (x == nullptr || y == nullptr)))
+    return MOE_ERR_INVALID_ARG;
+  if (D.fs > 0 && (!weights->ws1 || !weights->ws3 || !weights->ws2)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(y) || !ffn_weights_ok(weights)) return MOE_ERR_MISALIGNED;
+  if (D.fs > 0 && (!aligned16(weights->ws1) || !aligned16(weights->ws3) || !aligned16(weights->ws2)))
+    return MOE_ERR_MISALIGNED;
+  const Layout L = layout(D);
+  if ((s = check_ws(ws, ws_bytes, L.layer_end)) != MOE_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+
+  int32_t* idx = at<int32_t*>(ws, L.idx);
+  float* w = at<float*>(ws, L.w);
+  int32_t* row_map = at<int32_t*>(ws, L.row_map);
+  int32_t* seg_off = at<int32_t*>(ws, L.seg_off);
+  int32_t* seg_count = at<int32_t*>(ws, L.seg_count);
+  void* xp = at<void*>(ws, L.xp);
+  void* h = at<void*>(ws, L.h);
+  void* out_rows = xp;  // the permuted rows are dead once GEMM1 has read them
+  void* shared_out = D.fs ? at<void*>(ws, L.sh) : nullptr;
+
+  if ((s = do_route(D, x, weights->w_router, weights->router_bias, nullptr, nullptr, idx, w, stats, ws, st)) !=
+      MOE_OK)
+    return s;
+  if ((s = do_dispatch(D, x, idx, row_map, seg_off, seg_count, xp, stats, ws, st)) != MOE_OK) return s;
+  if ((s = do_ffn(D, xp, seg_off, seg_count, weights->w1, weights->w3, weights->w2, D.f, false, h, out_rows, ws,
+                  st)) != MOE_OK)
+    return s;
+  if (D.fs > 0 && (s = do_ffn(D, x, nullptr, nullptr, weights->ws1, weights->ws3, weights->ws2, D.fs, true,
+                              at<void*>(ws, L.hs), shared_out, ws, st)) != MOE_OK)
+    return s;
+  return do_combine(D, out_rows, row_map, w, shared_out, y, st);
+}
+
+moe_status_t moe_read_flags(const void* ws, size_t ws_bytes, uint32_t* flags, moe_stream_t stream) {
+  if (ws == nullptr || ws_bytes < sizeof(uint32_t) || flags == nullptr) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t v = 0;
+  cudaError_t e = cudaMemcpyAsync(&v, ws, sizeof(uint32_t), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_status(e);
+  *flags = v;
+  if (v & MOE_FLAG_NONFINITE_LOGITS) return MOE_ERR_NONFINITE;
+  if (v & (MOE_FLAG_BAD_EXPERT_INDEX | MOE_FLAG_WAIT_TIMEOUT)) return MOE_ERR_DEVICE;
+  return MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,274 @@
+"""Thin ctypes binding of libmoe.so (include/moe.h).
+
+Argument marshalling only: every step of the MoE layer runs in the library's
+CUDA kernels.  PyTorch provides device memory and the current stream.  The
+module raises ImportError when the shared library is missing: there is no
+fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmoe.so")
+HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "moe.h")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"libmoe.so is not built ({LIB_PATH}); run "
+                      "`python -m expert_router_gemm_b200.build`")
+_lib = ctypes.CDLL(LIB_PATH)
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_MISALIGNED = 0, 1, 2, 3
+MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_NONFINITE, MOE_ERR_DEVICE = 4, 5, 6, 7
+MOE_F32, MOE_BF16 = 0, 1
+MOE_FLAG_NONFINITE_LOGITS, MOE_FLAG_BAD_EXPERT_INDEX, MOE_FLAG_WAIT_TIMEOUT = 1, 2, 4
+
+
+class moe_config_t(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int64), ("d", ctypes.c_int32), ("N", ctypes.c_int32),
+                ("k", ctypes.c_int32), ("f", ctypes.c_int32), ("f_shared", ctypes.c_int32),
+                ("capacity_factor", ctypes.c_double), ("capacity", ctypes.c_int32),
+                ("act_dtype", ctypes.c_int), ("seg_align", ctypes.c_int32)]
+
+
+class moe_weights_t(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("w_router", "router_bias", "w1", "w3", "w2", "ws1", "ws3", "ws2")]
+
+
+class moe_stats_t(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("y_frac", "z_mean", "l_aux_p3", "l_aux_switch", "counts", "kept", "num_dropped")]
+
+
+_P = ctypes.c_void_p
+_SZ = ctypes.c_size_t
+_PROTOS = {
+    "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "moe_last_cuda_error": (ctypes.c_char_p, []),
+    "moe_version": (ctypes.c_char_p, []),
+    "moe_capacity": (ctypes.c_int, [ctypes.POINTER(moe_config_t), ctypes.POINTER(ctypes.c_int32)]),
+    "moe_workspace_size": (ctypes.c_int, [ctypes.POINTER(moe_config_t), ctypes.POINTER(_SZ),
+                                          ctypes.POINTER(_SZ), ctypes.POINTER(ctypes.c_int64)]),
+    "moe_route": (ctypes.c_int, [ctypes.POINTER(moe_config_t), _P, _P, _P, _P, _P, _P,
+                                 ctypes.POINTER(moe_stats_t), _P, _SZ, _P]),
+    "moe_route_from_logits": (ctypes.c_int, [ctypes.POINTER(moe_config_t), _P, _P, _P,
+                                             ctypes.POINTER(moe_stats_t), _P, _SZ, _P]),
+    "moe_dispatch": (ctypes.c_int, [ctypes.POINTER(moe_config_t), _P, _P, _P, _P, _P, _P,
+                                    ctypes.POINTER(moe_stats_t), _P, _SZ, _P]),
+    "moe_expert_ffn": (ctypes.c_int, [ctypes.POINTER(moe_config_t), _P, _P, _P,
+                                      ctypes.POINTER(moe_weights_t), _P, _P, _P, _SZ, _P]),
+    "moe_shared_expert_ffn": (ctypes.c_int, [ctypes.POINTER(moe_config_t), _P,
+                                             ctypes.POINTER(moe_weights_t), _P, _P, _P, _SZ, _P]),
+    "moe_combine": (ctypes.c_int, [ctypes.POINTER(moe_config_t), _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "moe_layer_fwd": (ctypes.c_int, [ctypes.POINTER(moe_config_t), ctypes.POINTER(moe_weights_t),
+                                     _P, _P, ctypes.POINTER(moe_stats_t), _P, _SZ, _P]),
+    "moe_read_flags": (ctypes.c_int, [_P, _SZ, ctypes.POINTER(ctypes.c_uint32), _P]),
+}
+for _name, (_res, _args) in _PROTOS.items():
+    _fn = getattr(_lib, _name)
+    _fn.restype = _res
+    _fn.argtypes = _args
+
+
+def header_functions():
+    """Names of the functions declared in include/moe.h."""
+    with open(HEADER_PATH) as fh:
+        text = fh.read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*(moe_[a-z_0-9]+)\s*\(",
+                                 text, flags=re.M)))
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        msg = _lib.moe_status_string(status).decode()
+        if status == MOE_ERR_CUDA:
+            msg += f" ({_lib.moe_last_cuda_error().decode()})"
+        super().__init__(f"{where}: {msg}")
+        self.status = status
+
+
+def _check(status: int, where: str):
+    if status != MOE_OK:
+        raise MoeError(status, where)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        return int(t)
+    if t.numel() and not t.is_contiguous():
+        raise ValueError("tensors passed to libmoe must be contiguous")
+    return t.data_ptr() or None
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        if not torch.cuda.is_available():
+            return None
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def make_config(T: int, d: int, N: int, k: int, f: int, f_shared: int = 0,
+                capacity_factor: float = 1.0, capacity: int = -1, dtype: str = "bf16",
+                seg_align: int = 0) -> moe_config_t:
+    return moe_config_t(T, d, N, k, f, f_shared, capacity_factor, capacity,
+                        MOE_BF16 if dtype == "bf16" else MOE_F32, seg_align)
+
+
+def config_from_workload(w, T: Optional[int] = None, **over) -> moe_config_t:
+    kw = dict(T=w.T if T is None else T, d=w.d, N=w.N, k=w.k, f=w.f, f_shared=w.f_shared,
+              capacity_factor=w.capacity_factor, dtype=w.dtype)
+    kw.update(over)
+    return make_config(**kw)
+
+
+def make_weights(w_router, router_bias=None, w1=None, w3=None, w2=None, ws1=None, ws3=None,
+                 ws2=None) -> moe_weights_t:
+    return moe_weights_t(*[_ptr(t) for t in (w_router, router_bias, w1, w3, w2, ws1, ws3, ws2)])
+
+
+def make_stats(y_frac=None, z_mean=None, l_aux_p3=None, l_aux_switch=None, counts=None,
+               kept=None, num_dropped=None) -> moe_stats_t:
+    return moe_stats_t(*[_ptr(t) for t in (y_frac, z_mean, l_aux_p3, l_aux_switch, counts, kept,
+                                            num_dropped)])
+
+
+# ---------------------------------------------------------------- the C-ABI calls
+def moe_version() -> str:
+    return _lib.moe_version().decode()
+
+
+def moe_status_string(status: int) -> str:
+    return _lib.moe_status_string(status).decode()
+
+
+def moe_capacity(cfg: moe_config_t) -> int:
+    c = ctypes.c_int32()
+    _check(_lib.moe_capacity(ctypes.byref(cfg), ctypes.byref(c)), "moe_capacity")
+    return c.value
+
+
+def moe_workspace_size(cfg: moe_config_t):
+    """-> (layer_bytes, op_bytes, max_rows)"""
+    lb, ob, mr = _SZ(), _SZ(), ctypes.c_int64()
+    _check(_lib.moe_workspace_size(ctypes.byref(cfg), ctypes.byref(lb), ctypes.byref(ob),
+                                   ctypes.byref(mr)), "moe_workspace_size")
+    return lb.value, ob.value, mr.value
+
+
+def _stats_ref(stats: Optional[moe_stats_t]):
+    return ctypes.byref(stats) if stats is not None else None
+
+
+def moe_route(cfg, x, w_router, router_bias, logits_out, topk_idx, topk_w, stats, ws,
+              stream=None):
+    _check(_lib.moe_route(ctypes.byref(cfg), _ptr(x), _ptr(w_router), _ptr(router_bias),
+                          _ptr(logits_out), _ptr(topk_idx), _ptr(topk_w), _stats_ref(stats),
+                          _ptr(ws), ws.numel() if ws is not None else 0, _stream(stream)),
+           "moe_route")
+
+
+def moe_route_from_logits(cfg, logits, topk_idx, topk_w, stats, ws, stream=None):
+    _check(_lib.moe_route_from_logits(ctypes.byref(cfg), _ptr(logits), _ptr(topk_idx),
+                                      _ptr(topk_w), _stats_ref(stats), _ptr(ws),
+                                      ws.numel() if ws is not None else 0, _stream(stream)),
+           "moe_route_from_logits")
+
+
+def moe_dispatch(cfg, x, topk_idx, row_map, seg_off, seg_count, xp, stats, ws, stream=None):
+    _check(_lib.moe_dispatch(ctypes.byref(cfg), _ptr(x), _ptr(topk_idx), _ptr(row_map),
+                             _ptr(seg_off), _ptr(seg_count), _ptr(xp), _stats_ref(stats),
+                             _ptr(ws), ws.numel() if ws is not None else 0, _stream(stream)),
+           "moe_dispatch")
+
+
+def moe_expert_ffn(cfg, xp, seg_off, seg_count, weights: moe_weights_t, h, out_rows, ws,
+                   stream=None):
+    _check(_lib.moe_expert_ffn(ctypes.byref(cfg), _ptr(xp), _ptr(seg_off), _ptr(seg_count),
+                               ctypes.byref(weights), _ptr(h), _ptr(out_rows), _ptr(ws),
+                               ws.numel() if ws is not None else 0, _stream(stream)),
+           "moe_expert_ffn")
+
+
+def moe_shared_expert_ffn(cfg, x, weights: moe_weights_t, h_shared, shared_out, ws,
+                          stream=None):
+    _check(_lib.moe_shared_expert_ffn(ctypes.byref(cfg), _ptr(x), ctypes.byref(weights),
+                                      _ptr(h_shared), _ptr(shared_out), _ptr(ws),
+                                      ws.numel() if ws is not None else 0, _stream(stream)),
+           "moe_shared_expert_ffn")
+
+
+def moe_combine(cfg, out_rows, row_map, topk_w, shared_out, y, ws, stream=None):
+    _check(_lib.moe_combine(ctypes.byref(cfg), _ptr(out_rows), _ptr(row_map), _ptr(topk_w),
+                            _ptr(shared_out), _ptr(y), _ptr(ws),
+                            ws.numel() if ws is not None else 0, _stream(stream)),
+           "moe_combine")
+
+
+def moe_layer_fwd(cfg, weights: moe_weights_t, x, y, stats, ws, stream=None):
+    _check(_lib.moe_layer_fwd(ctypes.byref(cfg), ctypes.byref(weights), _ptr(x), _ptr(y),
+                              _stats_ref(stats), _ptr(ws), ws.numel() if ws is not None else 0,
+                              _stream(stream)), "moe_layer_fwd")
+
+
+def moe_read_flags(ws, stream=None) -> int:
+    """Waits for the stream; returns the flags word (raises on a set bit)."""
+    v = ctypes.c_uint32()
+    st = _lib.moe_read_flags(_ptr(ws), ws.numel(), ctypes.byref(v), _stream(stream))
+    if st not in (MOE_OK, MOE_ERR_NONFINITE, MOE_ERR_DEVICE):
+        _check(st, "moe_read_flags")
+    return v.value
+
+
+def raw_call(name: str, *args) -> int:
+    """Call a C-ABI function with raw ctypes arguments; returns its status (tests)."""
+    return getattr(_lib, name)(*args)
+
+
+# ---------------------------------------------------------------- conveniences
+@dataclass
+class DeviceLayer:
+    """Device copies of one layer's inputs (torch tensors on cuda)."""
+    cfg: moe_config_t
+    x: torch.Tensor
+    w_router: torch.Tensor
+    bias: Optional[torch.Tensor]
+    w1: torch.Tensor
+    w3: torch.Tensor
+    w2: torch.Tensor
+    ws1: Optional[torch.Tensor] = None
+    ws3: Optional[torch.Tensor] = None
+    ws2: Optional[torch.Tensor] = None
+
+    def weights(self) -> moe_weights_t:
+        return make_weights(self.w_router, self.bias, self.w1, self.w3, self.w2,
+                            self.ws1, self.ws3, self.ws2)
+
+
+def to_device(inputs, cfg: moe_config_t, device="cuda") -> DeviceLayer:
+    """Upload host arrays (numpy; bf16 as uint16 bits) to device tensors."""
+    import numpy as np
+
+    def up(a):
+        if a is None:
+            return None
+        a = np.ascontiguousarray(a)
+        t = torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a)
+        return t.to(device)
+
+    return DeviceLayer(cfg, up(inputs.x), up(inputs.w_router), up(inputs.bias), up(inputs.w1),
+                       up(inputs.w3), up(inputs.w2), up(inputs.ws1), up(inputs.ws3),
+                       up(inputs.ws2))
+
+
+def act_dtype(cfg: moe_config_t):
+    return torch.int16 if cfg.act_dtype == MOE_BF16 else torch.float32

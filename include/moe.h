@@ -1,0 +1,255 @@
+/*
+ * moe.h - C ABI of libmoe.so: the forward pass of one Mixture-of-Experts layer
+ * on one NVIDIA B200 (sm_100a).
+ *
+ * The pass, in the notation of "MoE 训练加速实战：DeepEP + Grouped GeMM +
+ * Aux-Loss-Free" §2.2 "Router 数学" (N experts, token x in R^d, W_r in R^{d x N}):
+ *
+ *   g(x)   = x W_r (+ b)                               router logits, fp32
+ *   s(x)   = softmax(g(x))                             fp32, max-subtracted
+ *   y      = sum_{i in top-k(g)} s_i / (sum_{j in top-k} s_j) * Expert_i(x)
+ *
+ * with each expert a SwiGLU FFN  Expert_i(x) = (silu(x W1_i) * (x W3_i)) W2_i,
+ * a per-expert capacity C = ceil(capacity_factor * T * k / N) whose overflow is
+ * dropped in token order ("负载均衡策略：MoE训练稳定性保障", section "专家容量裁剪"),
+ * the kept assignments permuted into expert-contiguous rows (the single-GPU
+ * counterpart of the dispatch all-to-all, §3.2 of the first page), the experts
+ * run as one grouped GEMM (§4.2 "数学等价性"), and the load-balance statistics of
+ * L_aux = (T/N) sum_i y_i z_i ("负载均衡策略", section "辅助损失函数").
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every tensor pointer is a DEVICE pointer on the current CUDA device, owned
+ *    by the caller.  The library never allocates, frees or synchronises: work is
+ *    enqueued on `stream` (NULL = the legacy default stream) in call order.
+ *    The only exception is moe_read_flags(), which waits for the stream.
+ *  - Tensors are dense, row-major, with no padding between rows.
+ *  - "act" tensors (x, xp, h, out_rows, y, shared_out, expert weights) have the
+ *    config's act_dtype: MOE_F32 (float) or MOE_BF16 (uint16 bf16 bit patterns).
+ *    The router weight, bias, logits and routing weights are always fp32.
+ *  - Each call validates its arguments on the host before it launches anything
+ *    and returns a moe_status_t.  No call traps, aborts or throws.  A failed
+ *    launch returns MOE_ERR_CUDA (the CUDA error string is available from
+ *    moe_last_cuda_error()).  Conditions only the GPU can see (non-finite
+ *    logits, an out-of-range expert index, a pipeline wait that ran out) set
+ *    bits in the flags word at the start of the workspace; read them with
+ *    moe_read_flags().
+ *  - Buffers that kernels read or write with 16-byte vectors (x, xp, h,
+ *    out_rows, y, shared_out, weights) must be 16-byte aligned
+ *    (MOE_ERR_MISALIGNED).
+ *  - bf16 layers need d % 64 == 0 and f % 64 == 0 (and f_shared % 64 == 0):
+ *    the expert GEMMs step through K in 64-element slabs (MOE_ERR_UNSUPPORTED).
+ *  - Limits: 1 <= N <= 256, 1 <= k <= min(N, 32), T * k < 2^31, T >= 0 (T = 0
+ *    is a valid empty batch: outputs are left untouched, statistics are zeroed).
+ *  - Results are deterministic: the same inputs give the same bytes.
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream (cudaStream_t / CUstream); NULL is the legacy default stream. */
+typedef struct CUstream_st* moe_stream_t;
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,   /* NULL where required, bad sizes, k > N, ... */
+  MOE_ERR_UNSUPPORTED = 2,   /* valid but outside the supported shapes */
+  MOE_ERR_MISALIGNED = 3,    /* a vector-accessed buffer is not 16-byte aligned */
+  MOE_ERR_WORKSPACE = 4,     /* workspace NULL or smaller than the query says */
+  MOE_ERR_CUDA = 5,          /* a CUDA runtime call or launch failed */
+  MOE_ERR_NONFINITE = 6,     /* (from moe_read_flags) non-finite router logits */
+  MOE_ERR_DEVICE = 7,        /* (from moe_read_flags) bad index / device wait ran out */
+} moe_status_t;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype_t;
+
+/* Bits of the device flags word (moe_read_flags). */
+#define MOE_FLAG_NONFINITE_LOGITS 0x1u  /* some router logit was NaN or +-Inf */
+#define MOE_FLAG_BAD_EXPERT_INDEX 0x2u  /* topk_idx outside [0,N) or repeated in a row */
+#define MOE_FLAG_WAIT_TIMEOUT     0x4u  /* a GEMM pipeline wait exceeded its bound */
+
+typedef struct {
+  int64_t T;               /* tokens in the batch */
+  int32_t d;               /* model dimension */
+  int32_t N;               /* routed experts */
+  int32_t k;               /* experts per token (top-k) */
+  int32_t f;               /* SwiGLU hidden size of a routed expert */
+  int32_t f_shared;        /* hidden size of the shared expert; 0 = no shared expert */
+  double capacity_factor;  /* C = ceil(capacity_factor * T * k / N), exact on this double */
+  int32_t capacity;        /* >= 0: use this C instead of the formula; < 0: derive */
+  moe_dtype_t act_dtype;   /* MOE_F32 or MOE_BF16 */
+  int32_t seg_align;       /* expert segments start at multiples of this many rows; 0 -> 128 */
+} moe_config_t;
+
+typedef struct {
+  const float* w_router;     /* [d, N] fp32 */
+  const float* router_bias;  /* [N] fp32, added to the logits; NULL = none */
+  const void* w1;            /* [N][d][f] act: gate projection */
+  const void* w3;            /* [N][d][f] act: up projection */
+  const void* w2;            /* [N][f][d] act: down projection */
+  const void* ws1;           /* [d][f_shared] act, shared expert gate; NULL if f_shared == 0 */
+  const void* ws3;           /* [d][f_shared] act, shared expert up */
+  const void* ws2;           /* [f_shared][d] act, shared expert down */
+} moe_weights_t;
+
+/* Load-balance and capacity statistics.  Device pointers; each may be NULL. */
+typedef struct {
+  float* y_frac;        /* [N] y_i: share of the T*k top-k selections (before the drop) */
+  float* z_mean;        /* [N] z_i: mean softmax score over the T tokens */
+  float* l_aux_p3;      /* [1] (T/N) * sum_i y_i z_i  ("负载均衡策略", "辅助损失函数") */
+  float* l_aux_switch;  /* [1] N * sum_i y_i z_i      (Switch form, §5.2 of the first page) */
+  int32_t* counts;      /* [N] top-k selections per expert before the drop */
+  int32_t* kept;        /* [N] min(counts, C) */
+  int32_t* num_dropped; /* [1] sum_i (counts_i - kept_i) */
+} moe_stats_t;
+
+/* Human-readable name of a status. Never NULL. */
+const char* moe_status_string(moe_status_t status);
+
+/* Text of the last CUDA error seen by this thread ("" if none). Never NULL. */
+const char* moe_last_cuda_error(void);
+
+/* Library version string. */
+const char* moe_version(void);
+
+/*
+ * moe_capacity - host-only: the per-expert capacity C of `cfg`.
+ * "负载均衡策略：MoE训练稳定性保障", section "专家容量裁剪": capacity_factor times
+ * the ideal share, e.g. 1024 tokens / 8 experts * 1.25 = 160; with k experts per
+ * token the ideal share is T*k/N.  If cfg->capacity >= 0 that value is returned.
+ * The product is evaluated exactly (128-bit integers) on the given double.
+ * Errors: MOE_ERR_INVALID_ARG for NULL, T < 0, N < 1, k < 1, capacity_factor
+ * not finite or < 0, or a capacity above 2^31-1.
+ */
+moe_status_t moe_capacity(const moe_config_t* cfg, int32_t* capacity);
+
+/*
+ * moe_workspace_size - host-only sizes the caller must provide.
+ *   layer_bytes: workspace of moe_layer_fwd (routing arrays, the permuted rows,
+ *                the SwiGLU hidden rows and the expert outputs);
+ *   op_bytes:    workspace of the single-step entry points (moe_route,
+ *                moe_route_from_logits, moe_dispatch, moe_expert_ffn,
+ *                moe_shared_expert_ffn, moe_combine);
+ *   max_rows:    rows the caller must allocate for xp / h / out_rows:
+ *                min(T*k, N*min(C,T)) + N*(seg_align-1).
+ * Any output pointer may be NULL.  Errors as moe_capacity, plus the shape checks.
+ */
+moe_status_t moe_workspace_size(const moe_config_t* cfg, size_t* layer_bytes,
+                                size_t* op_bytes, int64_t* max_rows);
+
+/*
+ * moe_route - router GEMM, fp32 softmax, top-k and renormalised weights.
+ * "MoE 训练加速实战" §2.2 "Router 数学": g = x W_r, scores = softmax(g), the k
+ * largest g selected (ties: lower expert index first; slots in descending g),
+ * weight_j = s_{idx_j} / sum_{j'} s_{idx_j'}.
+ *   x          [T, d] act          input tokens (read)
+ *   w_router   [d, N] fp32, bias [N] fp32 or NULL
+ *   logits_out [T, N] fp32 or NULL: g including the bias
+ *   topk_idx   [T, k] int32 (written), topk_w [T, k] fp32 (written)
+ *   stats      may be NULL: fills y_frac, z_mean, l_aux_p3, l_aux_switch, counts
+ *   ws         op workspace (>= op_bytes); its flags word is cleared first.
+ * Non-finite logits raise MOE_FLAG_NONFINITE_LOGITS (read with moe_read_flags).
+ */
+moe_status_t moe_route(const moe_config_t* cfg, const void* x, const float* w_router,
+                       const float* router_bias, float* logits_out, int32_t* topk_idx,
+                       float* topk_w, moe_stats_t* stats, void* ws, size_t ws_bytes,
+                       moe_stream_t stream);
+
+/*
+ * moe_route_from_logits - the same softmax / top-k / weights / statistics as
+ * moe_route, starting from caller-supplied fp32 logits [T, N] (no GEMM).  This is
+ * the entry point on which routing is compared bit-for-bit with a reference.
+ */
+moe_status_t moe_route_from_logits(const moe_config_t* cfg, const float* logits,
+                                   int32_t* topk_idx, float* topk_w, moe_stats_t* stats,
+                                   void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * moe_dispatch - capacity clip and permutation into expert-contiguous rows.
+ * "负载均衡策略", section "专家容量裁剪" (at most C tokens per expert, the rest
+ * dropped) and "ETP专家并行加速MoE模型", section "动态路由下的高效通信" (tokens are
+ * re-shuffled to their experts).  Within expert e the assignments are ranked in
+ * token order; rank < C is kept.
+ *   x         [T, d] act (read)
+ *   topk_idx  [T, k] int32 in [0, N), distinct within a row (read)
+ *   row_map   [T, k] int32 (written): seg_off[e] + rank, or -1 if dropped
+ *   seg_off   [N+1] int32 (written): segment starts, multiples of seg_align;
+ *             seg_off[N] = rows in use
+ *   seg_count [N] int32 (written): kept rows of each expert = min(count, C)
+ *   xp        [max_rows, d] act (written): xp[row_map[t][j]] = x[t] bit for bit;
+ *             rows between segments are not written
+ *   stats     may be NULL: fills counts, kept, num_dropped
+ * An index outside [0, N) or repeated in a row raises MOE_FLAG_BAD_EXPERT_INDEX;
+ * that slot is dropped.
+ */
+moe_status_t moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* topk_idx,
+                          int32_t* row_map, int32_t* seg_off, int32_t* seg_count, void* xp,
+                          moe_stats_t* stats, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * moe_expert_ffn - all routed experts as one grouped GEMM pair, SwiGLU fused.
+ * "MoE 训练加速实战" §4.1-4.2: one kernel serves every expert, y_i = W_i x_i.
+ * For every expert e and row r in [seg_off[e], seg_off[e] + seg_count[e]):
+ *   h[r]        = silu(xp[r] W1_e) * (xp[r] W3_e)      (fp32 math, one rounding to act)
+ *   out_rows[r] = h[r] W2_e                            (fp32 accumulation)
+ *   xp, h, out_rows: [max_rows, d], [max_rows, f], [max_rows, d] act.
+ * Rows outside the segments are neither read for results nor written.
+ * bf16 runs on the tcgen05 tensor cores; fp32 runs on the CUDA cores.
+ */
+moe_status_t moe_expert_ffn(const moe_config_t* cfg, const void* xp, const int32_t* seg_off,
+                            const int32_t* seg_count, const moe_weights_t* weights, void* h,
+                            void* out_rows, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * moe_shared_expert_ffn - the always-on shared expert ("MoE 训练加速实战" §2.3
+ * spec table and §9.1: DeepSeek-V3 uses one) over all T tokens:
+ *   shared_out[t] = (silu(x[t] Ws1) * (x[t] Ws3)) Ws2
+ *   h_shared [T, f_shared] act scratch; shared_out [T, d] act.
+ * MOE_ERR_INVALID_ARG if cfg->f_shared == 0.
+ */
+moe_status_t moe_shared_expert_ffn(const moe_config_t* cfg, const void* x,
+                                   const moe_weights_t* weights, void* h_shared,
+                                   void* shared_out, void* ws, size_t ws_bytes,
+                                   moe_stream_t stream);
+
+/*
+ * moe_combine - weighted sum back to token order ("MoE 训练加速实战" §2.1,
+ * "权重加和"):  y[t] = sum_{j=0..k-1, row_map[t][j] >= 0} topk_w[t][j] *
+ * out_rows[row_map[t][j]]  (+ shared_out[t]), accumulated in fp32 in slot
+ * order, rounded once to act.  Dropped slots add nothing; the kept weights are
+ * not renormalised.  shared_out may be NULL.  y [T, d] act (written).
+ */
+moe_status_t moe_combine(const moe_config_t* cfg, const void* out_rows, const int32_t* row_map,
+                         const float* topk_w, const void* shared_out, void* y, void* ws,
+                         size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * moe_layer_fwd - the whole layer: route, dispatch, routed experts, shared
+ * expert (if cfg->f_shared > 0), combine.  x [T, d] act (read), y [T, d] act
+ * (written), stats may be NULL, ws >= layer_bytes of moe_workspace_size.  The
+ * permuted rows and the expert outputs share one workspace region.
+ */
+moe_status_t moe_layer_fwd(const moe_config_t* cfg, const moe_weights_t* weights,
+                           const void* x, void* y, moe_stats_t* stats, void* ws,
+                           size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * moe_read_flags - wait for `stream`, then copy the workspace's device flags
+ * word (MOE_FLAG_* bits, cleared by moe_route / moe_route_from_logits /
+ * moe_layer_fwd) to *flags.  Returns MOE_ERR_NONFINITE or MOE_ERR_DEVICE when a
+ * bit is set, MOE_OK otherwise.
+ */
+moe_status_t moe_read_flags(const void* ws, size_t ws_bytes, uint32_t* flags,
+                            moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H_ */

@@ -1,0 +1,108 @@
+"""GPU parity of the whole layer (routed experts on the tcgen05 grouped GEMM,
+shared expert, combine) against the fp64 oracle, at sizes the oracle finishes in
+seconds that still span several tiles and ragged tails.
+
+Tolerances (relative Frobenius error of the layer output): 1e-5 for the fp32
+layer and 2e-2 for bf16 compute with fp32 accumulation."""
+import numpy as np
+import pytest
+import torch
+
+from expert_router_gemm_b200 import configs, synth
+from expert_router_gemm_b200.configs import Workload
+from oracle import moe_oracle as orc
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+from expert_router_gemm_b200 import moe  # noqa: E402
+from tests import gpu_util as gu  # noqa: E402
+from tests.layer_check import compare_layer  # noqa: E402
+
+TOL_F32 = 1e-5
+TOL_BF16 = 2e-2
+
+SMALL = [
+    # ragged tiles: d = 320 leaves a 64-column tail in the down projection's
+    # 256-column tiles, f = 192 a 64-column tail in the 128-column SwiGLU tiles
+    Workload("ragged-bf16", T=700, d=320, N=8, k=2, f=192, capacity_factor=1.1),
+    Workload("finegrained-bf16", T=1024, d=512, N=128, k=8, f=256, capacity_factor=1.0),
+    Workload("shared-bf16", T=520, d=256, N=16, k=4, f=128, f_shared=192, capacity_factor=1.25),
+    Workload("skewed-bf16", T=2048, d=256, N=8, k=2, f=512, capacity_factor=1.25,
+             bias_pattern=configs.SKEW.bias_pattern, bias_beta_gamma=configs.SKEW_BETA_GAMMA),
+    Workload("topN-bf16", T=300, d=128, N=8, k=8, f=128, capacity_factor=1.0),
+    Workload("manytiles-bf16", T=1536, d=1024, N=4, k=2, f=1024, capacity_factor=1.0),
+]
+
+
+def _run(w: Workload, align=0):
+    inp = synth.make_inputs(w)
+    cfg = moe.config_from_workload(w, seg_align=align)
+    dl = moe.to_device(inp, cfg)
+    staged = gu.staged_layer(dl)
+    y, st, flags = gu.layer_fwd(dl)
+    assert flags == 0 and staged["flags"] == 0
+    return inp, staged, y, st
+
+
+def test_tiny_fp32_layer():
+    w = configs.TINY
+    inp, staged, y, st = _run(w)
+    np.testing.assert_array_equal(y, staged["y"])
+    rel, n, flips = compare_layer(inp, w, y, staged["idx"], staged["row_map"], staged["logits"],
+                                  tol=TOL_F32)
+    assert n == w.T - flips
+    ref = orc.layer_forward(inp.x, inp.w_router, inp.bias, inp.w1, inp.w3, inp.w2, k=w.k,
+                            capacity_factor=w.capacity_factor, bf16=False, tokens=[])
+    np.testing.assert_array_equal(st["kept"], ref.disp.kept)
+    np.testing.assert_allclose(st["z_mean"], ref.stats.z_mean, rtol=1e-5)
+
+
+@pytest.mark.parametrize("w", SMALL, ids=[w.name for w in SMALL])
+def test_small_bf16_layers(w):
+    inp, staged, y, st = _run(w)
+    np.testing.assert_array_equal(y, staged["y"])          # one-call layer == staged steps
+    rel, n, flips = compare_layer(inp, w, y, staged["idx"], staged["row_map"], staged["logits"],
+                                  tol=TOL_BF16)
+    assert n >= w.T - 3 * flips
+    print(f"{w.name}: rel_frob={rel:.3e} over {n} tokens, {flips} near-tie flips")
+
+
+@pytest.mark.parametrize("align", [1, 32])
+def test_segment_alignment_variants(align):
+    w = SMALL[1]
+    inp, staged, y, st = _run(w, align=align)
+    compare_layer(inp, w, y, staged["idx"], staged["row_map"], staged["logits"], tol=TOL_BF16,
+                  align=align)
+
+
+def test_capacity_zero_gives_shared_only():
+    w = Workload("cap0-shared", T=96, d=128, N=4, k=2, f=64, f_shared=128, capacity_factor=0.0)
+    inp, staged, y, st = _run(w)
+    assert int(st["num_dropped"][0]) == w.T * w.k
+    x64 = orc.as_f64(inp.x)
+    want = orc.swiglu_ffn(x64, inp.ws1, inp.ws3, inp.ws2, True)
+    got = gu.y_as_f64(y)
+    assert orc.rel_frobenius(got, want) <= TOL_BF16
+
+
+def test_deterministic_repeat():
+    w = SMALL[2]
+    inp = synth.make_inputs(w)
+    dl = moe.to_device(inp, moe.config_from_workload(w))
+    a, sa, _ = gu.layer_fwd(dl)
+    b, sb, _ = gu.layer_fwd(dl)
+    np.testing.assert_array_equal(a, b)
+    for key in sa:
+        np.testing.assert_array_equal(sa[key], sb[key])
+
+
+def test_empty_layer():
+    w = Workload("empty", T=0, d=128, N=8, k=2, f=128)
+    inp = synth.make_inputs(w)
+    dl = moe.to_device(inp, moe.config_from_workload(w))
+    y, st, flags = gu.layer_fwd(dl)
+    assert flags == 0 and y.shape == (0, 128)
+    assert np.all(st["counts"] == 0) and np.all(st["kept"] == 0) and st["num_dropped"][0] == 0

@@ -1,0 +1,149 @@
+"""GPU parity of routing and dispatch against the fp64 oracle.
+
+Routing indices, the permutation (row map, segment offsets, permuted rows), the
+drop mask and the expert counts must be bit-exact given identical fp32 logits,
+which reach the GPU through the test entry point moe_route_from_logits.  The
+routing weights and the load-balance statistics are fp32 on the GPU and fp64 in
+the oracle: relative tolerance 2e-6 (a few fp32 ulps of the softmax)."""
+import numpy as np
+import pytest
+import torch
+
+from expert_router_gemm_b200 import synth
+from oracle import moe_oracle as orc
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+from expert_router_gemm_b200 import moe  # noqa: E402
+from tests import gpu_util as gu  # noqa: E402
+
+W_RTOL = 2e-6
+
+
+def _check_route(T, N, k, pattern, seed=0):
+    logits = synth.make_logits(seed, T, N, pattern)
+    cfg = moe.make_config(T=T, d=64, N=N, k=k, f=64, capacity_factor=1.0, dtype="bf16")
+    idx, w, st, flags = gu.route_from_logits(cfg, logits)
+    assert flags == 0
+    g = logits.astype(np.float64)
+    want_idx = orc.topk(g, k)
+    np.testing.assert_array_equal(idx, want_idx)
+    s = orc.softmax(g)
+    np.testing.assert_allclose(w, orc.topk_weights(s, want_idx), rtol=W_RTOL, atol=1e-7)
+    ref = orc.aux_stats(want_idx, s, N)
+    np.testing.assert_array_equal(st["counts"], np.bincount(want_idx.reshape(-1), minlength=N))
+    np.testing.assert_allclose(st["y_frac"], ref.y_frac, rtol=1e-6, atol=0)
+    np.testing.assert_allclose(st["z_mean"], ref.z_mean, rtol=1e-5, atol=1e-7)
+    np.testing.assert_allclose(st["l_aux_p3"][0], ref.l_aux_p3, rtol=1e-5)
+    np.testing.assert_allclose(st["l_aux_switch"][0], ref.l_aux_switch, rtol=1e-5)
+
+
+@pytest.mark.parametrize("N,k", [(8, 1), (8, 2), (8, 8), (5, 3), (16, 4), (33, 7), (64, 32),
+                                 (128, 8), (256, 8), (256, 1), (1, 1)])
+@pytest.mark.parametrize("pattern", ["normal", "ties", "zeros", "onehot", "skewed"])
+def test_route_from_logits_bitexact(N, k, pattern):
+    for T in (1, 37, 300):
+        _check_route(T, N, k, pattern, seed=T)
+
+
+def test_route_from_logits_many_tokens():
+    _check_route(8192, 128, 8, "normal", seed=3)
+    _check_route(16384, 8, 2, "skewed", seed=4)
+
+
+def test_route_nonfinite_flag():
+    logits = synth.make_logits(0, 64, 8, "normal")
+    logits[5, 3] = np.nan
+    logits[9, 0] = np.inf
+    cfg = moe.make_config(T=64, d=64, N=8, k=2, f=64)
+    idx, w, st, flags = gu.route_from_logits(cfg, logits)
+    assert flags & moe.MOE_FLAG_NONFINITE_LOGITS
+    # the other tokens are routed as usual, and every index stays in range
+    ok = np.ones(64, bool)
+    ok[[5, 9]] = False
+    np.testing.assert_array_equal(idx[ok], orc.topk(logits[ok].astype(np.float64), 2))
+    assert idx.min() >= 0 and idx.max() < 8
+
+
+def _check_dispatch(T, N, k, d, cap, align, dtype, pattern, seed=0):
+    logits = synth.make_logits(seed, T, N, pattern)
+    idx = orc.topk(logits.astype(np.float64), k)
+    if dtype == "bf16":
+        x = synth.f32_to_bf16_bits(synth.normal_f32(seed, 99, (T, d)))
+    else:
+        x = synth.normal_f32(seed, 99, (T, d))
+    cfg = moe.make_config(T=T, d=d, N=N, k=k, f=64, capacity=cap, dtype=dtype, seg_align=align)
+    r = gu.dispatch(cfg, gu.cuda_tensor(x), gu.cuda_tensor(idx))
+    assert r["flags"] == 0
+    want = orc.dispatch(idx, N, cap, align)
+    np.testing.assert_array_equal(r["row_map"], want.row_map)
+    np.testing.assert_array_equal(r["seg_off"], want.seg_off)
+    np.testing.assert_array_equal(r["seg_count"], want.kept)
+    np.testing.assert_array_equal(r["stats"]["counts"], want.counts)
+    np.testing.assert_array_equal(r["stats"]["kept"], want.kept)
+    assert int(r["stats"]["num_dropped"][0]) == want.num_dropped
+    rows = orc.permuted_rows(x, want)
+    for row, xr in rows.items():
+        assert np.array_equal(r["xp"][row], xr), row
+
+
+@pytest.mark.parametrize("T,N,k,d,cap,align,dtype,pattern", [
+    (256, 8, 2, 128, 80, 128, "f32", "normal"),
+    (300, 8, 2, 64, 40, 128, "bf16", "skewed"),
+    (257, 16, 4, 64, 70, 32, "bf16", "normal"),
+    (100, 5, 5, 64, 100, 1, "bf16", "ties"),
+    (64, 4, 1, 64, 0, 8, "bf16", "normal"),          # capacity 0: everything dropped
+    (50, 3, 2, 64, 1000, 16, "f32", "normal"),       # capacity >= T: nothing dropped
+    (333, 8, 2, 64, 60, 128, "bf16", "onehot"),      # one over-full expert, others empty
+    (1, 8, 2, 64, 1, 128, "bf16", "normal"),
+    (1000, 128, 8, 256, 62, 128, "bf16", "normal"),
+    (777, 256, 8, 128, 24, 128, "bf16", "skewed"),
+    (129, 64, 32, 64, 80, 64, "bf16", "normal"),     # k = 32
+])
+def test_dispatch_bitexact(T, N, k, d, cap, align, dtype, pattern):
+    _check_dispatch(T, N, k, d, cap, align, dtype, pattern)
+
+
+def test_route_then_dispatch_bitexact():
+    # the GPU's own top-k feeds the GPU dispatch; both match the oracle on the same logits
+    T, N, k = 4096, 128, 8
+    logits = synth.make_logits(11, T, N, "skewed")
+    cfg = moe.make_config(T=T, d=64, N=N, k=k, f=64, capacity_factor=1.0, dtype="bf16")
+    idx, _, _, _ = gu.route_from_logits(cfg, logits)
+    x = synth.f32_to_bf16_bits(synth.normal_f32(1, 98, (T, 64)))
+    r = gu.dispatch(cfg, gu.cuda_tensor(x), gu.cuda_tensor(idx))
+    want = orc.dispatch(orc.topk(logits.astype(np.float64), k), N, orc.capacity(1.0, T, k, N), 128)
+    np.testing.assert_array_equal(r["row_map"], want.row_map)
+    np.testing.assert_array_equal(r["seg_off"], want.seg_off)
+    assert want.num_dropped > 0
+
+
+def test_dispatch_bad_index_flag():
+    T, N, k = 40, 8, 2
+    idx = orc.topk(synth.make_logits(2, T, N, "normal").astype(np.float64), k)
+    idx[3, 1] = 8        # out of range
+    idx[7, 0] = -1       # negative
+    idx[11, 1] = idx[11, 0]  # repeated within the row
+    x = synth.f32_to_bf16_bits(synth.normal_f32(2, 97, (T, 64)))
+    cfg = moe.make_config(T=T, d=64, N=N, k=k, f=64, capacity=T, dtype="bf16")
+    r = gu.dispatch(cfg, gu.cuda_tensor(x), gu.cuda_tensor(idx))
+    assert r["flags"] & moe.MOE_FLAG_BAD_EXPERT_INDEX
+    assert r["row_map"][3, 1] == -1 and r["row_map"][7, 0] == -1 and r["row_map"][11, 1] == -1
+    # valid slots are ranked as if the invalid ones were absent
+    clean = idx.copy()
+    keep = np.ones_like(idx, bool)
+    keep[3, 1] = keep[7, 0] = keep[11, 1] = False
+    assert r["stats"]["counts"].sum() == keep.sum()
+
+
+def test_empty_batch():
+    cfg = moe.make_config(T=0, d=64, N=8, k=2, f=64, capacity_factor=1.25)
+    idx, w, st, flags = gu.route_from_logits(cfg, np.zeros((0, 8), np.float32))
+    assert flags == 0 and idx.shape == (0, 2)
+    assert np.all(st["counts"] == 0) and np.all(st["y_frac"] == 0) and st["l_aux_p3"][0] == 0
+    r = gu.dispatch(cfg, torch.empty((0, 64), dtype=torch.int16, device="cuda"),
+                    torch.empty((0, 2), dtype=torch.int32, device="cuda"))
+    assert np.all(r["seg_off"] == 0) and np.all(r["seg_count"] == 0)
