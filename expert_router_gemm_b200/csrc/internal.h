@@ -71,6 +71,17 @@ struct DispatchArgs {
 };
 cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t s);
 
+// Validates a dispatch call and fills every field of `a` except the scratch
+// pointers (mask, base, counts, ticket) and flags; *blocks receives the number
+// of 32-token blocks.  Host only, touches no device state.
+moe_status_t dispatch_prepare(const moe_config_t* cfg, const void* x, const int32_t* topk_idx,
+                              int32_t* row_map, int32_t* seg_off, int32_t* seg_count, void* xp,
+                              const moe_stats_t* stats, DispatchArgs* a, int64_t* blocks);
+// T == 0: zero the segment table and the dispatch statistics.
+moe_status_t dispatch_empty(const DispatchArgs& a, cudaStream_t s);
+// MOE_OK for cudaSuccess, else MOE_ERR_CUDA with the error kept for moe_last_cuda_error().
+moe_status_t cuda_error_status(cudaError_t e);
+
 // ------------------------------------------------------------ expert FFN
 // One grouped SwiGLU FFN over G groups of rows.  Group g owns rows
 // [row0_g, row0_g + count_g) of `a` / `h` / `out`, where row0_g = seg_off[g]

@@ -288,6 +288,50 @@ bool ffn_weights_ok(const moe_weights_t* w) {
 
 }  // namespace
 
+namespace moe {
+
+moe_status_t dispatch_prepare(const moe_config_t* cfg, const void* x, const int32_t* topk_idx,
+                              int32_t* row_map, int32_t* seg_off, int32_t* seg_count, void* xp,
+                              const moe_stats_t* stats, DispatchArgs* a, int64_t* blocks) {
+  Dims D;
+  moe_status_t s = derive(cfg, &D);
+  if (s != MOE_OK) return s;
+  if (seg_off == nullptr || seg_count == nullptr) return MOE_ERR_INVALID_ARG;
+  if (D.T > 0 && (x == nullptr || topk_idx == nullptr || row_map == nullptr || xp == nullptr))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(xp)) return MOE_ERR_MISALIGNED;
+  *a = DispatchArgs{};
+  a->T = D.T;
+  a->d = D.d;
+  a->N = D.N;
+  a->k = D.k;
+  a->capacity = D.C;
+  a->align = D.align;
+  a->elem_bytes = D.elem;
+  a->x = x;
+  a->topk_idx = topk_idx;
+  a->row_map = row_map;
+  a->seg_off = seg_off;
+  a->seg_count = seg_count;
+  a->xp = xp;
+  if (stats) a->stats = *stats;
+  *blocks = (D.T + kDispatchTokens - 1) / kDispatchTokens;
+  return MOE_OK;
+}
+
+moe_status_t cuda_error_status(cudaError_t e) { return cuda_status(e); }
+
+moe_status_t dispatch_empty(const DispatchArgs& a, cudaStream_t st) {
+  cudaError_t e = cudaMemsetAsync(a.seg_off, 0, sizeof(int32_t) * (a.N + 1), st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(a.seg_count, 0, sizeof(int32_t) * a.N, st);
+  if (e == cudaSuccess && a.stats.counts) e = cudaMemsetAsync(a.stats.counts, 0, 4 * a.N, st);
+  if (e == cudaSuccess && a.stats.kept) e = cudaMemsetAsync(a.stats.kept, 0, 4 * a.N, st);
+  if (e == cudaSuccess && a.stats.num_dropped) e = cudaMemsetAsync(a.stats.num_dropped, 0, 4, st);
+  return cuda_status(e);
+}
+
+}  // namespace moe
+
 extern "C" {
 
 const char* moe_status_string(moe_status_t s) {

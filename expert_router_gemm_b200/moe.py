@@ -62,6 +62,8 @@ _PROTOS = {
                                              ctypes.POINTER(moe_stats_t), _P, _SZ, _P]),
     "moe_dispatch": (ctypes.c_int, [ctypes.POINTER(moe_config_t), _P, _P, _P, _P, _P, _P,
                                     ctypes.POINTER(moe_stats_t), _P, _SZ, _P]),
+    "moe_dispatch_static": (ctypes.c_int, [ctypes.POINTER(moe_config_t), _P, _P, _P, _P, _P, _P,
+                                           ctypes.POINTER(moe_stats_t), _P, _P]),
     "moe_expert_ffn": (ctypes.c_int, [ctypes.POINTER(moe_config_t), _P, _P, _P,
                                       ctypes.POINTER(moe_weights_t), _P, _P, _P, _SZ, _P]),
     "moe_shared_expert_ffn": (ctypes.c_int, [ctypes.POINTER(moe_config_t), _P,
@@ -189,6 +191,16 @@ def moe_dispatch(cfg, x, topk_idx, row_map, seg_off, seg_count, xp, stats, ws, s
                              _ptr(seg_off), _ptr(seg_count), _ptr(xp), _stats_ref(stats),
                              _ptr(ws), ws.numel() if ws is not None else 0, _stream(stream)),
            "moe_dispatch")
+
+
+def moe_dispatch_static(cfg, x, topk_idx, row_map, seg_off, seg_count, xp, stats,
+                        device_flags=None, stream=None):
+    _check(_lib.moe_dispatch_static(ctypes.byref(cfg), _ptr(x), _ptr(topk_idx), _ptr(row_map),
+                                    _ptr(seg_off), _ptr(seg_count), _ptr(xp), _stats_ref(stats),
+                                    _ptr(device_flags), _stream(stream)), "moe_dispatch_static")
+
+
+MOE_DISPATCH_STATIC_MAX_CELLS = 131072
 
 
 def moe_expert_ffn(cfg, xp, seg_off, seg_count, weights: moe_weights_t, h, out_rows, ws,

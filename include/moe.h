@@ -193,6 +193,39 @@ moe_status_t moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t*
                           moe_stats_t* stats, void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * moe_dispatch_static - moe_dispatch without a workspace: it allocates nothing
+ * and takes no scratch buffer from the caller.  The pages have no counterpart of
+ * this entry point.  It is meant for callers that cannot allocate device memory
+ * at the point where they dispatch: for example code whose device memory is
+ * owned by another allocator (a framework's memory pool), or a runtime that
+ * allocates only at start-up and must not call cudaMalloc (which can fail, and
+ * synchronises the device) while it serves batches.
+ *
+ * Inputs, outputs, results and errors are those of moe_dispatch, except:
+ *  - the scratch (per-block token masks and rank bases, counts, a ticket) lives
+ *    in one fixed array of MOE_DISPATCH_STATIC_SCRATCH_BYTES in the library's
+ *    device memory; every GPU that loads the library holds it until the process
+ *    exits;
+ *  - a batch needs ceil(T/32) * N <= MOE_DISPATCH_STATIC_MAX_CELLS (e.g. T up to
+ *    16384 with N = 256); larger batches return MOE_ERR_WORKSPACE and launch
+ *    nothing;
+ *  - device_flags (may be NULL) receives the MOE_FLAG_* bits by bitwise OR; the
+ *    caller zeroes it beforehand.  With NULL a bad index is still dropped
+ *    (row_map -1) but not reported.
+ *  - all calls share the one array and it keeps the last call's contents (each
+ *    call rewrites every part it reads).  Calls whose work overlaps on the GPU
+ *    (different streams, or several host threads) race on it: order them.
+ *  - the first call on a device looks up the array's device address (once per
+ *    device, with that device current); make that first call before any stream
+ *    capture.
+ */
+#define MOE_DISPATCH_STATIC_MAX_CELLS 131072
+#define MOE_DISPATCH_STATIC_SCRATCH_BYTES (2u * 4u * MOE_DISPATCH_STATIC_MAX_CELLS + 2048u)
+moe_status_t moe_dispatch_static(const moe_config_t* cfg, const void* x, const int32_t* topk_idx,
+                                 int32_t* row_map, int32_t* seg_off, int32_t* seg_count, void* xp,
+                                 moe_stats_t* stats, uint32_t* device_flags, moe_stream_t stream);
+
+/*
  * moe_expert_ffn - all routed experts as one grouped GEMM pair, SwiGLU fused.
  * "MoE 训练加速实战" §4.1-4.2: one kernel serves every expert, y_i = W_i x_i.
  * For every expert e and row r in [seg_off[e], seg_off[e] + seg_count[e]):
