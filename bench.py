@@ -231,6 +231,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work")
     ap.add_argument("--quick", action="store_true", help="layer loop only (profiling runs)")
+    ap.add_argument("--shape", default="",
+                    help="override workload fields for small profiling cases, e.g. T=2048,N=32")
     args = ap.parse_args()
     if args.warmup < 3 and not args.quick:
         ap.error("--warmup must be >= 3")
@@ -239,6 +241,10 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     w = configs.get(args.config)
+    if args.shape:
+        from dataclasses import replace
+        kv = dict(item.split("=") for item in args.shape.split(","))
+        w = replace(w, name=f"{w.name}[{args.shape}]", **{key: int(v) for key, v in kv.items()})
 
     if args.impl == "reference":
         run_reference(args, w, rank, world)
