@@ -389,12 +389,21 @@ def main():
         def tfs(fl, ms_):
             return fl / (ms_ / 1e3) / 1e12 if ms_ > 0 else None
 
+        tc_router = w.dtype == "bf16" and N > 32
+        route_entry = {"ms": round(stage_ms["route"], 4), "bytes": route_bytes, "flops": route_flops,
+                       "GB/s": round(gbs(route_bytes, stage_ms["route"]), 1),
+                       "frac_hbm": round(gbs(route_bytes, stage_ms["route"]) / hbm, 4),
+                       "TFLOP/s_fp32_equiv": round(tfs(route_flops, stage_ms["route"]), 2)}
+        if tc_router:
+            # tensor cores: three bf16 MMAs per fp32 weight (exact split)
+            route_entry["engine"] = "tcgen05, 3-part bf16 split"
+            route_entry["frac_tensor_executed"] = round(
+                tfs(3 * route_flops, stage_ms["route"]) / tc_peak, 4)
+        else:
+            route_entry["engine"] = "CUDA-core FFMA"
+            route_entry["frac_fp32_alu"] = round(tfs(route_flops, stage_ms["route"]) / FP32_ALU_TFLOPS, 4)
         kern = {
-            "route": {"ms": round(stage_ms["route"], 4), "bytes": route_bytes, "flops": route_flops,
-                      "GB/s": round(gbs(route_bytes, stage_ms["route"]), 1),
-                      "frac_hbm": round(gbs(route_bytes, stage_ms["route"]) / hbm, 4),
-                      "TFLOP/s_fp32": round(tfs(route_flops, stage_ms["route"]), 2),
-                      "frac_fp32_alu": round(tfs(route_flops, stage_ms["route"]) / FP32_ALU_TFLOPS, 4)},
+            "route": route_entry,
             "dispatch": {"ms": round(stage_ms["dispatch"], 4), "bytes": disp_bytes,
                          "GB/s": round(gbs(disp_bytes, stage_ms["dispatch"]), 1),
                          "frac_hbm": round(gbs(disp_bytes, stage_ms["dispatch"]) / hbm, 4)},

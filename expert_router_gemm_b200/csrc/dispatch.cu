@@ -65,6 +65,7 @@ __global__ void __launch_bounds__(1024) dispatch_scan_kernel(const DispatchArgs 
   __shared__ int part[32][33];
   __shared__ int is_last;
   __shared__ int kept_s[256];
+  __shared__ int drop_s[256];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int N = a.N;
   const int e = blockIdx.x * 32 + lane;
@@ -94,25 +95,40 @@ __global__ void __launch_bounds__(1024) dispatch_scan_kernel(const DispatchArgs 
   __threadfence();
 
   // last block: kept counts, aligned segment offsets, statistics
-  long long dropped = 0;
   for (int x = threadIdx.x; x < N; x += blockDim.x) {
     const int c = __ldcg(a.counts + x);
     const int kept = min(c, a.capacity);
     kept_s[x] = kept;
+    drop_s[x] = c - kept;
     a.seg_count[x] = kept;
     if (a.stats.counts) a.stats.counts[x] = c;
     if (a.stats.kept) a.stats.kept[x] = kept;
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    long long off = 0;
-    for (int x = 0; x < N; ++x) {
+  if (warp == 0) {
+    // exclusive scan of the aligned segment sizes: 8 experts per lane, then a warp scan
+    const int per = (N + 31) / 32;
+    const int x_lo = min(N, lane * per), x_hi = min(N, x_lo + per);
+    long long local = 0, drop = 0;
+    for (int x = x_lo; x < x_hi; ++x) {
+      local += (kept_s[x] + a.align - 1) / a.align * static_cast<long long>(a.align);
+      drop += drop_s[x];
+    }
+    long long incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) drop += __shfl_xor_sync(0xffffffffu, drop, o);
+    long long off = incl - local;
+    for (int x = x_lo; x < x_hi; ++x) {
       a.seg_off[x] = static_cast<int32_t>(off);
       off += (kept_s[x] + a.align - 1) / a.align * static_cast<long long>(a.align);
-      dropped += __ldcg(a.counts + x) - kept_s[x];
     }
-    a.seg_off[N] = static_cast<int32_t>(off);
-    if (a.stats.num_dropped) a.stats.num_dropped[0] = static_cast<int32_t>(dropped);
+    if (lane == 31) a.seg_off[N] = static_cast<int32_t>(incl);
+    if (lane == 0 && a.stats.num_dropped) a.stats.num_dropped[0] = static_cast<int32_t>(drop);
   }
 }
 

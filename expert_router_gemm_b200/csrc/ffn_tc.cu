@@ -339,38 +339,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------- host side
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  });
-  return fn;
-}
-
-// 2-D bf16 tensor [outer, inner] (row-major, rows of `inner` elements), box of
-// box_inner x box_outer elements, 128-byte swizzle, zero fill outside.
-bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint32_t box_inner,
-              uint32_t box_outer) {
-  EncodeTiledFn fn = encode_fn();
-  if (fn == nullptr) return false;
-  const cuuint64_t dims[2] = {inner, outer};
-  const cuuint64_t strides[1] = {inner * 2};
-  const cuuint32_t box[2] = {box_inner, box_outer};
-  const cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int MODE>
 cudaError_t set_smem_attr() {
   static std::once_flag once[64];
@@ -402,9 +370,9 @@ cudaError_t launch_ffn_bf16(const FfnArgs& a, cudaStream_t s) {
   const bool dense = a.seg_off == nullptr;
   const uint64_t G = dense ? 1 : static_cast<uint64_t>(a.G);
   CUtensorMap mA1, mW1, mW3, mA2, mW2;
-  if (!make_map(&mA1, a.a, a.d, a.max_rows, BK, BM) ||
-      !make_map(&mW1, a.w1, a.f, G * a.d, 64, BK) || !make_map(&mW3, a.w3, a.f, G * a.d, 64, BK) ||
-      !make_map(&mA2, a.h, a.f, a.max_rows, BK, BM) || !make_map(&mW2, a.w2, a.d, G * a.f, 64, BK))
+  if (!make_tma_2d_bf16(&mA1, a.a, a.d, a.max_rows, BK, BM) ||
+      !make_tma_2d_bf16(&mW1, a.w1, a.f, G * a.d, 64, BK) || !make_tma_2d_bf16(&mW3, a.w3, a.f, G * a.d, 64, BK) ||
+      !make_tma_2d_bf16(&mA2, a.h, a.f, a.max_rows, BK, BM) || !make_tma_2d_bf16(&mW2, a.w2, a.d, G * a.f, 64, BK))
     return cudaErrorInvalidValue;
 
   TcParams p{};

@@ -35,20 +35,26 @@ struct RouteArgs {
   float* logits_out;        // [T, N] or nullptr
   int32_t* topk_idx;        // [T, k]
   float* topk_w;            // [T, k]
-  int32_t* hist;            // [blocks, N]
-  float* zpart;             // [blocks, N]
+  int32_t* cnt_acc;         // [N] zeroed: top-k counts (statistics)
+  unsigned long long* z_acc;  // [N] zeroed: sum of softmax scores, 32 fraction bits
+  uint32_t* ticket;         // [1] zeroed: blocks finished (last one finalises)
+  int want_stats;           // fill `stats` (else the statistics are skipped)
+  moe_stats_t stats;        // device pointers, each may be null
   uint32_t* flags;
 };
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t s);
 
-struct RouteStatsArgs {
-  int64_t T;
-  int N, k, blocks;
-  const int32_t* hist;
-  const float* zpart;
-  moe_stats_t stats;        // device pointers, each may be null
-};
-cudaError_t launch_route_stats(const RouteStatsArgs& a, cudaStream_t s);
+// Router GEMM on the tensor cores (bf16 x, N > 32): splits W_r into the three
+// bf16 slabs at `split` (router_split_bytes) and writes fp32 logits (+ bias) to
+// `logits` [T, N]; the softmax / top-k pass then runs in logits mode.
+constexpr int kRouterTcMinExperts = 33;
+size_t router_split_bytes(int d, int N);
+cudaError_t launch_router_tc(const RouteArgs& a, void* split, float* logits, cudaStream_t s);
+
+// 2-D bf16 TMA tensor map over a row-major [outer, inner] tensor, 128-byte
+// swizzle, zero fill outside the tensor.
+bool make_tma_2d_bf16(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                      uint32_t box_outer);
 
 // --------------------------------------------------------------- dispatch
 constexpr int kDispatchTokens = 32;   // tokens per dispatch block (one bit each)

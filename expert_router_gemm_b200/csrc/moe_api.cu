@@ -116,14 +116,15 @@ moe_status_t derive(const moe_config_t* cfg, Dims* D) {
   return MOE_OK;
 }
 
+// Workspace layout.  The first bytes (flags word, route ticket, route count and
+// z accumulators) are zeroed by one memset at the start of every routing call.
 struct Layout {
-  size_t flags, rhist, rz, dmask, dbase, dcounts, dticket, op_end;
+  size_t flags, rticket, rcnt, rz, zero_end, rsplit, rlogits, dmask, dbase, dcounts, dticket, op_end;
   size_t idx, w, row_map, seg_off, seg_count, xp, h, hs, sh, layer_end;
 };
 
 Layout layout(const Dims& D) {
   Layout L{};
-  const int64_t rb = (D.T + route_bt(route_np(D.N)) - 1) / route_bt(route_np(D.N));
   const int64_t db = (D.T + kDispatchTokens - 1) / kDispatchTokens;
   size_t o = 0;
   auto take = [&](size_t bytes) {
@@ -131,9 +132,15 @@ Layout layout(const Dims& D) {
     o = round_up(o + bytes, kAlign);
     return at;
   };
-  L.flags = take(kAlign);
-  L.rhist = take(sizeof(int32_t) * rb * D.N);
-  L.rz = take(sizeof(float) * rb * D.N);
+  L.flags = 0;
+  L.rticket = sizeof(uint32_t);
+  take(kAlign);
+  L.rcnt = take(sizeof(int32_t) * D.N);
+  L.rz = take(sizeof(unsigned long long) * D.N);
+  L.zero_end = o;
+  const bool tc_router = D.bf16 && D.N >= kRouterTcMinExperts;
+  L.rsplit = take(tc_router ? router_split_bytes(D.d, D.N) : 0);
+  L.rlogits = take(tc_router ? sizeof(float) * D.T * D.N : 0);
   L.dmask = take(sizeof(uint32_t) * db * D.N);
   L.dbase = take(sizeof(int32_t) * db * D.N);
   L.dcounts = take(sizeof(int32_t) * D.N);
@@ -173,8 +180,20 @@ moe_status_t do_route(const Dims& D, const void* x, const float* w_router, const
                       const float* logits_in, float* logits_out, int32_t* topk_idx, float* topk_w,
                       const moe_stats_t* stats, void* ws, cudaStream_t st) {
   const Layout L = layout(D);
-  cudaError_t e = cudaMemsetAsync(at<uint32_t*>(ws, L.flags), 0, sizeof(uint32_t), st);
+  cudaError_t e = cudaMemsetAsync(ws, 0, L.zero_end, st);
   if (e != cudaSuccess) return cuda_status(e);
+  const bool want_stats = route_stats_requested(stats);
+  if (D.T == 0) {  // empty batch: statistics are zero
+    if (want_stats) {
+      const moe_stats_t& s = *stats;
+      if (e == cudaSuccess && s.y_frac) e = cudaMemsetAsync(s.y_frac, 0, sizeof(float) * D.N, st);
+      if (e == cudaSuccess && s.z_mean) e = cudaMemsetAsync(s.z_mean, 0, sizeof(float) * D.N, st);
+      if (e == cudaSuccess && s.counts) e = cudaMemsetAsync(s.counts, 0, sizeof(int32_t) * D.N, st);
+      if (e == cudaSuccess && s.l_aux_p3) e = cudaMemsetAsync(s.l_aux_p3, 0, sizeof(float), st);
+      if (e == cudaSuccess && s.l_aux_switch) e = cudaMemsetAsync(s.l_aux_switch, 0, sizeof(float), st);
+    }
+    return cuda_status(e);
+  }
   RouteArgs a{};
   a.T = D.T;
   a.d = D.d;
@@ -188,23 +207,22 @@ moe_status_t do_route(const Dims& D, const void* x, const float* w_router, const
   a.logits_out = logits_out;
   a.topk_idx = topk_idx;
   a.topk_w = topk_w;
-  a.hist = at<int32_t*>(ws, L.rhist);
-  a.zpart = at<float*>(ws, L.rz);
+  a.cnt_acc = at<int32_t*>(ws, L.rcnt);
+  a.z_acc = at<unsigned long long*>(ws, L.rz);
+  a.ticket = at<uint32_t*>(ws, L.rticket);
+  a.want_stats = want_stats ? 1 : 0;
+  if (want_stats) a.stats = *stats;
   a.flags = at<uint32_t*>(ws, L.flags);
+  if (logits_in == nullptr && D.bf16 && D.N >= kRouterTcMinExperts && D.T > 0) {
+    // tensor-core router GEMM -> fp32 logits, then softmax / top-k in logits mode
+    float* logits = logits_out != nullptr ? logits_out : at<float*>(ws, L.rlogits);
+    e = launch_router_tc(a, at<void*>(ws, L.rsplit), logits, st);
+    if (e != cudaSuccess) return cuda_status(e);
+    a.logits_in = logits;
+    a.logits_out = nullptr;
+  }
   e = launch_route(a, st);
   if (e != cudaSuccess) return cuda_status(e);
-  if (route_stats_requested(stats)) {
-    RouteStatsArgs s{};
-    s.T = D.T;
-    s.N = D.N;
-    s.k = D.k;
-    s.blocks = static_cast<int>((D.T + route_bt(route_np(D.N)) - 1) / route_bt(route_np(D.N)));
-    s.hist = a.hist;
-    s.zpart = a.zpart;
-    s.stats = *stats;
-    e = launch_route_stats(s, st);
-    if (e != cudaSuccess) return cuda_status(e);
-  }
   return MOE_OK;
 }
 

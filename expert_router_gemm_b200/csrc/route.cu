@@ -155,91 +155,140 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
     __syncthreads();
   }
 
-  // ---------------- softmax + top-k, one warp per token ----------------
+  // ---------------- softmax + top-k, TPW tokens per warp at a time ----------------
+  // The TPW tokens of a warp are processed in lock step so that their shuffle
+  // reductions overlap.
   constexpr int NPL = NP >= 32 ? NP / 32 : 1;  // logits held per lane
+  constexpr int TPW = 4;
+  constexpr int NW = kRouteThreads / 32;
   const int warp = tid >> 5, lane = tid & 31;
   float zacc[NPL];
 #pragma unroll
   for (int c = 0; c < NPL; ++c) zacc[c] = 0.f;
 
-  for (int tl = warp; tl < BT; tl += kRouteThreads / 32) {
-    const int64_t t = t0 + tl;
-    if (t >= T) break;
-    float v[NPL];
+  for (int tl0 = warp * TPW; tl0 < BT; tl0 += NW * TPW) {
+    float v[TPW][NPL], s[TPW][NPL];
+    bool valid[TPW];
     bool bad = false;
 #pragma unroll
-    for (int c = 0; c < NPL; ++c) {
-      const int e = lane + 32 * c;
-      v[c] = e < NP ? sm.u.lg[tl][e] : -INFINITY;
-      if (e < N && !isfinite(v[c])) bad = true;
-    }
-    if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(a.flags, kFlagNonfinite);
-
-    float m = -INFINITY;
-#pragma unroll
-    for (int c = 0; c < NPL; ++c) m = fmaxf(m, v[c]);
-    m = warp_max(m);
-    float ex[NPL], sum = 0.f;
-#pragma unroll
-    for (int c = 0; c < NPL; ++c) {
-      ex[c] = (lane + 32 * c < N) ? expf(v[c] - m) : 0.f;
-      sum += ex[c];
-    }
-    sum = warp_sum(sum);
-    float s[NPL];
-#pragma unroll
-    for (int c = 0; c < NPL; ++c) {
-      s[c] = ex[c] / sum;
-      zacc[c] += s[c];
-      if (isnan(v[c])) v[c] = -INFINITY;  // out of contract; keeps the selection well defined
-    }
-
-    // top-k on the logits: k rounds of a warp arg-max, (larger value, lower index) first
-    uint32_t taken = 0;
-    int my_idx = 0;
-    float my_s = 0.f, ssum = 0.f;
-    for (int j = 0; j < k; ++j) {
-      float bv = -INFINITY;
-      int bi = 0x7fffffff;
+    for (int q = 0; q < TPW; ++q) {
+      valid[q] = tl0 + q < BT && t0 + tl0 + q < T;
 #pragma unroll
       for (int c = 0; c < NPL; ++c) {
         const int e = lane + 32 * c;
-        if (e < N && !((taken >> c) & 1u) && (v[c] > bv || (v[c] == bv && e < bi))) {
-          bv = v[c];
-          bi = e;
-        }
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-        if (ov > bv || (ov == bv && oi < bi)) {
-          bv = ov;
-          bi = oi;
-        }
-      }
-      const int owner = bi & 31, slot = bi >> 5;
-      float sv = 0.f;
-      if (lane == owner) {
-        taken |= 1u << slot;
-#pragma unroll
-        for (int c = 0; c < NPL; ++c)
-          if (c == slot) sv = s[c];
-      }
-      sv = __shfl_sync(0xffffffffu, sv, owner);
-      ssum += sv;
-      if (lane == j) {
-        my_idx = bi;
-        my_s = sv;
+        v[q][c] = (valid[q] && e < NP) ? sm.u.lg[tl0 + q][e] : -INFINITY;
+        if (valid[q] && e < N && !isfinite(v[q][c])) bad = true;
       }
     }
-    if (lane < k) {
-      a.topk_idx[t * k + lane] = my_idx;
-      a.topk_w[t * k + lane] = my_s / ssum;
-      atomicAdd(&sm.hist[my_idx], 1);
+    if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(a.flags, kFlagNonfinite);
+
+    float m[TPW], sum[TPW];
+#pragma unroll
+    for (int q = 0; q < TPW; ++q) {
+      m[q] = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < NPL; ++c) m[q] = fmaxf(m[q], v[q][c]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+      for (int q = 0; q < TPW; ++q) m[q] = fmaxf(m[q], __shfl_xor_sync(0xffffffffu, m[q], o));
+#pragma unroll
+    for (int q = 0; q < TPW; ++q) {
+      sum[q] = 0.f;
+#pragma unroll
+      for (int c = 0; c < NPL; ++c) {
+        s[q][c] = (valid[q] && lane + 32 * c < N) ? expf(v[q][c] - m[q]) : 0.f;
+        sum[q] += s[q][c];
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+      for (int q = 0; q < TPW; ++q) sum[q] += __shfl_xor_sync(0xffffffffu, sum[q], o);
+#pragma unroll
+    for (int q = 0; q < TPW; ++q)
+#pragma unroll
+      for (int c = 0; c < NPL; ++c) {
+        if (valid[q]) {
+          s[q][c] = s[q][c] / sum[q];
+          zacc[c] += s[q][c];
+        }
+        if (isnan(v[q][c])) v[q][c] = -INFINITY;  // out of contract; keeps the selection defined
+      }
+
+    // top-k on the logits: k rounds of a warp arg-max, (larger value, lower index) first
+    uint32_t taken[TPW];
+    int my_idx[TPW];
+    float my_s[TPW], ssum[TPW];
+#pragma unroll
+    for (int q = 0; q < TPW; ++q) {
+      taken[q] = 0u;
+      my_idx[q] = 0;
+      my_s[q] = 0.f;
+      ssum[q] = 0.f;
+    }
+    for (int j = 0; j < k; ++j) {
+      float bv[TPW];
+      int bi[TPW];
+#pragma unroll
+      for (int q = 0; q < TPW; ++q) {
+        bv[q] = -INFINITY;
+        bi[q] = 0x7fffffff;
+#pragma unroll
+        for (int c = 0; c < NPL; ++c) {
+          const int e = lane + 32 * c;
+          if (e < N && !((taken[q] >> c) & 1u) && (v[q][c] > bv[q] || (v[q][c] == bv[q] && e < bi[q]))) {
+            bv[q] = v[q][c];
+            bi[q] = e;
+          }
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+        for (int q = 0; q < TPW; ++q) {
+          const float ov = __shfl_xor_sync(0xffffffffu, bv[q], o);
+          const int oi = __shfl_xor_sync(0xffffffffu, bi[q], o);
+          if (ov > bv[q] || (ov == bv[q] && oi < bi[q])) {
+            bv[q] = ov;
+            bi[q] = oi;
+          }
+        }
+#pragma unroll
+      for (int q = 0; q < TPW; ++q) {
+        const int owner = bi[q] & 31, slot = bi[q] >> 5;
+        float sv = 0.f;
+        if (lane == owner) {
+          taken[q] |= 1u << slot;
+#pragma unroll
+          for (int c = 0; c < NPL; ++c)
+            if (c == slot) sv = s[q][c];
+        }
+        sv = __shfl_sync(0xffffffffu, sv, owner);
+        ssum[q] += sv;
+        if (lane == j) {
+          my_idx[q] = bi[q];
+          my_s[q] = sv;
+        }
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < TPW; ++q) {
+      if (valid[q] && lane < k) {
+        const int64_t t = t0 + tl0 + q;
+        a.topk_idx[t * k + lane] = my_idx[q];
+        a.topk_w[t * k + lane] = my_s[q] / ssum[q];
+        if (a.want_stats) atomicAdd(&sm.hist[my_idx[q]], 1);
+      }
     }
   }
+  if (!a.want_stats) return;
 
+  // ---------------- load-balance statistics ----------------
+  // Block partials (fixed-order fp32 sum of the block's softmax scores, integer
+  // counts) go to global accumulators with integer atomics: the z sums as fixed
+  // point with 32 fraction bits, so the totals do not depend on block order.
 #pragma unroll
   for (int c = 0; c < NPL; ++c) {
     const int e = lane + 32 * c;
@@ -249,45 +298,38 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
   for (int e = tid; e < N; e += kRouteThreads) {
     float z = 0.f;
 #pragma unroll
-    for (int w = 0; w < kRouteThreads / 32; ++w) z += sm.zw[w][e];
-    a.zpart[static_cast<int64_t>(blockIdx.x) * N + e] = z;
-    a.hist[static_cast<int64_t>(blockIdx.x) * N + e] = sm.hist[e];
+    for (int w = 0; w < NW; ++w) z += sm.zw[w][e];
+    atomicAdd(a.z_acc + e, static_cast<unsigned long long>(__double2ull_rn(static_cast<double>(z) * 4294967296.0)));
+    if (sm.hist[e] != 0) atomicAdd(a.cnt_acc + e, sm.hist[e]);
   }
-}
-
-// Column sums of the per-block partials, in a fixed order, and the L_aux
-// scalars.  One warp per expert; lanes stride over the blocks.
-__global__ void __launch_bounds__(1024) route_stats_kernel(const RouteStatsArgs a) {
-  __shared__ double prod[256];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int N = a.N;
-  for (int e = warp; e < N; e += 32) {
-    long long cnt = 0;
-    double z = 0.0;
-    for (int b = lane; b < a.blocks; b += 32) {
-      cnt += a.hist[static_cast<int64_t>(b) * N + e];
-      z += static_cast<double>(a.zpart[static_cast<int64_t>(b) * N + e]);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
-      z += __shfl_xor_sync(0xffffffffu, z, o);
-    }
-    if (lane == 0) {
-      const double y = a.T > 0 ? static_cast<double>(cnt) / (static_cast<double>(a.T) * a.k) : 0.0;
-      const double zm = a.T > 0 ? z / static_cast<double>(a.T) : 0.0;
-      if (a.stats.counts) a.stats.counts[e] = static_cast<int32_t>(cnt);
-      if (a.stats.y_frac) a.stats.y_frac[e] = static_cast<float>(y);
-      if (a.stats.z_mean) a.stats.z_mean[e] = static_cast<float>(zm);
-      prod[e] = y * zm;
-    }
+  __threadfence();
+  __syncthreads();
+  __shared__ int is_last;
+  if (tid == 0) is_last = atomicAdd(a.ticket, 1u) == gridDim.x - 1;
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  double* prod = reinterpret_cast<double*>(&sm.u);   // the logits tile is no longer needed
+  for (int e = tid; e < N; e += kRouteThreads) {
+    const int cnt = __ldcg(a.cnt_acc + e);
+    const double zsum = static_cast<double>(__ldcg(a.z_acc + e)) * (1.0 / 4294967296.0);
+    const double y = static_cast<double>(cnt) / (static_cast<double>(T) * k);
+    const double zm = zsum / static_cast<double>(T);
+    if (a.stats.counts) a.stats.counts[e] = cnt;
+    if (a.stats.y_frac) a.stats.y_frac[e] = static_cast<float>(y);
+    if (a.stats.z_mean) a.stats.z_mean[e] = static_cast<float>(zm);
+    prod[e] = y * zm;
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
+  if (warp == 0) {
     double acc = 0.0;
-    for (int e = 0; e < N; ++e) acc += prod[e];
-    if (a.stats.l_aux_p3) a.stats.l_aux_p3[0] = static_cast<float>(static_cast<double>(a.T) / N * acc);
-    if (a.stats.l_aux_switch) a.stats.l_aux_switch[0] = static_cast<float>(N * acc);
+    for (int e = lane; e < N; e += 32) acc += prod[e];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) {
+      if (a.stats.l_aux_p3) a.stats.l_aux_p3[0] = static_cast<float>(static_cast<double>(T) / N * acc);
+      if (a.stats.l_aux_switch) a.stats.l_aux_switch[0] = static_cast<float>(N * acc);
+    }
   }
 }
 
@@ -314,11 +356,6 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t s) {
     case 128: return launch_np<128>(a, s);
     default: return launch_np<256>(a, s);
   }
-}
-
-cudaError_t launch_route_stats(const RouteStatsArgs& a, cudaStream_t s) {
-  route_stats_kernel<<<1, 1024, 0, s>>>(a);
-  return cudaGetLastError();
 }
 
 }  // namespace moe

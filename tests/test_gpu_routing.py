@@ -19,6 +19,7 @@ if not torch.cuda.is_available():
 
 from expert_router_gemm_b200 import moe  # noqa: E402
 from tests import gpu_util as gu  # noqa: E402
+from tests.layer_check import logit_bound  # noqa: E402
 
 W_RTOL = 2e-6
 
@@ -52,6 +53,73 @@ def test_route_from_logits_bitexact(N, k, pattern):
 def test_route_from_logits_many_tokens():
     _check_route(8192, 128, 8, "normal", seed=3)
     _check_route(16384, 8, 2, "skewed", seed=4)
+
+
+@pytest.mark.parametrize("T,d,N,k,dtype,bias", [
+    (300, 128, 8, 2, "f32", False),      # CUDA-core router, fp32 x
+    (257, 512, 8, 2, "bf16", True),      # CUDA-core router (N <= 32)
+    (300, 320, 33, 4, "bf16", False),    # tensor-core router, N not a multiple of 16
+    (1000, 256, 64, 8, "bf16", True),
+    (300, 4096, 128, 8, "bf16", False),
+    (129, 1024, 100, 6, "bf16", True),
+    (4800, 256, 256, 8, "bf16", False),  # more tiles than SMs: 128-wide expert tiles
+    (640, 7168, 256, 8, "bf16", True),
+])
+def test_route_gemm_logits(T, d, N, k, dtype, bias):
+    """Router GEMM against the oracle's fp64 logits; the top-k taken on the GPU's
+    own fp32 logits is checked as a property (larger logit first, ties to the
+    lower index), and agrees with the oracle's except at near ties."""
+    x = synth.normal_f32(7, 1, (T, d))
+    if dtype == "bf16":
+        x = synth.f32_to_bf16_bits(x)
+    wr = synth.normal_f32(7, 2, (d, N)) * np.float32(1 / np.sqrt(d))
+    b = synth.normal_f32(7, 3, (N,)) if bias else None
+    cfg = moe.make_config(T=T, d=d, N=N, k=k, f=64, capacity_factor=1.0, dtype=dtype)
+    logits = torch.full((T, N), float("nan"), device="cuda")
+    idx = torch.full((T, k), -1, dtype=torch.int32, device="cuda")
+    wt = torch.zeros((T, k), device="cuda")
+    ws = gu.op_workspace(cfg)
+    moe.moe_route(cfg, gu.cuda_tensor(x), gu.cuda_tensor(wr), None if b is None else gu.cuda_tensor(b),
+                  logits, idx, wt, None, ws)
+    assert moe.moe_read_flags(ws) == 0
+    g = gu.host(logits).astype(np.float64)
+    ref = orc.router_logits(x, wr, b)
+    assert np.all(np.abs(g - ref) <= logit_bound(x, wr, b))
+    got = gu.host(idx)
+    # property: the selection is the top-k of the GPU's own logits (ties -> lower index)
+    for t in range(T):
+        sel = list(got[t])
+        key = sorted(range(N), key=lambda e: (-g[t, e], e))[:k]
+        assert sel == key, (t, sel, key)
+    differ = np.any(got != orc.topk(ref, k), axis=1)
+    assert differ.sum() <= max(1, T // 500)
+
+
+@pytest.mark.parametrize("d,N,bias", [(256, 8, True), (320, 33, False), (512, 128, True),
+                                      (1024, 256, True)])
+def test_route_gemm_exact_on_one_hot_tokens(d, N, bias):
+    """Token t = unit vector e_(t mod d): every logit is one product 1 * w, so
+    the router GEMM must return the fp32 weight exactly (plus the bias, one fp32
+    addition).  This pins the exact three-way bf16 split of the weights and the
+    coverage of every K slab and expert tile, which the accumulation bound of
+    the random-input test is too loose to see."""
+    T = max(d, 300)
+    x = np.zeros((T, d), np.float32)
+    x[np.arange(T), np.arange(T) % d] = 1.0
+    x = synth.f32_to_bf16_bits(x)
+    wr = synth.normal_f32(8, 2, (d, N)) * np.float32(1 / np.sqrt(d))
+    b = synth.normal_f32(8, 3, (N,)) if bias else None
+    cfg = moe.make_config(T=T, d=d, N=N, k=min(N, 4), f=64, capacity_factor=1.0)
+    logits = torch.full((T, N), float("nan"), device="cuda")
+    idx = torch.empty((T, cfg.k), dtype=torch.int32, device="cuda")
+    wt = torch.empty((T, cfg.k), device="cuda")
+    ws = gu.op_workspace(cfg)
+    moe.moe_route(cfg, gu.cuda_tensor(x), gu.cuda_tensor(wr), None if b is None else gu.cuda_tensor(b),
+                  logits, idx, wt, None, ws)
+    want = wr[np.arange(T) % d]
+    if b is not None:
+        want = want + b[None, :]          # one fp32 addition, round to nearest
+    np.testing.assert_array_equal(gu.host(logits), want)
 
 
 def test_route_nonfinite_flag():
