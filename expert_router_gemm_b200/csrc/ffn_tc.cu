@@ -6,24 +6,36 @@
 //   GEMM1 (SWIGLU): h[r] = silu(xp[r] W1_e) * (xp[r] W3_e)  -> bf16
 //   GEMM2 (PLAIN):  out[r] = h[r] W2_e                       -> bf16
 //
-// Design (per CTA, one CTA per SM, 192 threads):
-//   warp 0 lane 0   TMA producer: A tile 128 x 64 (K-major rows of the permuted
-//                   activations) and B tile 64 x 256 (rows of the row-major weight,
-//                   i.e. MN-major) per stage, 128-byte swizzle, 4-stage ring.
-//   warp 1 lane 0   MMA issuer: tcgen05.mma kind::f16, M=128 N=256 K=16, fp32
-//                   accumulator in tensor memory; two accumulators (512 TMEM
-//                   columns) so the epilogue of tile i overlaps the main loop of
-//                   tile i+1.  Warp 1 also allocates and frees the TMEM.
+// Per CTA (one per SM, 192 threads):
+//   warp 0 lane 0   TMA producer: A slab 128 x 64 (K-major rows of the permuted
+//                   activations) and B slab 64 x (256/CG) (rows of the row-major
+//                   weight, i.e. MN-major), 128-byte swizzle, multi-stage ring.
+//   warp 1          allocates 512 TMEM columns (two accumulators, so the
+//                   epilogue of tile i overlaps the main loop of tile i+1);
+//                   lane 0 issues tcgen05.mma kind::f16, K=16, fp32 accumulator.
 //   warps 2-5       epilogue: tcgen05.ld of the accumulator rows, SwiGLU in fp32
 //                   (gate = columns 0-127, up = columns 128-255 of one tile, so
-//                   both halves of a hidden unit sit in the same CTA), one
-//                   rounding to bf16, masked stores of the valid rows.
+//                   both halves of a hidden unit meet in one thread), one
+//                   rounding to bf16, stores of the valid rows.
+// CG = 1: each CTA computes a 128 x 256 accumulator tile alone (M=128 MMA).
+// CG = 2: a cluster of two CTAs on two SMs computes a 256 x 256 tile with one
+//   cta_group::2 MMA (M=256) issued by the even CTA: each CTA stages its own 128
+//   rows of A and its own 128 columns of B (for SwiGLU: CTA 0 the W1 columns,
+//   CTA 1 the W3 columns), so per SM the operand traffic per flop is 2/3 of
+//   CG = 1 and six 32 KB stages fit instead of four 48 KB ones.  Both CTAs'
+//   loads count on the even CTA's barrier, its MMA commits to both CTAs'
+//   barriers, and both epilogues release the accumulator on the even CTA's
+//   barrier.  A pair tile covers 256 rows of one expert; an expert with an odd
+//   number of 128-row tiles leaves the second CTA's half of its last pair tile
+//   partly or fully outside the segment (computed, not stored).
 // Tiles are ordered (expert, N tile, M tile) with M fastest, so CTAs running at
 // the same time share weight slabs in L2; every CTA derives the tile list from
 // the device-side segment table, so no host synchronisation is needed.
 // Every mbarrier wait is bounded; on a timeout the kernel raises
 // MOE_FLAG_WAIT_TIMEOUT, waits (bounded) for its own copies and MMAs in flight,
 // frees its TMEM and returns.
+#include <algorithm>
+#include <cstdlib>
 #include <mutex>
 
 #include "device_utils.cuh"
@@ -32,21 +44,27 @@
 namespace moe {
 namespace {
 
-constexpr int BM = 128;                    // rows per tile (MMA M)
+constexpr int BM = 128;                    // rows per CTA (A slab rows)
 constexpr int BK = 64;                     // K per stage: 64 bf16 = one 128-byte swizzle row
 constexpr int MMA_N = 256;                 // accumulator columns per tile
 constexpr int MMA_K = 16;
-constexpr int STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;       // 16 KB
 constexpr int B_CHUNK = 64 * BK * 2;       // 8 KB: 64 output columns x 64 K rows
-constexpr int B_BYTES = 4 * B_CHUNK;       // 32 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int kThreads = 192;
 constexpr int kTmemCols = 2 * MMA_N;
 constexpr int kMaxGroups = 256;
-constexpr uint32_t kIdesc = idesc_bf16_f32(BM, MMA_N, /*b_mn_major=*/1);
 
 enum { MODE_SWIGLU = 0, MODE_PLAIN = 1 };
+
+template <int CG>
+struct Cfg {
+  static constexpr int B_CHUNKS = 4 / CG;                   // 64-column chunks of B per CTA
+  static constexpr int B_BYTES = B_CHUNKS * B_CHUNK;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;     // per CTA
+  static constexpr int STAGES = CG == 1 ? 4 : 6;
+  static constexpr int TILE_M = BM * CG;                    // accumulator rows of one (pair) tile
+  static constexpr uint32_t IDESC = idesc_bf16_f32(TILE_M, MMA_N, /*b_mn_major=*/1);
+};
 
 struct TcParams {
   const int32_t* seg_off;    // [G+1] or nullptr (one dense group of dense_rows rows)
@@ -61,8 +79,8 @@ struct TcParams {
 };
 
 struct TcTail {
-  uint64_t full[STAGES];
-  uint64_t empty[STAGES];
+  uint64_t full[8];
+  uint64_t empty[8];
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t drain;
@@ -73,13 +91,17 @@ struct TcTail {
   int32_t count[kMaxGroups];
 };
 
-constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(STAGES) * STAGE_BYTES + sizeof(TcTail);
+template <int CG>
+constexpr size_t smem_bytes() {
+  return 1024 + static_cast<size_t>(Cfg<CG>::STAGES) * Cfg<CG>::STAGE_BYTES + sizeof(TcTail);
+}
 
 struct Tile {
   int g, m0, n0;
 };
 
-__device__ __forceinline__ Tile decode_tile(const TcTail& s, int G, int bn, int t) {
+// tile t -> (group, first row of the (pair) tile, first output column)
+__device__ __forceinline__ Tile decode_tile(const TcTail& s, int G, int bn, int tile_m, int t) {
   int lo = 0, hi = G;  // largest g with tile_start[g] <= t
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
@@ -89,40 +111,56 @@ __device__ __forceinline__ Tile decode_tile(const TcTail& s, int G, int bn, int 
       hi = mid;
   }
   const int local = t - s.tile_start[lo];
-  const int mt = (s.count[lo] + BM - 1) / BM;
+  const int mt = (s.count[lo] + tile_m - 1) / tile_m;
   Tile r;
   r.g = lo;
   r.n0 = (local / mt) * bn;
-  r.m0 = (local % mt) * BM;
+  r.m0 = (local % mt) * tile_m;
   return r;
 }
 
 __device__ __forceinline__ float silu_f32(float u) { return u / (1.0f + expf(-u)); }
 
-template <int MODE>
+__device__ __forceinline__ void store_row32(uint16_t* orow, int col, int n_out, const uint32_t (&pk)[16]) {
+  if (col + 32 <= n_out) {
+    uint4* dst = reinterpret_cast<uint4*>(orow + col);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      if (col + i < n_out) orow[col + i] = static_cast<uint16_t>((pk[i >> 1] >> ((i & 1) * 16)) & 0xFFFFu);
+  }
+}
+
+template <int MODE, int CG>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_ffn_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                        const __grid_constant__ CUtensorMap tmB1, const TcParams p) {
+  using C = Cfg<CG>;
   constexpr int BN = MODE == MODE_SWIGLU ? MMA_N / 2 : MMA_N;  // output columns per tile
   extern __shared__ uint8_t dsmem[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = base;
-  uint8_t* sB = base + STAGES * A_BYTES;
-  TcTail& tl = *reinterpret_cast<TcTail*>(base + STAGES * STAGE_BYTES);
+  uint8_t* sB = base + C::STAGES * A_BYTES;
+  TcTail& tl = *reinterpret_cast<TcTail*>(base + C::STAGES * C::STAGE_BYTES);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = CG == 2 ? cluster_ctarank() : 0u;  // 0: this CTA issues the MMAs
+  const int unit = CG == 2 ? static_cast<int>(blockIdx.x) / 2 : static_cast<int>(blockIdx.x);
+  const int n_units = CG == 2 ? static_cast<int>(gridDim.x) / 2 : static_cast<int>(gridDim.x);
   const int G = p.seg_off != nullptr ? p.G : 1;
   const int n_tiles = (p.n_out + BN - 1) / BN;
   const int KB = p.K / BK;
 
   if (warp == 0 && lane == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(smem_addr(&tl.full[s]), 1);
       mbar_init(smem_addr(&tl.empty[s]), 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(smem_addr(&tl.tfull[a]), 1);
-      mbar_init(smem_addr(&tl.tempty[a]), 128);
+      mbar_init(smem_addr(&tl.tempty[a]), 128 * CG);
     }
     mbar_init(smem_addr(&tl.drain), 1);
     tl.abort = 0u;
@@ -132,8 +170,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (MODE == MODE_SWIGLU) tma_prefetch_desc(&tmB1);
   }
   if (warp == 1) {
-    tmem_alloc(smem_addr(&tl.tmem_base), kTmemCols);
-    tmem_relinquish();
+    if (CG == 2) {
+      tmem_alloc_pair(smem_addr(&tl.tmem_base), kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_addr(&tl.tmem_base), kTmemCols);
+      tmem_relinquish();
+    }
   }
   if (warp == 2) {
     // segment table -> per-group row range (clamped to the buffer) and tile prefix
@@ -153,7 +196,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tl.row0[g] = r0;
       tl.count[g] = c;
-      local += (c + BM - 1) / BM * n_tiles;
+      local += (c + C::TILE_M - 1) / C::TILE_M * n_tiles;
     }
     int incl = local;
 #pragma unroll
@@ -164,12 +207,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     int run = incl - local;
     for (int g = g_lo; g < g_hi; ++g) {
       tl.tile_start[g] = run;
-      run += (tl.count[g] + BM - 1) / BM * n_tiles;
+      run += (tl.count[g] + C::TILE_M - 1) / C::TILE_M * n_tiles;
     }
     if (lane == 31) tl.tile_start[G] = incl;
   }
   tc_fence_before();
-  __syncthreads();
+  if (CG == 2)
+    cluster_sync();  // both CTAs' barriers are initialised before any cross-CTA signal
+  else
+    __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = tl.tmem_base;
   const int total = tl.tile_start[G];
@@ -180,48 +226,66 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---------------------------------------------------------------- producer
       uint32_t stage = 0, phase = 0, issued = 0, last_par = 0;
       bool ok = true;
-      for (int t = blockIdx.x; ok && t < total; t += gridDim.x) {
-        const Tile tile = decode_tile(tl, G, BN, t);
-        const int a_row = tl.row0[tile.g] + tile.m0;
+      for (int t = unit; ok && t < total; t += n_units) {
+        const Tile tile = decode_tile(tl, G, BN, C::TILE_M, t);
+        const int a_row = tl.row0[tile.g] + tile.m0 + static_cast<int>(rank) * BM;
         const int b_row = tile.g * p.K;
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(smem_addr(&tl.empty[stage]), phase ^ 1u, abort, p.flags, kFlagTimeout)) {
             ok = false;
             break;
           }
-          const uint32_t fb = smem_addr(&tl.full[stage]);
-          mbar_arrive_expect_tx(fb, STAGE_BYTES);
-          tma_load_2d(smem_addr(sA + stage * A_BYTES), &tmA, fb, kb * BK, a_row);
-          const uint32_t bdst = smem_addr(sB + stage * B_BYTES);
+          const uint32_t fb_local = smem_addr(&tl.full[stage]);
+          const uint32_t a_dst = smem_addr(sA + stage * A_BYTES);
+          const uint32_t b_dst = smem_addr(sB + stage * C::B_BYTES);
           const int ky = b_row + kb * BK;
-          if (MODE == MODE_SWIGLU) {
-            tma_load_2d(bdst, &tmB0, fb, tile.n0, ky);
-            tma_load_2d(bdst + B_CHUNK, &tmB0, fb, tile.n0 + 64, ky);
-            tma_load_2d(bdst + 2 * B_CHUNK, &tmB1, fb, tile.n0, ky);
-            tma_load_2d(bdst + 3 * B_CHUNK, &tmB1, fb, tile.n0 + 64, ky);
-          } else {
+          if (CG == 1) {
+            mbar_arrive_expect_tx(fb_local, C::STAGE_BYTES);
+            tma_load_2d(a_dst, &tmA, fb_local, kb * BK, a_row);
+            if (MODE == MODE_SWIGLU) {
+              tma_load_2d(b_dst, &tmB0, fb_local, tile.n0, ky);
+              tma_load_2d(b_dst + B_CHUNK, &tmB0, fb_local, tile.n0 + 64, ky);
+              tma_load_2d(b_dst + 2 * B_CHUNK, &tmB1, fb_local, tile.n0, ky);
+              tma_load_2d(b_dst + 3 * B_CHUNK, &tmB1, fb_local, tile.n0 + 64, ky);
+            } else {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) tma_load_2d(bdst + i * B_CHUNK, &tmB0, fb, tile.n0 + 64 * i, ky);
+              for (int i = 0; i < 4; ++i) tma_load_2d(b_dst + i * B_CHUNK, &tmB0, fb_local, tile.n0 + 64 * i, ky);
+            }
+          } else {
+            // both CTAs' bytes complete on the even CTA's barrier
+            const uint32_t fb = rank == 0 ? fb_local : mapa_shared(fb_local, 0);
+            if (rank == 0) mbar_arrive_expect_tx(fb_local, 2 * C::STAGE_BYTES);
+            tma_load_2d_pair(a_dst, &tmA, fb, kb * BK, a_row);
+            const CUtensorMap* bmap = (MODE == MODE_SWIGLU && rank == 1) ? &tmB1 : &tmB0;
+            const int bcol = MODE == MODE_SWIGLU ? tile.n0 : tile.n0 + 128 * static_cast<int>(rank);
+            tma_load_2d_pair(b_dst, bmap, fb, bcol, ky);
+            tma_load_2d_pair(b_dst + B_CHUNK, bmap, fb, bcol + 64, ky);
           }
           issued |= 1u << stage;
           last_par = (last_par & ~(1u << stage)) | (phase << stage);
-          if (++stage == STAGES) {
+          if (++stage == C::STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
       }
-      // every load issued by this thread has landed before the CTA may exit
-      for (int s = 0; s < STAGES; ++s)
-        if ((issued >> s) & 1u)
-          mbar_wait(smem_addr(&tl.full[s]), (last_par >> s) & 1u, nullptr, p.flags, kFlagTimeout);
+      // Every load issued by this thread has landed before the CTA may exit:
+      // the even CTA sees its barrier complete; the odd CTA sees the MMA that
+      // consumed the load release the stage.
+      for (int s = 0; s < C::STAGES; ++s)
+        if ((issued >> s) & 1u) {
+          if (rank == 0)
+            mbar_wait(smem_addr(&tl.full[s]), (last_par >> s) & 1u, nullptr, p.flags, kFlagTimeout);
+          else
+            mbar_wait(smem_addr(&tl.empty[s]), (last_par >> s) & 1u, nullptr, p.flags, kFlagTimeout);
+        }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    if (lane == 0 && rank == 0) {
       // ---------------------------------------------------------------- MMA issuer
       uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
       bool ok = true, issued_any = false;
-      for (int t = blockIdx.x; ok && t < total; t += gridDim.x) {
+      for (int t = unit; ok && t < total; t += n_units) {
         if (!mbar_wait(smem_addr(&tl.tempty[acc]), acc_phase ^ 1u, abort, p.flags, kFlagTimeout)) break;
         tc_fence_after();
         issued_any = true;
@@ -233,41 +297,59 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
           const uint32_t a_addr = smem_addr(sA + stage * A_BYTES);
-          const uint32_t b_addr = smem_addr(sB + stage * B_BYTES);
+          const uint32_t b_addr = smem_addr(sB + stage * C::B_BYTES);
 #pragma unroll
           for (int kk = 0; kk < BK / MMA_K; ++kk) {
             // A: K-major, advance 16 elements (32 bytes) inside the swizzle row
             const uint64_t adesc = smem_desc_sw128(a_addr + kk * 32, 16, 1024);
             // B: MN-major, advance 16 K rows = two 8-row swizzle atoms (2048 bytes)
             const uint64_t bdesc = smem_desc_sw128(b_addr + kk * 2048, B_CHUNK, 1024);
-            tc_mma_f16(d_tmem, adesc, bdesc, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+            if (CG == 2)
+              tc_mma_f16_pair(d_tmem, adesc, bdesc, C::IDESC, (kb | kk) != 0 ? 1u : 0u);
+            else
+              tc_mma_f16(d_tmem, adesc, bdesc, C::IDESC, (kb | kk) != 0 ? 1u : 0u);
           }
-          tc_commit(smem_addr(&tl.empty[stage]));
-          if (++stage == STAGES) {
+          if (CG == 2) {
+            const uint32_t e = smem_addr(&tl.empty[stage]);
+            tc_commit_pair(e);
+            tc_commit_pair(mapa_shared(e, 1));
+          } else {
+            tc_commit(smem_addr(&tl.empty[stage]));
+          }
+          if (++stage == C::STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        tc_commit(smem_addr(&tl.tfull[acc]));
+        if (CG == 2) {
+          const uint32_t f = smem_addr(&tl.tfull[acc]);
+          tc_commit_pair(f);
+          tc_commit_pair(mapa_shared(f, 1));
+        } else {
+          tc_commit(smem_addr(&tl.tfull[acc]));
+        }
         if (++acc == 2) {
           acc = 0;
           acc_phase ^= 1u;
         }
       }
-      // all MMAs issued by this thread are complete before TMEM is released
+      // every MMA issued by this thread completes before TMEM is released
       if (issued_any) {
-        tc_commit(smem_addr(&tl.drain));
+        if (CG == 2)
+          tc_commit_pair(smem_addr(&tl.drain));
+        else
+          tc_commit(smem_addr(&tl.drain));
         mbar_wait(smem_addr(&tl.drain), 0u, nullptr, p.flags, kFlagTimeout);
       }
     }
   } else {
     // ------------------------------------------------------------------ epilogue
     const int quad = warp & 3;  // TMEM lanes 32*quad .. 32*quad+31 belong to this warp
-    const int r_in_tile = quad * 32 + lane;
+    const int r_in_tile = static_cast<int>(rank) * BM + quad * 32 + lane;
     uint32_t acc = 0, acc_phase = 0;
-    for (int t = blockIdx.x; t < total; t += gridDim.x) {
-      const Tile tile = decode_tile(tl, G, BN, t);
+    for (int t = unit; t < total; t += n_units) {
+      const Tile tile = decode_tile(tl, G, BN, C::TILE_M, t);
       if (!mbar_wait(smem_addr(&tl.tfull[acc]), acc_phase, abort, p.flags, kFlagTimeout)) break;
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * MMA_N;
@@ -289,15 +371,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               const float h1 = silu_f32(__uint_as_float(gv[2 * i + 1])) * __uint_as_float(uv[2 * i + 1]);
               pk[i] = pack_bf16x2(h0, h1);
             }
-            const int col = tile.n0 + c;
-            if (col + 32 <= p.n_out) {
-              uint4* dst = reinterpret_cast<uint4*>(orow + col);
-#pragma unroll
-              for (int q = 0; q < 4; ++q) dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-            } else {
-              for (int i = 0; i < 32 && col + i < p.n_out; ++i)
-                orow[col + i] = static_cast<uint16_t>((pk[i >> 1] >> ((i & 1) * 16)) & 0xFFFFu);
-            }
+            store_row32(orow, tile.n0 + c, p.n_out, pk);
           }
         }
       } else {
@@ -310,20 +384,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t pk[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-            const int col = tile.n0 + c;
-            if (col + 32 <= p.n_out) {
-              uint4* dst = reinterpret_cast<uint4*>(orow + col);
-#pragma unroll
-              for (int q = 0; q < 4; ++q) dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-            } else {
-              for (int i = 0; i < 32 && col + i < p.n_out; ++i)
-                orow[col + i] = static_cast<uint16_t>((pk[i >> 1] >> ((i & 1) * 16)) & 0xFFFFu);
-            }
+            store_row32(orow, tile.n0 + c, p.n_out, pk);
           }
         }
       }
       tc_fence_before();
-      mbar_arrive(smem_addr(&tl.tempty[acc]));
+      const uint32_t te = smem_addr(&tl.tempty[acc]);
+      if (CG == 2 && rank != 0)
+        mbar_arrive_cluster(mapa_shared(te, 0));
+      else
+        mbar_arrive(te);
       if (++acc == 2) {
         acc = 0;
         acc_phase ^= 1u;
@@ -331,15 +401,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
-  __syncthreads();
+  __syncwarp();
+  tc_fence_before();
+  if (CG == 2)
+    cluster_sync();  // the even CTA's MMAs (which write both CTAs' TMEM) have drained
+  else
+    __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, kTmemCols);
+    if (CG == 2)
+      tmem_dealloc_pair(tmem_base, kTmemCols);
+    else
+      tmem_dealloc(tmem_base, kTmemCols);
   }
 }
 
 // ---------------------------------------------------------------- host side
-template <int MODE>
+template <int MODE, int CG>
 cudaError_t set_smem_attr() {
   static std::once_flag once[64];
   int dev = 0;
@@ -347,20 +425,71 @@ cudaError_t set_smem_attr() {
   if (e != cudaSuccess) return e;
   cudaError_t r = cudaSuccess;
   std::call_once(once[dev & 63], [&] {
-    r = cudaFuncSetAttribute(tc_ffn_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kSmemBytes));
+    r = cudaFuncSetAttribute(tc_ffn_gemm_kernel<MODE, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem_bytes<CG>()));
   });
   return r;
 }
 
-template <int MODE>
+template <int MODE, int CG>
 cudaError_t launch_gemm(const CUtensorMap& A, const CUtensorMap& B0, const CUtensorMap& B1, const TcParams& p,
-                        int64_t bound_tiles, cudaStream_t s) {
-  cudaError_t e = set_smem_attr<MODE>();
+                        int64_t bound_units, cudaStream_t s) {
+  cudaError_t e = set_smem_attr<MODE, CG>();
   if (e != cudaSuccess) return e;
-  const int grid = static_cast<int>(std::min<int64_t>(device_sm_count(), std::max<int64_t>(bound_tiles, 1)));
-  tc_ffn_gemm_kernel<MODE><<<grid, kThreads, kSmemBytes, s>>>(A, B0, B1, p);
+  int units = device_sm_count() / CG;
+  units = static_cast<int>(std::min<int64_t>(units, std::max<int64_t>(bound_units, 1)));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(units * CG), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem_bytes<CG>();
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  if (CG == 2) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    // persistent: no more pairs than can be resident at once
+    int max_clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&max_clusters, tc_ffn_gemm_kernel<MODE, CG>, &cfg) == cudaSuccess &&
+        max_clusters > 0 && max_clusters < units)
+      cfg.gridDim.x = static_cast<unsigned>(max_clusters * 2);
+  }
+  e = cudaLaunchKernelEx(&cfg, tc_ffn_gemm_kernel<MODE, CG>, A, B0, B1, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+
+// CTA pairs pay off when experts have many rows; with few rows per expert the
+// 256-row pair tiles waste more of the MMA work on rows past the segment end.
+// MOE_FFN_CTA_GROUP=1|2 forces one variant (tests run both).
+int choose_cta_group(const FfnArgs& a) {
+  static int forced = [] {
+    const char* v = std::getenv("MOE_FFN_CTA_GROUP");
+    return v ? std::atoi(v) : 0;
+  }();
+  if (forced == 1 || forced == 2) return forced;
+  if (a.seg_off == nullptr) return 2;                     // dense shared expert: T rows
+  return a.mean_rows >= 384 ? 2 : 1;
+}
+
+template <int CG>
+cudaError_t launch_pair(const FfnArgs& a, const CUtensorMap& mA1, const CUtensorMap& mW1, const CUtensorMap& mW3,
+                        const CUtensorMap& mA2, const CUtensorMap& mW2, TcParams p, cudaStream_t s) {
+  const bool dense = a.seg_off == nullptr;
+  const int tile_m = Cfg<CG>::TILE_M;
+  const int64_t m_bound = (a.max_rows + tile_m - 1) / tile_m + (dense ? 0 : a.G);
+  p.K = a.d;
+  p.n_out = a.f;
+  p.out = static_cast<uint16_t*>(a.h);
+  cudaError_t e = launch_gemm<MODE_SWIGLU, CG>(mA1, mW1, mW3, p, m_bound * ((a.f + 127) / 128), s);
+  if (e != cudaSuccess) return e;
+  p.K = a.f;
+  p.n_out = a.d;
+  p.out = static_cast<uint16_t*>(a.out);
+  return launch_gemm<MODE_PLAIN, CG>(mA2, mW2, mW2, p, m_bound * ((a.d + 255) / 256), s);
 }
 
 }  // namespace
@@ -382,18 +511,8 @@ cudaError_t launch_ffn_bf16(const FfnArgs& a, cudaStream_t s) {
   p.dense_rows = a.dense_rows;
   p.max_rows = a.max_rows;
   p.flags = a.flags;
-  const int64_t m_bound = (a.max_rows + BM - 1) / BM + (dense ? 0 : a.G);
-
-  p.K = a.d;
-  p.n_out = a.f;
-  p.out = static_cast<uint16_t*>(a.h);
-  cudaError_t e = launch_gemm<MODE_SWIGLU>(mA1, mW1, mW3, p, m_bound * ((a.f + 127) / 128), s);
-  if (e != cudaSuccess) return e;
-
-  p.K = a.f;
-  p.n_out = a.d;
-  p.out = static_cast<uint16_t*>(a.out);
-  return launch_gemm<MODE_PLAIN>(mA2, mW2, mW2, p, m_bound * ((a.d + 255) / 256), s);
+  if (choose_cta_group(a) == 2) return launch_pair<2>(a, mA1, mW1, mW3, mA2, mW2, p, s);
+  return launch_pair<1>(a, mA1, mW1, mW3, mA2, mW2, p, s);
 }
 
 }  // namespace moe

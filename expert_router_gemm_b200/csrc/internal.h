@@ -97,6 +97,7 @@ struct FfnArgs {
   int G;
   int dense_rows;
   int max_count;            // upper bound of count_g (grid sizing of the fp32 path)
+  int64_t mean_rows;        // expected rows per group (tile-shape choice of the bf16 path)
   int64_t max_rows;         // rows of a / h / out buffers
   int d, f;
   const int32_t* seg_off;

@@ -269,6 +269,7 @@ moe_status_t do_ffn(const Dims& D, const void* a_rows, const int32_t* seg_off, c
   a.G = dense ? 1 : D.N;
   a.dense_rows = dense ? static_cast<int>(D.T) : 0;
   a.max_count = dense ? static_cast<int>(D.T) : static_cast<int>(D.max_count);
+  a.mean_rows = dense ? D.T : std::min<int64_t>(D.max_count, D.T * D.k / D.N);
   a.max_rows = dense ? D.T : D.max_rows;
   a.d = D.d;
   a.f = f;
