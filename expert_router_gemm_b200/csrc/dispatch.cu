@@ -24,7 +24,8 @@ namespace moe {
 namespace {
 
 constexpr int kMaskThreads = 256;
-constexpr int kScatterThreads = 32 * kDispatchTokens;  // one warp per token
+constexpr int kScatterTokens = 8;                         // tokens per scatter block
+constexpr int kScatterThreads = 32 * kScatterTokens;      // one warp per token
 constexpr int kCopyUnroll = 4;
 
 // true iff slot j of token t holds a valid expert index not used by an earlier slot
@@ -132,13 +133,16 @@ __global__ void __launch_bounds__(1024) dispatch_scan_kernel(const DispatchArgs 
   }
 }
 
+// One warp per token; a block covers 8 consecutive tokens of one 32-token mask
+// block (small blocks keep several resident per SM).
 __global__ void __launch_bounds__(kScatterThreads) dispatch_scatter_kernel(const DispatchArgs a) {
   __shared__ uint32_t m[256];
   __shared__ int base_s[256];
   __shared__ int off_s[256];
-  __shared__ int rows_s[kDispatchTokens][32];
+  __shared__ int rows_s[kScatterTokens][32];
   const int N = a.N, k = a.k;
-  const int64_t blk = blockIdx.x;
+  const int64_t t_first = static_cast<int64_t>(blockIdx.x) * kScatterTokens;
+  const int64_t blk = t_first / kDispatchTokens;                      // mask block
   for (int e = threadIdx.x; e < N; e += kScatterThreads) {
     m[e] = a.mask[blk * N + e];
     base_s[e] = a.base[blk * N + e];
@@ -146,7 +150,8 @@ __global__ void __launch_bounds__(kScatterThreads) dispatch_scatter_kernel(const
   }
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t t = blk * kDispatchTokens + warp;
+  const int64_t t = t_first + warp;
+  const int pos = static_cast<int>(t - blk * kDispatchTokens);        // bit of t in its mask word
   if (t >= a.T) return;
 
   if (lane < k) {
@@ -154,7 +159,7 @@ __global__ void __launch_bounds__(kScatterThreads) dispatch_scatter_kernel(const
     const int e = row[lane];
     int r = -1;
     if (slot_valid(row, lane, e, N)) {
-      const int rank = base_s[e] + __popc(m[e] & ((1u << warp) - 1u));
+      const int rank = base_s[e] + __popc(m[e] & ((1u << pos) - 1u));
       if (rank < a.capacity) r = off_s[e] + rank;
     }
     a.row_map[t * k + lane] = r;
@@ -188,7 +193,8 @@ cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t s) {
   const int blocks = static_cast<int>((a.T + kDispatchTokens - 1) / kDispatchTokens);
   dispatch_mask_kernel<<<blocks, kMaskThreads, 0, s>>>(a);
   dispatch_scan_kernel<<<(a.N + 31) / 32, 1024, 0, s>>>(a, blocks);
-  dispatch_scatter_kernel<<<blocks, kScatterThreads, 0, s>>>(a);
+  const unsigned sblocks = static_cast<unsigned>((a.T + kScatterTokens - 1) / kScatterTokens);
+  dispatch_scatter_kernel<<<sblocks, kScatterThreads, 0, s>>>(a);
   return cudaGetLastError();
 }
 

@@ -119,7 +119,10 @@ __device__ __forceinline__ Tile decode_tile(const TcTail& s, int G, int bn, int 
   return r;
 }
 
-__device__ __forceinline__ float silu_f32(float u) { return u / (1.0f + expf(-u)); }
+// silu(u) = u / (1 + e^-u) with the fast exponential and division: the result is
+// rounded to bf16 (8 significant bits), far above their fp32 error.  For very
+// negative u, e^-u overflows to inf and the quotient is -0.
+__device__ __forceinline__ float silu_f32(float u) { return __fdividef(u, 1.0f + __expf(-u)); }
 
 __device__ __forceinline__ void store_row32(uint16_t* orow, int col, int n_out, const uint32_t (&pk)[16]) {
   if (col + 32 <= n_out) {
@@ -131,6 +134,25 @@ __device__ __forceinline__ void store_row32(uint16_t* orow, int col, int n_out, 
     for (int i = 0; i < 32; ++i)
       if (col + i < n_out) orow[col + i] = static_cast<uint16_t>((pk[i >> 1] >> ((i & 1) * 16)) & 0xFFFFu);
   }
+}
+
+// The B operand of one K slab, as this CTA loads it: 64-column chunk i comes
+// from tensor map b_box_map(...) at column b_box_col(...).
+//   CG = 1, SwiGLU: W1 columns n0, n0+64 then W3 columns n0, n0+64
+//   CG = 1, plain:  W2 columns n0 + 64 i, i < 4
+//   CG = 2, SwiGLU: CTA 0 the two W1 chunks, CTA 1 the two W3 chunks
+//   CG = 2, plain:  CTA r the chunks at n0 + 128 r and n0 + 128 r + 64
+template <int MODE, int CG>
+__device__ __forceinline__ const CUtensorMap* b_box_map(const CUtensorMap* b0, const CUtensorMap* b1, uint32_t rank,
+                                                       int i) {
+  if (MODE != MODE_SWIGLU) return b0;
+  if (CG == 1) return i < 2 ? b0 : b1;
+  return rank == 0 ? b0 : b1;
+}
+template <int MODE, int CG>
+__device__ __forceinline__ int b_box_col(int n0, uint32_t rank, int i) {
+  if (CG == 1) return MODE == MODE_SWIGLU ? n0 + 64 * (i & 1) : n0 + 64 * i;
+  return MODE == MODE_SWIGLU ? n0 + 64 * i : n0 + 128 * static_cast<int>(rank) + 64 * i;
 }
 
 template <int MODE, int CG>
@@ -242,24 +264,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (CG == 1) {
             mbar_arrive_expect_tx(fb_local, C::STAGE_BYTES);
             tma_load_2d(a_dst, &tmA, fb_local, kb * BK, a_row);
-            if (MODE == MODE_SWIGLU) {
-              tma_load_2d(b_dst, &tmB0, fb_local, tile.n0, ky);
-              tma_load_2d(b_dst + B_CHUNK, &tmB0, fb_local, tile.n0 + 64, ky);
-              tma_load_2d(b_dst + 2 * B_CHUNK, &tmB1, fb_local, tile.n0, ky);
-              tma_load_2d(b_dst + 3 * B_CHUNK, &tmB1, fb_local, tile.n0 + 64, ky);
-            } else {
 #pragma unroll
-              for (int i = 0; i < 4; ++i) tma_load_2d(b_dst + i * B_CHUNK, &tmB0, fb_local, tile.n0 + 64 * i, ky);
-            }
+            for (int i = 0; i < Cfg<CG>::B_CHUNKS; ++i)
+              tma_load_2d(b_dst + i * B_CHUNK, b_box_map<MODE, CG>(&tmB0, &tmB1, rank, i), fb_local,
+                          b_box_col<MODE, CG>(tile.n0, rank, i), ky);
           } else {
             // both CTAs' bytes complete on the even CTA's barrier
             const uint32_t fb = rank == 0 ? fb_local : mapa_shared(fb_local, 0);
             if (rank == 0) mbar_arrive_expect_tx(fb_local, 2 * C::STAGE_BYTES);
             tma_load_2d_pair(a_dst, &tmA, fb, kb * BK, a_row);
-            const CUtensorMap* bmap = (MODE == MODE_SWIGLU && rank == 1) ? &tmB1 : &tmB0;
-            const int bcol = MODE == MODE_SWIGLU ? tile.n0 : tile.n0 + 128 * static_cast<int>(rank);
-            tma_load_2d_pair(b_dst, bmap, fb, bcol, ky);
-            tma_load_2d_pair(b_dst + B_CHUNK, bmap, fb, bcol + 64, ky);
+#pragma unroll
+            for (int i = 0; i < Cfg<CG>::B_CHUNKS; ++i)
+              tma_load_2d_pair(b_dst + i * B_CHUNK, b_box_map<MODE, CG>(&tmB0, &tmB1, rank, i), fb,
+                               b_box_col<MODE, CG>(tile.n0, rank, i), ky);
           }
           issued |= 1u << stage;
           last_par = (last_par & ~(1u << stage)) | (phase << stage);

@@ -44,10 +44,10 @@ struct RouteArgs {
 };
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t s);
 
-// Router GEMM on the tensor cores (bf16 x, N > 32): splits W_r into the three
+// Router GEMM on the tensor cores (bf16 x): splits W_r into the three
 // bf16 slabs at `split` (router_split_bytes) and writes fp32 logits (+ bias) to
 // `logits` [T, N]; the softmax / top-k pass then runs in logits mode.
-constexpr int kRouterTcMinExperts = 33;
+constexpr int kRouterTcMinExperts = 1;  // every bf16 layer
 size_t router_split_bytes(int d, int N);
 cudaError_t launch_router_tc(const RouteArgs& a, void* split, float* logits, cudaStream_t s);
 

@@ -45,11 +45,16 @@ struct RouteSmem {
   int hist[NP];
 };
 
+// Tokens per block in logits mode (no GEMM tile to fill): small blocks keep
+// every SM busy even when T is small or N has few experts.
+constexpr int kLogitsTokens = 32;
+
 template <int NP, bool FROM_LOGITS>
 __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a) {
   using S = RouteSmem<NP>;
-  constexpr int TX = S::TX, RT = S::RT, BT = S::BT;
-  static_assert(BT == route_bt(NP), "route block size mismatch");
+  constexpr int TX = S::TX, RT = S::RT, BT = FROM_LOGITS ? kLogitsTokens : S::BT;
+  static_assert(FROM_LOGITS || BT == route_bt(NP), "route block size mismatch");
+  static_assert(BT <= S::BT, "the logits tile holds at most S::BT tokens");
   static_assert(NP / TX == 8, "each thread owns 8 experts");
   __shared__ __align__(16) S sm;
 
@@ -335,7 +340,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
 
 template <int NP>
 cudaError_t launch_np(const RouteArgs& a, cudaStream_t s) {
-  const int bt = route_bt(NP);
+  const int bt = a.logits_in != nullptr ? kLogitsTokens : route_bt(NP);
   const unsigned blocks = static_cast<unsigned>((a.T + bt - 1) / bt);
   if (a.logits_in != nullptr)
     route_kernel<NP, true><<<blocks, kRouteThreads, 0, s>>>(a);

@@ -1,4 +1,5 @@
-// Router GEMM on the tcgen05 tensor cores for bf16 layers with N > 32 experts:
+// Router GEMM on the tcgen05 tensor cores for bf16 layers (any N <= 256; the
+// weight split is padded to a multiple of 64 experts with zeros):
 //   logits[t, e] = sum_c x[t, c] * W_r[c, e]  (+ b[e])        fp32 result
 // ("MoE 训练加速实战：DeepEP + Grouped GeMM + Aux-Loss-Free" §2.2: g = x W_r; the
 // router stays fp32, §1 pain point 4).
@@ -221,10 +222,12 @@ cudaError_t launch_bn(const CUtensorMap& mx, const CUtensorMap& mw, const RtPara
 
 }  // namespace
 
-size_t router_split_bytes(int d, int N) { return 3ull * d * route_np(N) * sizeof(uint16_t); }
+// the split slabs are [3][d][NPS] with NPS = N rounded up to a multiple of 64
+static int split_cols(int N) { return (N + 63) / 64 * 64; }
+size_t router_split_bytes(int d, int N) { return 3ull * d * split_cols(N) * sizeof(uint16_t); }
 
 cudaError_t launch_router_tc(const RouteArgs& a, void* split, float* logits, cudaStream_t s) {
-  const int NP = route_np(a.N);
+  const int NP = split_cols(a.N);
   const int64_t total = static_cast<int64_t>(a.d) * NP;
   const int threads = 256;
   const int blocks = static_cast<int>(std::min<int64_t>((total + threads - 1) / threads, 4 * device_sm_count()));
@@ -237,7 +240,7 @@ cudaError_t launch_router_tc(const RouteArgs& a, void* split, float* logits, cud
   RtParams p{a.T, a.N, a.d, a.bias, logits, a.flags};
   // 64-wide expert tiles while they fit in one wave, else 128-wide
   const int64_t m_tiles = (a.T + BM - 1) / BM;
-  if (m_tiles * ((a.N + 63) / 64) <= device_sm_count() || NP < 128) return launch_bn<64>(mx, mw, p, s);
+  if (m_tiles * (NP / 64) <= device_sm_count() || NP < 128) return launch_bn<64>(mx, mw, p, s);
   return launch_bn<128>(mx, mw, p, s);
 }
 

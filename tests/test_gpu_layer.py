@@ -78,6 +78,39 @@ def test_segment_alignment_variants(align):
                   align=align)
 
 
+_VARIANT_SCRIPT = r"""
+import sys
+sys.path.insert(0, {root!r})
+from expert_router_gemm_b200 import synth, moe
+from expert_router_gemm_b200.configs import Workload
+from tests import gpu_util as gu
+from tests.layer_check import compare_layer
+w = Workload("variant", T=1500, d=320, N=6, k=2, f=192, f_shared=128, capacity_factor=1.1)
+inp = synth.make_inputs(w)
+dl = moe.to_device(inp, moe.config_from_workload(w))
+st = gu.staged_layer(dl)
+assert st["flags"] == 0
+rel, n, flips = compare_layer(inp, w, st["y"], st["idx"], st["row_map"], st["logits"], tol=2e-2)
+print("REL", rel)
+"""
+
+
+@pytest.mark.parametrize("cta_group", ["1", "2"])
+def test_grouped_gemm_cta_group_variants(cta_group):
+    """Both tile shapes of the grouped GEMM (one CTA per 128x256 tile, or CTA
+    pairs per 256x256 tile) on a ragged layer with a shared expert.  The choice
+    is made once per process, so each variant runs in its own process."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, MOE_FFN_CTA_GROUP=cta_group)
+    r = subprocess.run([sys.executable, "-c", _VARIANT_SCRIPT.format(root=root)], env=env,
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert "REL" in r.stdout
+
+
 def test_capacity_zero_gives_shared_only():
     w = Workload("cap0-shared", T=96, d=128, N=4, k=2, f=64, f_shared=128, capacity_factor=0.0)
     inp, staged, y, st = _run(w)
