@@ -32,6 +32,8 @@ struct RouteArgs {
   const float* w_router;    // [d, N]
   const float* bias;        // [N] or nullptr
   const float* logits_in;   // [T, N] (logits mode) or nullptr
+  int n_partials;           // logits mode: logits_in holds this many [T, N] partial sums (>= 1),
+                            // added in order, then the bias (if any) is added
   float* logits_out;        // [T, N] or nullptr
   int32_t* topk_idx;        // [T, k]
   float* topk_w;            // [T, k]
@@ -48,8 +50,12 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t s);
 // bf16 slabs at `split` (router_split_bytes) and writes fp32 logits (+ bias) to
 // `logits` [T, N]; the softmax / top-k pass then runs in logits mode.
 constexpr int kRouterTcMinExperts = 1;  // every bf16 layer
+// The router GEMM splits K into up to kRouterMaxPartials slices (more CTAs for
+// small T or N); slice z writes partial sums to partials + z * T * N, without
+// the bias.  *n_partials receives the number of slices used.
+constexpr int kRouterMaxPartials = 4;
 size_t router_split_bytes(int d, int N);
-cudaError_t launch_router_tc(const RouteArgs& a, void* split, float* logits, cudaStream_t s);
+cudaError_t launch_router_tc(const RouteArgs& a, void* split, float* partials, int* n_partials, cudaStream_t s);
 
 // 2-D bf16 TMA tensor map over a row-major [outer, inner] tensor, 128-byte
 // swizzle, zero fill outside the tensor.

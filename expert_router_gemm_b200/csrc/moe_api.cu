@@ -140,7 +140,7 @@ Layout layout(const Dims& D) {
   L.zero_end = o;
   const bool tc_router = D.bf16 && D.N >= kRouterTcMinExperts;
   L.rsplit = take(tc_router ? router_split_bytes(D.d, D.N) : 0);
-  L.rlogits = take(tc_router ? sizeof(float) * D.T * D.N : 0);
+  L.rlogits = take(tc_router ? sizeof(float) * kRouterMaxPartials * D.T * D.N : 0);
   L.dmask = take(sizeof(uint32_t) * db * D.N);
   L.dbase = take(sizeof(int32_t) * db * D.N);
   L.dcounts = take(sizeof(int32_t) * D.N);
@@ -213,13 +213,15 @@ moe_status_t do_route(const Dims& D, const void* x, const float* w_router, const
   a.want_stats = want_stats ? 1 : 0;
   if (want_stats) a.stats = *stats;
   a.flags = at<uint32_t*>(ws, L.flags);
+  a.n_partials = 1;
   if (logits_in == nullptr && D.bf16 && D.N >= kRouterTcMinExperts && D.T > 0) {
-    // tensor-core router GEMM -> fp32 logits, then softmax / top-k in logits mode
-    float* logits = logits_out != nullptr ? logits_out : at<float*>(ws, L.rlogits);
-    e = launch_router_tc(a, at<void*>(ws, L.rsplit), logits, st);
+    // tensor-core router GEMM -> fp32 partial sums over K slices; the softmax /
+    // top-k pass adds them (and the bias) in a fixed order and writes logits_out
+    int parts = 1;
+    e = launch_router_tc(a, at<void*>(ws, L.rsplit), at<float*>(ws, L.rlogits), &parts, st);
     if (e != cudaSuccess) return cuda_status(e);
-    a.logits_in = logits;
-    a.logits_out = nullptr;
+    a.logits_in = at<float*>(ws, L.rlogits);
+    a.n_partials = parts;
   }
   e = launch_route(a, st);
   if (e != cudaSuccess) return cuda_status(e);

@@ -45,6 +45,16 @@ struct RouteSmem {
   int hist[NP];
 };
 
+// Monotone map of a float to an unsigned key (larger float -> larger key; -0.0
+// maps like +0.0) and back.
+__device__ __forceinline__ uint32_t order_key(float v) {
+  const uint32_t u = __float_as_uint(v == 0.f ? 0.f : v);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_value(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
 // Tokens per block in logits mode (no GEMM tile to fill): small blocks keep
 // every SM busy even when T is small or N has few experts.
 constexpr int kLogitsTokens = 32;
@@ -151,10 +161,18 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
       }
     }
   } else {
+    // logits = partial sums added in order (one for caller-supplied logits), + bias
+    const int64_t pstride = T * N;
     for (int v = tid; v < BT * NP; v += kRouteThreads) {
       const int r = v / NP, e = v % NP;
       float g = -INFINITY;
-      if (e < N && t0 + r < T) g = a.logits_in[(t0 + r) * N + e];
+      if (e < N && t0 + r < T) {
+        const float* src = a.logits_in + (t0 + r) * N + e;
+        g = src[0];
+        for (int z = 1; z < a.n_partials; ++z) g += src[z * pstride];
+        if (a.bias != nullptr) g += a.bias[e];
+        if (a.logits_out != nullptr) a.logits_out[(t0 + r) * N + e] = g;
+      }
       sm.u.lg[r][e] = g;
     }
     __syncthreads();
@@ -222,58 +240,62 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
         if (isnan(v[q][c])) v[q][c] = -INFINITY;  // out of contract; keeps the selection defined
       }
 
-    // top-k on the logits: k rounds of a warp arg-max, (larger value, lower index) first
-    uint32_t taken[TPW];
+    // top-k on the logits.  Each (logit, expert) becomes one 64-bit key whose
+    // unsigned order is "larger logit first, then lower expert index" (-0.0 is
+    // taken as +0.0 so equal logits tie).  A lane sorts its few keys; each round
+    // is one warp-wide max over the lanes' leading keys, and the winning lane
+    // drops its leading key.  The winner's weight is recomputed from its logit
+    // with the softmax's own expression.
+    uint64_t key[TPW][NPL];
+#pragma unroll
+    for (int q = 0; q < TPW; ++q) {
+#pragma unroll
+      for (int c = 0; c < NPL; ++c) {
+        const int e = lane + 32 * c;
+        key[q][c] = e < N ? (static_cast<uint64_t>(order_key(v[q][c])) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(e))
+                          : 0ull;
+      }
+#pragma unroll
+      for (int i = 1; i < NPL; ++i)
+#pragma unroll
+        for (int j2 = i; j2 > 0; --j2)
+          if (key[q][j2] > key[q][j2 - 1]) {
+            const uint64_t tmp = key[q][j2];
+            key[q][j2] = key[q][j2 - 1];
+            key[q][j2 - 1] = tmp;
+          }
+    }
     int my_idx[TPW];
     float my_s[TPW], ssum[TPW];
 #pragma unroll
     for (int q = 0; q < TPW; ++q) {
-      taken[q] = 0u;
       my_idx[q] = 0;
       my_s[q] = 0.f;
       ssum[q] = 0.f;
     }
     for (int j = 0; j < k; ++j) {
-      float bv[TPW];
-      int bi[TPW];
+      uint64_t best[TPW];
 #pragma unroll
-      for (int q = 0; q < TPW; ++q) {
-        bv[q] = -INFINITY;
-        bi[q] = 0x7fffffff;
-#pragma unroll
-        for (int c = 0; c < NPL; ++c) {
-          const int e = lane + 32 * c;
-          if (e < N && !((taken[q] >> c) & 1u) && (v[q][c] > bv[q] || (v[q][c] == bv[q] && e < bi[q]))) {
-            bv[q] = v[q][c];
-            bi[q] = e;
-          }
-        }
-      }
+      for (int q = 0; q < TPW; ++q) best[q] = key[q][0];
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1)
 #pragma unroll
         for (int q = 0; q < TPW; ++q) {
-          const float ov = __shfl_xor_sync(0xffffffffu, bv[q], o);
-          const int oi = __shfl_xor_sync(0xffffffffu, bi[q], o);
-          if (ov > bv[q] || (ov == bv[q] && oi < bi[q])) {
-            bv[q] = ov;
-            bi[q] = oi;
-          }
+          const uint64_t other = __shfl_xor_sync(0xffffffffu, best[q], o);
+          best[q] = other > best[q] ? other : best[q];
         }
 #pragma unroll
       for (int q = 0; q < TPW; ++q) {
-        const int owner = bi[q] & 31, slot = bi[q] >> 5;
-        float sv = 0.f;
-        if (lane == owner) {
-          taken[q] |= 1u << slot;
+        if (key[q][0] == best[q]) {  // keys are unique: exactly one lane drops its head
 #pragma unroll
-          for (int c = 0; c < NPL; ++c)
-            if (c == slot) sv = s[q][c];
+          for (int c = 0; c + 1 < NPL; ++c) key[q][c] = key[q][c + 1];
+          key[q][NPL - 1] = 0ull;
         }
-        sv = __shfl_sync(0xffffffffu, sv, owner);
+        const int e = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(best[q]));
+        const float sv = expf(key_value(static_cast<uint32_t>(best[q] >> 32)) - m[q]) / sum[q];
         ssum[q] += sv;
         if (lane == j) {
-          my_idx[q] = bi[q];
+          my_idx[q] = e;
           my_s[q] = sv;
         }
       }

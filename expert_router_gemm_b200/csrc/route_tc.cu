@@ -1,6 +1,10 @@
 // Router GEMM on the tcgen05 tensor cores for bf16 layers (any N <= 256; the
-// weight split is padded to a multiple of 64 experts with zeros):
-//   logits[t, e] = sum_c x[t, c] * W_r[c, e]  (+ b[e])        fp32 result
+// weight split is padded with zero columns to whole expert tiles):
+//   logits[t, e] = sum_c x[t, c] * W_r[c, e]                   fp32 result
+// written as 1, 2 or 4 partial sums over K slices (split z covers its share of
+// the K slabs, so small layers still fill the GPU); the softmax / top-k kernel
+// adds the partials in split order, then the bias.  No atomics: the result does
+// not depend on scheduling.
 // ("MoE 训练加速实战：DeepEP + Grouped GeMM + Aux-Loss-Free" §2.2: g = x W_r; the
 // router stays fp32, §1 pain point 4).
 //
@@ -11,11 +15,15 @@
 // MMAs of a K slab accumulate x*w in the fp32 tensor-memory accumulator.  The
 // result differs from a CUDA-core fp32 dot product only in summation order.
 //
-// One CTA per 128-token x BN-expert tile (BN = 64 or 128), 192 threads:
-// warp 0 lane 0 issues the TMA loads (x slab 128 x 64, three weight slabs
-// 64 x BN per stage), warp 1 allocates TMEM and lane 0 issues the MMAs, warps
-// 2-5 move the accumulator to registers, add the bias and store fp32 logits.
-// The softmax / top-k pass then runs on these logits (route.cu, logits mode).
+// 192 threads per CTA: warp 0 lane 0 issues the TMA loads (x slab 128 x 64 and
+// the three weight slabs of this CTA's experts per stage), warp 1 allocates TMEM
+// and lane 0 issues the MMAs, warps 2-5 move the accumulator to registers and
+// store the fp32 partial sums.  The operand stream is latency-bound (each
+// CTA streams its own tokens), so the work per staged byte decides the speed:
+//   CG = 1: one CTA per 128 tokens x 64 experts (M=128, N=64 MMA), N <= 64;
+//   CG = 2: a CTA pair per 256 tokens x 128 experts (cta_group::2, M=256,
+//           N=128): each CTA stages its own 128 tokens and 64 of the experts'
+//           weight columns, so each staged byte feeds twice the MMA work.
 // Every mbarrier wait is bounded (MOE_FLAG_WAIT_TIMEOUT).
 #include <algorithm>
 #include <mutex>
@@ -26,18 +34,22 @@
 namespace moe {
 namespace {
 
-constexpr int BM = 128;
+constexpr int BM = 128;                // tokens per CTA
 constexpr int BK = 64;
 constexpr int A_BYTES = BM * BK * 2;   // 16 KB
 constexpr int CHUNK = 64 * BK * 2;     // 8 KB: 64 expert columns x 64 K rows
 constexpr int kThreads = 192;
 
-template <int BN>
+template <int BN, int CG>
 struct RtCfg {
-  static constexpr int PART_BYTES = (BN / 64) * CHUNK;      // one of hi / mid / lo
+  static constexpr int COLS = BN / CG;                        // weight columns staged per CTA
+  static constexpr int CHUNKS = COLS / 64;
+  static constexpr int PART_BYTES = CHUNKS * CHUNK;           // one of hi / mid / lo
   static constexpr int STAGE_BYTES = A_BYTES + 3 * PART_BYTES;
-  static constexpr int STAGES = BN == 64 ? 5 : 3;
-  static constexpr int TMEM_COLS = BN;                      // power of two >= 32
+  static constexpr int STAGES = STAGE_BYTES <= 40 * 1024 ? 5 : 3;
+  static constexpr int TMEM_COLS = BN;                        // power of two >= 32
+  static constexpr uint32_t IDESC = idesc_bf16_f32(BM * CG, BN, 1);
+  static_assert(COLS % 64 == 0, "weight columns per CTA are whole 64-column chunks");
 };
 
 struct RtTail {
@@ -48,16 +60,16 @@ struct RtTail {
   uint32_t abort;
 };
 
-template <int BN>
+template <int BN, int CG>
 constexpr size_t rt_smem_bytes() {
-  return 1024 + static_cast<size_t>(RtCfg<BN>::STAGES) * RtCfg<BN>::STAGE_BYTES + sizeof(RtTail);
+  return 1024 + static_cast<size_t>(RtCfg<BN, CG>::STAGES) * RtCfg<BN, CG>::STAGE_BYTES + sizeof(RtTail);
 }
 
 struct RtParams {
   int64_t T;
   int N, d;
-  const float* bias;   // [N] or nullptr
-  float* logits;       // [T, N]
+  int kb_per_split;    // K slabs per split (blockIdx.z = split)
+  float* partials;     // [splits][T, N]: split z writes partials + z * T * N
   uint32_t* flags;
 };
 
@@ -81,19 +93,22 @@ __global__ void split_router_kernel(const float* __restrict__ w, uint16_t* __res
   }
 }
 
-template <int BN>
+template <int BN, int CG>
 __global__ void __launch_bounds__(kThreads, 1)
     router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                      const RtParams p) {
-  using C = RtCfg<BN>;
-  constexpr uint32_t kIdesc = idesc_bf16_f32(BM, BN, 1);
+  using C = RtCfg<BN, CG>;
   extern __shared__ uint8_t dsmem[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
   RtTail& tl = *reinterpret_cast<RtTail*>(base + C::STAGES * C::STAGE_BYTES);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * BM;
-  const int n0 = blockIdx.y * BN;
-  const int KB = p.d / BK;
+  const uint32_t rank = CG == 2 ? cluster_ctarank() : 0u;  // 0: this CTA issues the MMAs
+  const int m0 = (static_cast<int>(blockIdx.x) / CG) * (BM * CG) + static_cast<int>(rank) * BM;  // my tokens
+  const int n0 = blockIdx.y * BN;                           // the tile's first expert
+  const int ncol = n0 + static_cast<int>(rank) * C::COLS;   // my weight columns
+  const int kb0 = blockIdx.z * p.kb_per_split;              // this split's K slabs
+  const int KB = max(0, min(p.d / BK - kb0, p.kb_per_split));
+  float* const logits = p.partials + static_cast<int64_t>(blockIdx.z) * p.T * p.N;
 
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -107,11 +122,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tmW);
   }
   if (warp == 1) {
-    tmem_alloc(smem_addr(&tl.tmem_base), C::TMEM_COLS);
-    tmem_relinquish();
+    if (CG == 2) {
+      tmem_alloc_pair(smem_addr(&tl.tmem_base), C::TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_addr(&tl.tmem_base), C::TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if (CG == 2)
+    cluster_sync();
+  else
+    __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tl.tmem_base;
   volatile uint32_t* abort = &tl.abort;
@@ -121,16 +144,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t stage = 0, phase = 0, issued = 0, last_par = 0;
       for (int kb = 0; kb < KB; ++kb) {
         if (!mbar_wait(smem_addr(&tl.empty[stage]), phase ^ 1u, abort, p.flags, kFlagTimeout)) break;
-        const uint32_t fb = smem_addr(&tl.full[stage]);
-        mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
+        const uint32_t fb_local = smem_addr(&tl.full[stage]);
         const uint32_t sa = smem_addr(base + stage * C::STAGE_BYTES);
-        tma_load_2d(sa, &tmX, fb, kb * BK, m0);
+        if (CG == 1) {
+          mbar_arrive_expect_tx(fb_local, C::STAGE_BYTES);
+          tma_load_2d(sa, &tmX, fb_local, (kb0 + kb) * BK, m0);
 #pragma unroll
-        for (int part = 0; part < 3; ++part)
+          for (int part = 0; part < 3; ++part)
 #pragma unroll
-          for (int ch = 0; ch < BN / 64; ++ch)
-            tma_load_2d(sa + A_BYTES + part * C::PART_BYTES + ch * CHUNK, &tmW, fb, n0 + 64 * ch,
-                        part * p.d + kb * BK);
+            for (int ch = 0; ch < C::CHUNKS; ++ch)
+              tma_load_2d(sa + A_BYTES + part * C::PART_BYTES + ch * CHUNK, &tmW, fb_local, ncol + 64 * ch,
+                          part * p.d + (kb0 + kb) * BK);
+        } else {
+          // both CTAs' bytes complete on the even CTA's barrier
+          const uint32_t fb = rank == 0 ? fb_local : mapa_shared(fb_local, 0);
+          if (rank == 0) mbar_arrive_expect_tx(fb_local, 2 * C::STAGE_BYTES);
+          tma_load_2d_pair(sa, &tmX, fb, (kb0 + kb) * BK, m0);
+#pragma unroll
+          for (int part = 0; part < 3; ++part)
+#pragma unroll
+            for (int ch = 0; ch < C::CHUNKS; ++ch)
+              tma_load_2d_pair(sa + A_BYTES + part * C::PART_BYTES + ch * CHUNK, &tmW, fb, ncol + 64 * ch,
+                               part * p.d + (kb0 + kb) * BK);
+        }
         issued |= 1u << stage;
         last_par = (last_par & ~(1u << stage)) | (phase << stage);
         if (++stage == C::STAGES) {
@@ -138,12 +174,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           phase ^= 1u;
         }
       }
+      // every load issued here has landed before the CTA may exit
       for (int s = 0; s < C::STAGES; ++s)
-        if ((issued >> s) & 1u)
-          mbar_wait(smem_addr(&tl.full[s]), (last_par >> s) & 1u, nullptr, p.flags, kFlagTimeout);
+        if ((issued >> s) & 1u) {
+          if (rank == 0)
+            mbar_wait(smem_addr(&tl.full[s]), (last_par >> s) & 1u, nullptr, p.flags, kFlagTimeout);
+          else
+            mbar_wait(smem_addr(&tl.empty[s]), (last_par >> s) & 1u, nullptr, p.flags, kFlagTimeout);
+        }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    if (lane == 0 && rank == 0) {
       uint32_t stage = 0, phase = 0;
       bool ok = true, any = false;
       for (int kb = 0; kb < KB; ++kb) {
@@ -159,25 +200,40 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint64_t adesc = smem_desc_sw128(sa + kk * 32, 16, 1024);
             const uint64_t bdesc = smem_desc_sw128(sa + A_BYTES + part * C::PART_BYTES + kk * 2048, CHUNK, 1024);
-            tc_mma_f16(tmem, adesc, bdesc, kIdesc, (kb | part | kk) != 0 ? 1u : 0u);
+            const uint32_t acc = (kb | part | kk) != 0 ? 1u : 0u;
+            if (CG == 2)
+              tc_mma_f16_pair(tmem, adesc, bdesc, C::IDESC, acc);
+            else
+              tc_mma_f16(tmem, adesc, bdesc, C::IDESC, acc);
           }
         any = true;
-        tc_commit(smem_addr(&tl.empty[stage]));
+        const uint32_t e = smem_addr(&tl.empty[stage]);
+        if (CG == 2) {
+          tc_commit_pair(e);
+          tc_commit_pair(mapa_shared(e, 1));
+        } else {
+          tc_commit(e);
+        }
         if (++stage == C::STAGES) {
           stage = 0;
           phase ^= 1u;
         }
       }
       if (!ok) *abort = 1u;
-      if (any) {  // hand the accumulator to the epilogue; every MMA has drained before TMEM is freed
-        tc_commit(smem_addr(&tl.tfull));
-        mbar_wait(smem_addr(&tl.tfull), 0u, nullptr, p.flags, kFlagTimeout);
+      if (any) {  // hand the accumulator to the epilogues; every MMA has drained before TMEM is freed
+        const uint32_t f = smem_addr(&tl.tfull);
+        if (CG == 2) {
+          tc_commit_pair(f);
+          tc_commit_pair(mapa_shared(f, 1));
+        } else {
+          tc_commit(f);
+        }
+        mbar_wait(f, 0u, nullptr, p.flags, kFlagTimeout);
       }
     }
   } else {
     const int quad = warp & 3;
-    const int row = quad * 32 + lane;
-    const int64_t t = static_cast<int64_t>(m0) + row;
+    const int64_t t = static_cast<int64_t>(m0) + quad * 32 + lane;
     if (KB > 0 && mbar_wait(smem_addr(&tl.tfull), 0u, abort, p.flags, kFlagTimeout)) {
       tc_fence_after();
 #pragma unroll 1
@@ -186,48 +242,75 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + c, v);
         tmem_ld_wait();
         if (t < p.T) {
-          float* dst = p.logits + t * p.N + n0 + c;
+          float* dst = logits + t * p.N + n0 + c;
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             const int e = n0 + c + i;
-            if (e < p.N) dst[i] = __uint_as_float(v[i]) + (p.bias != nullptr ? p.bias[e] : 0.f);
+            if (e < p.N) dst[i] = __uint_as_float(v[i]);
           }
         }
       }
     }
   }
-  __syncthreads();
+  __syncwarp();
+  tc_fence_before();
+  if (CG == 2)
+    cluster_sync();  // the even CTA's MMAs (which write both CTAs' TMEM) have drained
+  else
+    __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, C::TMEM_COLS);
+    if (CG == 2)
+      tmem_dealloc_pair(tmem, C::TMEM_COLS);
+    else
+      tmem_dealloc(tmem, C::TMEM_COLS);
   }
 }
 
-template <int BN>
-cudaError_t launch_bn(const CUtensorMap& mx, const CUtensorMap& mw, const RtParams& p, cudaStream_t s) {
+template <int BN, int CG>
+cudaError_t launch_tile(const CUtensorMap& mx, const CUtensorMap& mw, const RtParams& p, int splits, cudaStream_t s) {
   static std::once_flag once[64];
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   cudaError_t r = cudaSuccess;
   std::call_once(once[dev & 63], [&] {
-    r = cudaFuncSetAttribute(router_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(rt_smem_bytes<BN>()));
+    r = cudaFuncSetAttribute(router_tc_kernel<BN, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(rt_smem_bytes<BN, CG>()));
   });
   if (r != cudaSuccess) return r;
-  const dim3 grid(static_cast<unsigned>((p.T + BM - 1) / BM), static_cast<unsigned>((p.N + BN - 1) / BN));
-  router_tc_kernel<BN><<<grid, kThreads, rt_smem_bytes<BN>(), s>>>(mx, mw, p);
+  cudaLaunchConfig_t cfg = {};
+  const int64_t tiles_m = (p.T + BM * CG - 1) / (BM * CG);
+  cfg.gridDim = dim3(static_cast<unsigned>(tiles_m * CG), static_cast<unsigned>((p.N + BN - 1) / BN),
+                     static_cast<unsigned>(splits));
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = rt_smem_bytes<BN, CG>();
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  if (CG == 2) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  e = cudaLaunchKernelEx(&cfg, router_tc_kernel<BN, CG>, mx, mw, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
+// The split slabs are [3][d][NPS]: N rounded up to the expert width of a tile
+// (128 for CTA pairs, used when N > 64; else 64), padded with zeros.
+int split_width(int N) { return N > 64 ? (N + 127) / 128 * 128 : (N + 63) / 64 * 64; }
+
 }  // namespace
 
-// the split slabs are [3][d][NPS] with NPS = N rounded up to a multiple of 64
-static int split_cols(int N) { return (N + 63) / 64 * 64; }
-size_t router_split_bytes(int d, int N) { return 3ull * d * split_cols(N) * sizeof(uint16_t); }
+size_t router_split_bytes(int d, int N) { return 3ull * d * split_width(N) * sizeof(uint16_t); }
 
-cudaError_t launch_router_tc(const RouteArgs& a, void* split, float* logits, cudaStream_t s) {
-  const int NP = split_cols(a.N);
+cudaError_t launch_router_tc(const RouteArgs& a, void* split, float* partials, int* n_partials, cudaStream_t s) {
+  const bool pairs = a.N > 64;
+  const int NP = split_width(a.N);
   const int64_t total = static_cast<int64_t>(a.d) * NP;
   const int threads = 256;
   const int blocks = static_cast<int>(std::min<int64_t>((total + threads - 1) / threads, 4 * device_sm_count()));
@@ -237,11 +320,20 @@ cudaError_t launch_router_tc(const RouteArgs& a, void* split, float* logits, cud
   CUtensorMap mx, mw;
   if (!make_tma_2d_bf16(&mx, a.x, a.d, a.T, BK, BM) || !make_tma_2d_bf16(&mw, split, NP, 3ull * a.d, 64, BK))
     return cudaErrorInvalidValue;
-  RtParams p{a.T, a.N, a.d, a.bias, logits, a.flags};
-  // 64-wide expert tiles while they fit in one wave, else 128-wide
-  const int64_t m_tiles = (a.T + BM - 1) / BM;
-  if (m_tiles * (NP / 64) <= device_sm_count() || NP < 128) return launch_bn<64>(mx, mw, p, s);
-  return launch_bn<128>(mx, mw, p, s);
+  // Split K while the grid stays within one wave and every split keeps >= 8 slabs.
+  const int tile_m = pairs ? 2 * BM : BM;
+  const int tile_n = pairs ? 128 : 64;
+  const int64_t ctas = (a.T + tile_m - 1) / tile_m * ((a.N + tile_n - 1) / tile_n) * (pairs ? 2 : 1);
+  const int kb_total = a.d / BK;
+  int splits = 1;
+  while (splits < kRouterMaxPartials && ctas * splits * 2 <= device_sm_count() && kb_total / (splits * 2) >= 8)
+    splits *= 2;
+  const int kbs = (kb_total + splits - 1) / splits;
+  splits = (kb_total + kbs - 1) / kbs;  // every split has at least one slab
+  *n_partials = splits;
+  RtParams p{a.T, a.N, a.d, kbs, partials, a.flags};
+  if (pairs) return launch_tile<128, 2>(mx, mw, p, splits, s);
+  return launch_tile<64, 1>(mx, mw, p, splits, s);
 }
 
 }  // namespace moe
