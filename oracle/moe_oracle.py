@@ -29,6 +29,12 @@ What is computed, in the pages' order and notation:
   8. load-balance statistics y_i (token fraction), z_i (mean gate score) and
      L_aux = (N_tok/E) sum y_i z_i ("负载均衡策略" section "辅助损失函数"), plus the
      Switch form N_exp * sum f_i P_i (§5.2 "传统方案：Auxiliary Loss").
+  9. Aux-Loss-Free routing: a per-expert bias b added to g for the top-k choice
+     only, and its update b_i <- b_i + gamma sign(1/N - f_i) (§5.3-5.4 of the
+     first page).
+ 10. router z-loss and the load-health figures (load std, top-2 share, tokens
+     per expert) ("负载均衡策略", hyper-parameter table, z_loss_weight; §9.1 of
+     the first page; "ms-swift + Megatron：MoE模型加速10倍实测" §3.3 "监控与诊断").
 
 Readings taken where the pages are silent or ambiguous (each also listed in the
 design notes):
@@ -49,6 +55,13 @@ design notes):
   (ix)  the shared expert is added with weight 1 after the routed sum;
   (x)   segment starts are rounded up to `align` rows (a layout choice that the
         oracle takes as a parameter).
+  (xi)  the selection bias is added to the fp32 logits in fp32; the weights and
+        z_i come from the unbiased softmax; f_i in the bias update counts the
+        top-k selections before the capacity drop;
+  (xii) the z-loss is the mean over tokens of (logsumexp_i g_ti)^2, the squared
+        log-partition of the router (the pages call it an L2 penalty on the
+        gate logits and give only its weight);
+  (xiii) the load figures follow the readings stated in load_metrics.
 """
 from __future__ import annotations
 
@@ -112,15 +125,50 @@ def softmax(g: np.ndarray) -> np.ndarray:
     return z / z.sum(axis=1, keepdims=True)
 
 
-def topk(g: np.ndarray, k: int) -> np.ndarray:
+def topk(g: np.ndarray, k: int, selection_bias: Optional[np.ndarray] = None) -> np.ndarray:
     """Indices of the k largest logits per token, in descending order.
 
     Equal logits are ordered by the lower expert index first: a stable sort of
     -g keeps equal keys in index order.  Returns int32 [T, k].
+
+    With a selection bias b (Aux-Loss-Free balancing, "MoE 训练加速实战" §5.3:
+    a per-expert offset that only steers the top-k choice) the experts are
+    ranked on g + b.  That sum is formed in fp32, the precision in which the
+    GPU takes the same decision; the weights are unaffected (topk_weights uses
+    the unbiased scores).
     """
     g = np.asarray(g, dtype=np.float64)
+    if selection_bias is not None:
+        g = (g.astype(np.float32) + np.asarray(selection_bias, np.float32)[None, :]).astype(np.float64)
     order = np.argsort(-g, axis=1, kind="stable")
     return order[:, :k].astype(np.int32)
+
+
+def bias_update(selection_bias: np.ndarray, counts: np.ndarray, T: int, k: int,
+                gamma: float) -> np.ndarray:
+    """One Aux-Loss-Free step ("MoE 训练加速实战" §5.4):
+    b_i <- b_i + gamma * sign(1/N - f_i), with f_i = counts_i / (T k) the share
+    of the batch's top-k assignments that expert i received (before the
+    capacity drop).  The sign is taken exactly, as sign(T k - N counts_i); the
+    update is one fp32 addition (b_i and gamma are fp32)."""
+    counts = np.asarray(counts, dtype=np.int64)
+    N = counts.shape[0]
+    sgn = np.sign(T * k - N * counts).astype(np.float32)
+    return np.asarray(selection_bias, np.float32) + np.float32(gamma) * sgn
+
+
+def router_z_loss(g: np.ndarray) -> float:
+    """Router z-loss: the mean over tokens of (log sum_i exp g_ti)^2.  The pages
+    name it as an L2 penalty on the gate logits that keeps them from growing
+    ("负载均衡策略：MoE训练稳定性保障", hyper-parameter table, z_loss_weight, and
+    section "常见问题"; "MoE 训练加速实战" §9.1 router_z_loss); the penalised
+    quantity is the log-partition z = logsumexp(g) of each token."""
+    g = np.asarray(g, dtype=np.float64)
+    if g.shape[0] == 0:
+        return 0.0
+    m = g.max(axis=1)
+    lse = m + np.log(np.exp(g - m[:, None]).sum(axis=1))
+    return float(np.mean(lse ** 2))
 
 
 def topk_weights(s: np.ndarray, idx: np.ndarray) -> np.ndarray:
@@ -233,6 +281,37 @@ def aux_stats(idx: np.ndarray, s: np.ndarray, N: int) -> AuxStats:
     return AuxStats(y, z, (T / N) * yz, N * yz)
 
 
+@dataclass
+class LoadMetrics:
+    load_std: float               # population std over experts of f_i = counts_i / (T k)
+    top2_ratio: float             # share of the T k selections taken by the two busiest experts
+    avg_tokens_per_expert: float  # rows the experts process, sum_i kept_i, over N
+
+
+def load_metrics(counts: np.ndarray, kept: np.ndarray, T: int, k: int) -> LoadMetrics:
+    """The three load-health figures of "ms-swift + Megatron：MoE模型加速10倍实测"
+    §3.3 "监控与诊断" (expert load std, top2_expert_ratio, avg_tokens_per_expert).
+
+    Readings: the load of expert i is its share f_i of the batch's T k top-k
+    selections (before the capacity drop) and the std is the population one
+    (over the N experts); top2_expert_ratio is the share of the selections
+    that the two most selected experts received (2/N when balanced, the page's
+    0.25 for 8 experts); avg_tokens_per_expert counts the rows an expert
+    actually processes, i.e. the kept assignments, averaged over the N experts.
+    An empty batch gives zeros.
+    """
+    counts = np.asarray(counts, dtype=np.int64)
+    kept = np.asarray(kept, dtype=np.int64)
+    N = counts.shape[0]
+    if T == 0:
+        return LoadMetrics(0.0, 0.0, 0.0)
+    f = counts / float(T * k)
+    load_std = float(np.sqrt(np.mean((f - f.mean()) ** 2)))
+    top = np.sort(counts)[::-1][:2]
+    top2 = float(top.sum()) / float(T * k)
+    return LoadMetrics(load_std, top2, float(kept.sum()) / float(N))
+
+
 # ----------------------------------------------------------------------------
 # the whole layer
 # ----------------------------------------------------------------------------
@@ -255,18 +334,20 @@ def layer_forward(x: np.ndarray, w_router: np.ndarray, bias: Optional[np.ndarray
                   capacity_factor: float = 1.0, cap: Optional[int] = None,
                   bf16: bool = True, ws1=None, ws3=None, ws2=None, align: int = 128,
                   tokens: Optional[Sequence[int]] = None,
-                  logits: Optional[np.ndarray] = None) -> LayerResult:
+                  logits: Optional[np.ndarray] = None,
+                  selection_bias: Optional[np.ndarray] = None) -> LayerResult:
     """Forward pass of one MoE layer.
 
     Routing and dispatch always cover all T tokens (the capacity clip depends on
     every earlier token); the expert FFN and combine are evaluated for `tokens`
     (default: all).  `logits`, if given, replaces step 1 (routing-parity mode).
+    `selection_bias` (Aux-Loss-Free routing) steers only the top-k choice.
     """
     T = x.shape[0]
     N = w_router.shape[1]
     g = router_logits(x, w_router, bias) if logits is None else np.asarray(logits, np.float64)
     s = softmax(g) if T else np.zeros((0, N))
-    idx = topk(g, k) if T else np.zeros((0, k), np.int32)
+    idx = topk(g, k, selection_bias) if T else np.zeros((0, k), np.int32)
     w = topk_weights(s, idx) if T else np.zeros((0, k))
     C = capacity(capacity_factor, T, k, N) if cap is None else int(cap)
     disp = dispatch(idx, N, C, align)

@@ -342,6 +342,119 @@ def test_aux_uniform():
 
 
 # --------------------------------------------------------------------------
+# Aux-Loss-Free selection bias and its update ("MoE 训练加速实战" §5.3-5.4)
+# --------------------------------------------------------------------------
+
+def check_selection_bias_hand(o=orc):
+    # g = (1, 7/8, 0, -1), b = (0, 1/4, 0, 0): the biased scores are (1, 9/8, 0, -1),
+    # so expert 1 wins the choice while the weights stay those of the plain softmax
+    g = np.array([[1.0, 0.875, 0.0, -1.0]])
+    b = np.array([0.0, 0.25, 0.0, 0.0], np.float32)
+    np.testing.assert_array_equal(o.topk(g, 1, b), [[1]])
+    np.testing.assert_array_equal(o.topk(g, 2, b), [[1, 0]])
+    np.testing.assert_array_equal(o.topk(g, 2), [[0, 1]])
+    e1, e78 = math.exp(1.0), math.exp(0.875)
+    w = o.topk_weights(o.softmax(g), o.topk(g, 2, b))
+    np.testing.assert_allclose(w, [[e78 / (e1 + e78), e1 / (e1 + e78)]], rtol=1e-15)
+    # an unbiased softmax: z_i of the statistics do not see the bias
+    st = o.aux_stats(o.topk(g, 1, b), o.softmax(g), 4)
+    np.testing.assert_allclose(st.y_frac, [0, 1, 0, 0])
+    np.testing.assert_allclose(st.z_mean, np.exp(g[0]) / np.exp(g[0]).sum(), rtol=1e-15)
+
+
+def check_selection_bias_bruteforce(o=orc):
+    # dyadic logits and biases (exact in fp32): the chosen set maximises
+    # sum_{i in S} (g_i + b_i) over all k-subsets; a bias constant over the
+    # experts changes nothing; a large bias on a set S of k experts forces S,
+    # ranked by g inside S
+    rng = np.random.default_rng(77)
+    N, k = 6, 3
+    for _ in range(40):
+        g = rng.integers(-64, 64, size=(1, N)) / 8.0
+        b = (rng.integers(-16, 16, size=N) / 8.0).astype(np.float32)
+        got = o.topk(g, k, b)[0]
+        sc = g[0] + b
+        best = max(itertools.combinations(range(N), k), key=lambda S: (sum(sc[i] for i in S), [-i for i in S]))
+        assert sorted(got.tolist()) == sorted(best), (g, b, got, best)
+        np.testing.assert_array_equal(o.topk(g, k, b + np.float32(0.5)), o.topk(g, k, b))
+        S = rng.choice(N, size=k, replace=False)
+        big = np.zeros(N, np.float32)
+        big[S] = 1024.0
+        want = sorted(S.tolist(), key=lambda i: (-g[0, i], i))
+        np.testing.assert_array_equal(o.topk(g, k, big)[0], want)
+        np.testing.assert_array_equal(o.topk(g, k, np.zeros(N, np.float32)), o.topk(g, k))
+
+
+def check_bias_update_hand(o=orc):
+    # T = 4 tokens, k = 2, N = 4: the fair share is T k / N = 2 selections.
+    # counts (3, 1, 0, 4): experts 0 and 3 over-loaded (b - gamma), 1 and 2
+    # under-loaded (b + gamma); an expert exactly at its share keeps its bias
+    b = np.array([0.5, 0.5, -0.5, 0.0], np.float32)
+    got = o.bias_update(b, np.array([3, 1, 0, 4]), T=4, k=2, gamma=0.25)
+    np.testing.assert_array_equal(got, np.array([0.25, 0.75, -0.25, -0.25], np.float32))
+    got = o.bias_update(b, np.array([2, 2, 2, 2]), T=4, k=2, gamma=0.25)
+    np.testing.assert_array_equal(got, b)
+    got = o.bias_update(b, np.array([2, 3, 1, 2]), T=4, k=2, gamma=0.25)
+    np.testing.assert_array_equal(got, np.array([0.5, 0.25, -0.25, 0.0], np.float32))
+    assert got.dtype == np.float32
+
+
+def test_selection_bias_hand():
+    check_selection_bias_hand()
+
+
+def test_selection_bias_bruteforce():
+    check_selection_bias_bruteforce()
+
+
+def test_bias_update_hand():
+    check_bias_update_hand()
+
+
+# --------------------------------------------------------------------------
+# router z-loss and the load-health figures
+# --------------------------------------------------------------------------
+
+def check_z_loss(o=orc):
+    # equal logits c over N experts: logsumexp = c + log N
+    for N, c in ((8, 0.0), (128, -2.5), (3, 7.0)):
+        g = np.full((5, N), c)
+        assert abs(o.router_z_loss(g) - (c + math.log(N)) ** 2) < 1e-12
+    # library special case: scipy's logsumexp, then the mean of its squares
+    g = np.random.default_rng(5).normal(size=(64, 32)) * 3
+    want = float(np.mean(scipy.special.logsumexp(g, axis=1) ** 2))
+    assert abs(o.router_z_loss(g) - want) < 1e-12 * want
+    # large logits (a stable log-sum-exp) and the empty batch
+    big = g + 1000.0
+    want = float(np.mean((scipy.special.logsumexp(g, axis=1) + 1000.0) ** 2))
+    assert abs(o.router_z_loss(big) - want) < 1e-12 * want
+    assert o.router_z_loss(np.zeros((0, 4))) == 0.0
+
+
+def check_load_metrics_hand(o=orc):
+    # counts (3, 1, 0, 4) of T k = 8 selections: f = (3, 1, 0, 4) / 8, mean 1/4,
+    # squared deviations (1, 1, 4, 4) / 64, so std = sqrt(10) / 16; the two
+    # busiest experts take 7 of 8; kept (3, 1, 0, 3) under C = 3 -> 7 / 4 rows each
+    m = o.load_metrics(np.array([3, 1, 0, 4]), np.array([3, 1, 0, 3]), T=4, k=2)
+    assert abs(m.load_std - math.sqrt(10) / 16) < 1e-15
+    assert m.top2_ratio == 7 / 8
+    assert m.avg_tokens_per_expert == 7 / 4
+    # perfectly balanced: std 0, top-2 share 2/N, T k / N rows per expert
+    m = o.load_metrics(np.full(8, 64), np.full(8, 64), T=256, k=2)
+    assert m.load_std == 0.0 and m.top2_ratio == 0.25 and m.avg_tokens_per_expert == 64.0
+    m = o.load_metrics(np.zeros(4, np.int64), np.zeros(4, np.int64), T=0, k=2)
+    assert (m.load_std, m.top2_ratio, m.avg_tokens_per_expert) == (0.0, 0.0, 0.0)
+
+
+def test_z_loss():
+    check_z_loss()
+
+
+def test_load_metrics_hand():
+    check_load_metrics_hand()
+
+
+# --------------------------------------------------------------------------
 # number formats
 # --------------------------------------------------------------------------
 
@@ -381,10 +494,12 @@ ALL_CHECKS = [check_capacity_worked_example, check_capacity_closed_forms, check_
               check_topk_bruteforce, check_topk_argmax, check_weights, check_dispatch_hand,
               check_dispatch_invariants, check_dense_mlp, check_dense_mixture,
               check_dropped_slots_contribute_zero, check_shared_expert_added, check_aux_hand,
-              check_aux_uniform, check_bf16_rounding, check_bf16_decode]
+              check_aux_uniform, check_bf16_rounding, check_bf16_decode, check_selection_bias_hand,
+              check_selection_bias_bruteforce, check_bias_update_hand, check_z_loss,
+              check_load_metrics_hand]
 
 
-def _mut_topk_high_index_ties(g, k):
+def _mut_topk_high_index_ties(g, k, selection_bias=None):
     g = np.asarray(g, np.float64)
     return np.argsort(g, axis=1, kind="stable")[:, ::-1][:, :k].astype(np.int32)
 
@@ -467,7 +582,58 @@ def _mut_bf16_decode_low_half(bits):
     return u32.view(np.float32).astype(np.float64)
 
 
-_ORIG = {n: getattr(orc, n) for n in ("dispatch", "swiglu_ffn", "aux_stats")}
+def _mut_topk_ignores_bias(g, k, selection_bias=None):
+    return _ORIG["topk"](g, k)
+
+
+def _mut_topk_bias_scaled(g, k, selection_bias=None):
+    # the bias applied with the wrong sign (it penalises the experts it should favour)
+    sb = None if selection_bias is None else -np.asarray(selection_bias, np.float32)
+    return _ORIG["topk"](g, k, sb)
+
+
+def _mut_bias_update_sign(b, counts, T, k, gamma):
+    counts = np.asarray(counts, np.int64)
+    return np.asarray(b, np.float32) + np.float32(gamma) * np.sign(counts.shape[0] * counts - T * k).astype(np.float32)
+
+
+def _mut_bias_update_share_of_tokens(b, counts, T, k, gamma):
+    counts = np.asarray(counts, np.int64)
+    return np.asarray(b, np.float32) + np.float32(gamma) * np.sign(T - counts.shape[0] * counts).astype(np.float32)
+
+
+def _mut_z_loss_unsquared(g):
+    g = np.asarray(g, np.float64)
+    return float(np.mean(scipy.special.logsumexp(g, axis=1))) if g.shape[0] else 0.0
+
+
+def _mut_z_loss_no_max(g):
+    g = np.asarray(g, np.float64)
+    with np.errstate(over="ignore"):
+        return float(np.mean(np.log(np.exp(g).sum(axis=1)) ** 2)) if g.shape[0] else 0.0
+
+
+def _mut_load_std_sample(counts, kept, T, k):
+    m = _ORIG["load_metrics"](counts, kept, T, k)
+    f = np.asarray(counts) / float(max(T * k, 1))
+    m.load_std = float(np.std(f, ddof=1))
+    return m
+
+
+def _mut_load_top1(counts, kept, T, k):
+    m = _ORIG["load_metrics"](counts, kept, T, k)
+    if T:
+        m.top2_ratio = float(np.max(counts)) / float(T * k)
+    return m
+
+
+def _mut_load_avg_counts(counts, kept, T, k):
+    m = _ORIG["load_metrics"](counts, kept, T, k)
+    m.avg_tokens_per_expert = float(np.sum(counts)) / len(counts)
+    return m
+
+
+_ORIG = {n: getattr(orc, n) for n in ("dispatch", "swiglu_ffn", "aux_stats", "topk", "load_metrics")}
 
 MUTANTS = [
     ("topk", _mut_topk_high_index_ties),
@@ -483,6 +649,15 @@ MUTANTS = [
     ("aux_stats", _mut_aux_p3_inverted),
     ("round_to_bf16", _mut_bf16_truncate),
     ("bf16_bits_to_f64", _mut_bf16_decode_low_half),
+    ("topk", _mut_topk_ignores_bias),
+    ("topk", _mut_topk_bias_scaled),
+    ("bias_update", _mut_bias_update_sign),
+    ("bias_update", _mut_bias_update_share_of_tokens),
+    ("router_z_loss", _mut_z_loss_unsquared),
+    ("router_z_loss", _mut_z_loss_no_max),
+    ("load_metrics", _mut_load_std_sample),
+    ("load_metrics", _mut_load_top1),
+    ("load_metrics", _mut_load_avg_counts),
 ]
 
 
