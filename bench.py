@@ -4,7 +4,11 @@
 
 A step is one forward pass of the whole layer (router GEMM + softmax + top-k +
 statistics, capacity clip + permutation, grouped SwiGLU GEMMs, combine) over one
-synthetic batch of the named workload, through the C ABI of libmoe.so.
+synthetic batch of the named workload, through the C ABI of libmoe.so.  The
+statistics include L_aux, the router z-loss and the load figures (last step's
+values in router_stats).  With --aux-free GAMMA the top-k choice also adds a
+per-expert selection bias, and each step ends with its on-device update
+(moe_bias_update) on the step's selection counts.
 
   value     tokens/s of moe_layer_fwd with inputs resident in HBM (K steps,
             CUDA events, max over ranks; every rank runs an independent replica,
@@ -231,6 +235,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work")
     ap.add_argument("--quick", action="store_true", help="layer loop only (profiling runs)")
+    ap.add_argument("--aux-free", type=float, default=0.0, metavar="GAMMA",
+                    help="Aux-Loss-Free routing: a selection bias, updated on the device with "
+                         "this step size after every layer call (0 = off)")
     ap.add_argument("--shape", default="",
                     help="override workload fields for small profiling cases, e.g. T=2048,N=32")
     args = ap.parse_args()
@@ -265,6 +272,9 @@ def main():
     inp = synth.make_inputs(w)
     cfg = moe.config_from_workload(w)
     dl = moe.to_device(inp, cfg)
+    aux_free = args.aux_free > 0
+    if aux_free:
+        dl.selection_bias = torch.zeros(w.N, dtype=torch.float32, device="cuda")
     act = moe.act_dtype(cfg)
     elem = 2 if w.dtype == "bf16" else 4
     lb, ob, max_rows = moe.moe_workspace_size(cfg)
@@ -274,13 +284,21 @@ def main():
                 l_aux_p3=torch.empty(1, device="cuda"), l_aux_switch=torch.empty(1, device="cuda"),
                 counts=torch.empty(w.N, dtype=torch.int32, device="cuda"),
                 kept=torch.empty(w.N, dtype=torch.int32, device="cuda"),
-                num_dropped=torch.empty(1, dtype=torch.int32, device="cuda"))
+                num_dropped=torch.empty(1, dtype=torch.int32, device="cuda"),
+                z_loss=torch.empty(1, device="cuda"), load_std=torch.empty(1, device="cuda"),
+                top2_ratio=torch.empty(1, device="cuda"),
+                avg_tokens_per_expert=torch.empty(1, device="cuda"))
     stats = moe.make_stats(**sbuf)
     weights = dl.weights()
     stream = torch.cuda.current_stream()
 
+    def layer_call(x_, y_):
+        moe.moe_layer_fwd(cfg, weights, x_, y_, stats, ws, stream)
+        if aux_free:
+            moe.moe_bias_update(cfg, dl.selection_bias, sbuf["counts"], args.aux_free, stream)
+
     def layer():
-        moe.moe_layer_fwd(cfg, weights, dl.x, y, stats, ws, stream)
+        layer_call(dl.x, y)
 
     def barrier():
         if dist is not None:
@@ -316,7 +334,14 @@ def main():
     value = world * w.T / (ms / 1e3)
     clocks = sampler.summary()
 
-    per_step_launches = 1 + 1 + 3 + 2 + (2 if w.f_shared else 0) + 1
+    # route: bf16 splits W_r, runs the tensor-core router GEMM and the softmax /
+    # top-k kernel (fp32: one fused kernel); dispatch: mask, scan, scatter; two
+    # grouped GEMMs (+ two for the shared expert); combine; the bias update
+    per_step_launches = ((3 if w.dtype == "bf16" else 1) + 3 + 2 + (2 if w.f_shared else 0) + 1
+                         + (1 if aux_free else 0))
+    router_stats = {key: round(float(sbuf[key].item()), 6) for key in
+                    ("l_aux_p3", "l_aux_switch", "z_loss", "load_std", "top2_ratio",
+                     "avg_tokens_per_expert")}
     line = {"metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
@@ -326,7 +351,11 @@ def main():
                               f"({(inp.w1.nbytes + inp.w3.nbytes + inp.w2.nbytes) / 1e9:.2f} GB) "
                               "exceed the 126 MB L2; no flush"),
             "gpu_launches": per_step_launches * args.steps, "clocks": clocks,
-            "device_flags": flags, "dropped": dropped}
+            "device_flags": flags, "dropped": dropped, "router_stats": router_stats}
+    if aux_free:
+        line["config"]["aux_loss_free_gamma"] = args.aux_free
+        b_last = dl.selection_bias.cpu()
+        line["selection_bias_range"] = [round(float(b_last.min()), 6), round(float(b_last.max()), 6)]
 
     if not args.quick:
         # -------------------------------------------- region B: per-stage events
@@ -341,11 +370,12 @@ def main():
         h = torch.empty((max_rows, f), dtype=act, device="cuda")
         hs = torch.empty((T, w.f_shared), dtype=act, device="cuda") if w.f_shared else None
         sh = torch.empty((T, d), dtype=act, device="cuda") if w.f_shared else None
-        names = ["route", "dispatch", "expert_ffn", "shared_ffn", "combine"]
+        names = ["route", "dispatch", "expert_ffn", "shared_ffn", "combine"] + (
+            ["bias_update"] if aux_free else [])
 
         def staged(evs):
             evs[0].record(stream)
-            moe.moe_route(cfg, dl.x, dl.w_router, dl.bias, None, idx, wt, stats, ws_op, stream)
+            moe.moe_route(cfg, dl.x, dl.w_router, dl.bias, dl.selection_bias, None, idx, wt, stats, ws_op, stream)
             evs[1].record(stream)
             moe.moe_dispatch(cfg, dl.x, idx, row_map, seg_off, seg_count, xp, stats, ws_op, stream)
             evs[2].record(stream)
@@ -356,10 +386,14 @@ def main():
             evs[4].record(stream)
             moe.moe_combine(cfg, xp, row_map, wt, sh, y, ws_op, stream)
             evs[5].record(stream)
+            if aux_free:
+                moe.moe_bias_update(cfg, dl.selection_bias, sbuf["counts"], args.aux_free, stream)
+                evs[6].record(stream)
 
+        n_ev = len(names) + 1
         for _ in range(3):
-            staged([torch.cuda.Event(enable_timing=True) for _ in range(6)])
-        all_evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+            staged([torch.cuda.Event(enable_timing=True) for _ in range(n_ev)])
+        all_evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
         barrier()
         torch.cuda.synchronize()
         for evs in all_evs:
@@ -389,7 +423,7 @@ def main():
         def tfs(fl, ms_):
             return fl / (ms_ / 1e3) / 1e12 if ms_ > 0 else None
 
-        tc_router = w.dtype == "bf16" and N > 32
+        tc_router = w.dtype == "bf16"
         route_entry = {"ms": round(stage_ms["route"], 4), "bytes": route_bytes, "flops": route_flops,
                        "GB/s": round(gbs(route_bytes, stage_ms["route"]), 1),
                        "frac_hbm": round(gbs(route_bytes, stage_ms["route"]) / hbm, 4),
@@ -416,6 +450,8 @@ def main():
                         "GB/s": round(gbs(comb_bytes, stage_ms["combine"]), 1),
                         "frac_hbm": round(gbs(comb_bytes, stage_ms["combine"]) / hbm, 4)},
         }
+        if aux_free:
+            kern["bias_update"] = {"ms": round(stage_ms["bias_update"], 5)}
         if w.f_shared:
             kern["shared_ffn"] = {"ms": round(stage_ms["shared_ffn"], 4), "flops": sh_flops,
                                   "TFLOP/s": round(tfs(sh_flops, stage_ms["shared_ffn"]), 1)}
@@ -460,7 +496,7 @@ def main():
             h2d_done[b].record(h2d)
             stream.wait_event(h2d_done[b])
             stream.wait_event(d2h_done[b])        # step i-2's output has left y_dev[b]
-            moe.moe_layer_fwd(cfg, weights, x_in[b], y_dev[b], stats, ws, stream)
+            layer_call(x_in[b], y_dev[b])
             comp_done[b].record(stream)
             d2h.wait_event(comp_done[b])
             with torch.cuda.stream(d2h):
@@ -485,7 +521,7 @@ def main():
         def serial_step(i):
             with torch.cuda.stream(stream):
                 x_in[0].copy_(x_host[0], non_blocking=True)
-            moe.moe_layer_fwd(cfg, weights, x_in[0], y_dev[0], stats, ws, stream)
+            layer_call(x_in[0], y_dev[0])
             with torch.cuda.stream(stream):
                 y_host[0].copy_(y_dev[0], non_blocking=True)
 

@@ -110,10 +110,11 @@ __global__ void __launch_bounds__(1024) dispatch_scan_kernel(const DispatchArgs 
     // exclusive scan of the aligned segment sizes: 8 experts per lane, then a warp scan
     const int per = (N + 31) / 32;
     const int x_lo = min(N, lane * per), x_hi = min(N, x_lo + per);
-    long long local = 0, drop = 0;
+    long long local = 0, drop = 0, kept_sum = 0;
     for (int x = x_lo; x < x_hi; ++x) {
       local += (kept_s[x] + a.align - 1) / a.align * static_cast<long long>(a.align);
       drop += drop_s[x];
+      kept_sum += kept_s[x];
     }
     long long incl = local;
 #pragma unroll
@@ -122,7 +123,10 @@ __global__ void __launch_bounds__(1024) dispatch_scan_kernel(const DispatchArgs 
       if (lane >= o) incl += v;
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) drop += __shfl_xor_sync(0xffffffffu, drop, o);
+    for (int o = 16; o > 0; o >>= 1) {
+      drop += __shfl_xor_sync(0xffffffffu, drop, o);
+      kept_sum += __shfl_xor_sync(0xffffffffu, kept_sum, o);
+    }
     long long off = incl - local;
     for (int x = x_lo; x < x_hi; ++x) {
       a.seg_off[x] = static_cast<int32_t>(off);
@@ -130,6 +134,8 @@ __global__ void __launch_bounds__(1024) dispatch_scan_kernel(const DispatchArgs 
     }
     if (lane == 31) a.seg_off[N] = static_cast<int32_t>(incl);
     if (lane == 0 && a.stats.num_dropped) a.stats.num_dropped[0] = static_cast<int32_t>(drop);
+    if (lane == 0 && a.stats.avg_tokens_per_expert)
+      a.stats.avg_tokens_per_expert[0] = static_cast<float>(static_cast<double>(kept_sum) / N);
   }
 }
 

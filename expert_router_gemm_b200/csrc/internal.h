@@ -31,6 +31,7 @@ struct RouteArgs {
   const void* x;            // [T, d] (GEMM mode) or nullptr
   const float* w_router;    // [d, N]
   const float* bias;        // [N] or nullptr
+  const float* sel_bias;    // [N] or nullptr: added to the logits for the top-k choice only
   const float* logits_in;   // [T, N] (logits mode) or nullptr
   int n_partials;           // logits mode: logits_in holds this many [T, N] partial sums (>= 1),
                             // added in order, then the bias (if any) is added
@@ -40,11 +41,17 @@ struct RouteArgs {
   int32_t* cnt_acc;         // [N] zeroed: top-k counts (statistics)
   unsigned long long* z_acc;  // [N] zeroed: sum of softmax scores, 32 fraction bits
   uint32_t* ticket;         // [1] zeroed: blocks finished (last one finalises)
+  double* zl_part;          // [blocks] per-block sums of logsumexp^2 (z-loss)
   int want_stats;           // fill `stats` (else the statistics are skipped)
   moe_stats_t stats;        // device pointers, each may be null
   uint32_t* flags;
 };
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t s);
+// The route kernel's blocks hold at least this many tokens (sizes zl_part).
+constexpr int kRouteMinBlockTokens = 32;
+
+// b[i] += gamma * sign(T*k - N*counts[i]) for i < N (one block).
+cudaError_t launch_bias_update(float* b, const int32_t* counts, int64_t Tk, int N, float gamma, cudaStream_t s);
 
 // Router GEMM on the tensor cores (bf16 x): splits W_r into the three
 // bf16 slabs at `split` (router_split_bytes) and writes fp32 logits (+ bias) to

@@ -119,7 +119,7 @@ moe_status_t derive(const moe_config_t* cfg, Dims* D) {
 // Workspace layout.  The first bytes (flags word, route ticket, route count and
 // z accumulators) are zeroed by one memset at the start of every routing call.
 struct Layout {
-  size_t flags, rticket, rcnt, rz, zero_end, rsplit, rlogits, dmask, dbase, dcounts, dticket, op_end;
+  size_t flags, rticket, rcnt, rz, zero_end, rzl, rsplit, rlogits, dmask, dbase, dcounts, dticket, op_end;
   size_t idx, w, row_map, seg_off, seg_count, xp, h, hs, sh, layer_end;
 };
 
@@ -138,6 +138,7 @@ Layout layout(const Dims& D) {
   L.rcnt = take(sizeof(int32_t) * D.N);
   L.rz = take(sizeof(unsigned long long) * D.N);
   L.zero_end = o;
+  L.rzl = take(sizeof(double) * ((D.T + kRouteMinBlockTokens - 1) / kRouteMinBlockTokens));
   const bool tc_router = D.bf16 && D.N >= kRouterTcMinExperts;
   L.rsplit = take(tc_router ? router_split_bytes(D.d, D.N) : 0);
   L.rlogits = take(tc_router ? sizeof(float) * kRouterMaxPartials * D.T * D.N : 0);
@@ -173,12 +174,13 @@ moe_status_t check_ws(void* ws, size_t ws_bytes, size_t need) {
 }
 
 bool route_stats_requested(const moe_stats_t* s) {
-  return s != nullptr && (s->y_frac || s->z_mean || s->l_aux_p3 || s->l_aux_switch || s->counts);
+  return s != nullptr && (s->y_frac || s->z_mean || s->l_aux_p3 || s->l_aux_switch || s->counts || s->z_loss ||
+                          s->load_std || s->top2_ratio);
 }
 
 moe_status_t do_route(const Dims& D, const void* x, const float* w_router, const float* bias,
-                      const float* logits_in, float* logits_out, int32_t* topk_idx, float* topk_w,
-                      const moe_stats_t* stats, void* ws, cudaStream_t st) {
+                      const float* sel_bias, const float* logits_in, float* logits_out, int32_t* topk_idx,
+                      float* topk_w, const moe_stats_t* stats, void* ws, cudaStream_t st) {
   const Layout L = layout(D);
   cudaError_t e = cudaMemsetAsync(ws, 0, L.zero_end, st);
   if (e != cudaSuccess) return cuda_status(e);
@@ -191,6 +193,9 @@ moe_status_t do_route(const Dims& D, const void* x, const float* w_router, const
       if (e == cudaSuccess && s.counts) e = cudaMemsetAsync(s.counts, 0, sizeof(int32_t) * D.N, st);
       if (e == cudaSuccess && s.l_aux_p3) e = cudaMemsetAsync(s.l_aux_p3, 0, sizeof(float), st);
       if (e == cudaSuccess && s.l_aux_switch) e = cudaMemsetAsync(s.l_aux_switch, 0, sizeof(float), st);
+      if (e == cudaSuccess && s.z_loss) e = cudaMemsetAsync(s.z_loss, 0, sizeof(float), st);
+      if (e == cudaSuccess && s.load_std) e = cudaMemsetAsync(s.load_std, 0, sizeof(float), st);
+      if (e == cudaSuccess && s.top2_ratio) e = cudaMemsetAsync(s.top2_ratio, 0, sizeof(float), st);
     }
     return cuda_status(e);
   }
@@ -203,6 +208,7 @@ moe_status_t do_route(const Dims& D, const void* x, const float* w_router, const
   a.x = x;
   a.w_router = w_router;
   a.bias = bias;
+  a.sel_bias = sel_bias;
   a.logits_in = logits_in;
   a.logits_out = logits_out;
   a.topk_idx = topk_idx;
@@ -210,6 +216,7 @@ moe_status_t do_route(const Dims& D, const void* x, const float* w_router, const
   a.cnt_acc = at<int32_t*>(ws, L.rcnt);
   a.z_acc = at<unsigned long long*>(ws, L.rz);
   a.ticket = at<uint32_t*>(ws, L.rticket);
+  a.zl_part = at<double*>(ws, L.rzl);
   a.want_stats = want_stats ? 1 : 0;
   if (want_stats) a.stats = *stats;
   a.flags = at<uint32_t*>(ws, L.flags);
@@ -238,6 +245,8 @@ moe_status_t do_dispatch(const Dims& D, const void* x, const int32_t* topk_idx, 
     if (e == cudaSuccess && stats && stats->counts) e = cudaMemsetAsync(stats->counts, 0, 4 * D.N, st);
     if (e == cudaSuccess && stats && stats->kept) e = cudaMemsetAsync(stats->kept, 0, 4 * D.N, st);
     if (e == cudaSuccess && stats && stats->num_dropped) e = cudaMemsetAsync(stats->num_dropped, 0, 4, st);
+    if (e == cudaSuccess && stats && stats->avg_tokens_per_expert)
+      e = cudaMemsetAsync(stats->avg_tokens_per_expert, 0, 4, st);
     return cuda_status(e);
   }
   DispatchArgs a{};
@@ -348,6 +357,7 @@ moe_status_t dispatch_empty(const DispatchArgs& a, cudaStream_t st) {
   if (e == cudaSuccess && a.stats.counts) e = cudaMemsetAsync(a.stats.counts, 0, 4 * a.N, st);
   if (e == cudaSuccess && a.stats.kept) e = cudaMemsetAsync(a.stats.kept, 0, 4 * a.N, st);
   if (e == cudaSuccess && a.stats.num_dropped) e = cudaMemsetAsync(a.stats.num_dropped, 0, 4, st);
+  if (e == cudaSuccess && a.stats.avg_tokens_per_expert) e = cudaMemsetAsync(a.stats.avg_tokens_per_expert, 0, 4, st);
   return cuda_status(e);
 }
 
@@ -396,8 +406,8 @@ moe_status_t moe_workspace_size(const moe_config_t* cfg, size_t* layer_bytes, si
 }
 
 moe_status_t moe_route(const moe_config_t* cfg, const void* x, const float* w_router, const float* router_bias,
-                       float* logits_out, int32_t* topk_idx, float* topk_w, moe_stats_t* stats, void* ws,
-                       size_t ws_bytes, moe_stream_t stream) {
+                       const float* selection_bias, float* logits_out, int32_t* topk_idx, float* topk_w,
+                       moe_stats_t* stats, void* ws, size_t ws_bytes, moe_stream_t stream) {
   Dims D;
   moe_status_t s = derive(cfg, &D);
   if (s != MOE_OK) return s;
@@ -405,19 +415,30 @@ moe_status_t moe_route(const moe_config_t* cfg, const void* x, const float* w_ro
     return MOE_ERR_INVALID_ARG;
   if (!aligned16(x)) return MOE_ERR_MISALIGNED;
   if ((s = check_ws(ws, ws_bytes, layout(D).op_end)) != MOE_OK) return s;
-  return do_route(D, x, w_router, router_bias, nullptr, logits_out, topk_idx, topk_w, stats, ws,
+  return do_route(D, x, w_router, router_bias, selection_bias, nullptr, logits_out, topk_idx, topk_w, stats, ws,
                   reinterpret_cast<cudaStream_t>(stream));
 }
 
-moe_status_t moe_route_from_logits(const moe_config_t* cfg, const float* logits, int32_t* topk_idx, float* topk_w,
-                                   moe_stats_t* stats, void* ws, size_t ws_bytes, moe_stream_t stream) {
+moe_status_t moe_route_from_logits(const moe_config_t* cfg, const float* logits, const float* selection_bias,
+                                   int32_t* topk_idx, float* topk_w, moe_stats_t* stats, void* ws,
+                                   size_t ws_bytes, moe_stream_t stream) {
   Dims D;
   moe_status_t s = derive(cfg, &D);
   if (s != MOE_OK) return s;
   if (D.T > 0 && (logits == nullptr || topk_idx == nullptr || topk_w == nullptr)) return MOE_ERR_INVALID_ARG;
   if ((s = check_ws(ws, ws_bytes, layout(D).op_end)) != MOE_OK) return s;
-  return do_route(D, nullptr, nullptr, nullptr, logits, nullptr, topk_idx, topk_w, stats, ws,
+  return do_route(D, nullptr, nullptr, nullptr, selection_bias, logits, nullptr, topk_idx, topk_w, stats, ws,
                   reinterpret_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_bias_update(const moe_config_t* cfg, float* selection_bias, const int32_t* counts, float gamma,
+                             moe_stream_t stream) {
+  Dims D;
+  moe_status_t s = derive(cfg, &D);
+  if (s != MOE_OK) return s;
+  if (selection_bias == nullptr || counts == nullptr || !std::isfinite(gamma)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_bias_update(selection_bias, counts, D.T * D.k, D.N, gamma,
+                                        reinterpret_cast<cudaStream_t>(stream)));
 }
 
 moe_status_t moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* topk_idx, int32_t* row_map,
@@ -505,8 +526,8 @@ moe_status_t moe_layer_fwd(const moe_config_t* cfg, const moe_weights_t* weights
   void* out_rows = xp;  // the permuted rows are dead once GEMM1 has read them
   void* shared_out = D.fs ? at<void*>(ws, L.sh) : nullptr;
 
-  if ((s = do_route(D, x, weights->w_router, weights->router_bias, nullptr, nullptr, idx, w, stats, ws, st)) !=
-      MOE_OK)
+  if ((s = do_route(D, x, weights->w_router, weights->router_bias, weights->selection_bias, nullptr, nullptr, idx, w,
+                    stats, ws, st)) != MOE_OK)
     return s;
   if ((s = do_dispatch(D, x, idx, row_map, seg_off, seg_count, xp, stats, ws, st)) != MOE_OK) return s;
   if ((s = do_ffn(D, xp, seg_off, seg_count, weights->w1, weights->w3, weights->w2, D.f, false, h, out_rows, ws,

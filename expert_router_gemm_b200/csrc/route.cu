@@ -42,6 +42,7 @@ struct RouteSmem {
     float lg[BT][NP + 1];
   } u;
   float zw[kRouteThreads / 32][NP];
+  double zl[kRouteThreads / 32];
   int hist[NP];
 };
 
@@ -66,6 +67,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
   static_assert(FROM_LOGITS || BT == route_bt(NP), "route block size mismatch");
   static_assert(BT <= S::BT, "the logits tile holds at most S::BT tokens");
   static_assert(NP / TX == 8, "each thread owns 8 experts");
+  static_assert(BT >= kRouteMinBlockTokens, "z-loss partials are sized for 32-token blocks");
   __shared__ __align__(16) S sm;
 
   const int tid = threadIdx.x;
@@ -188,6 +190,15 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
   float zacc[NPL];
 #pragma unroll
   for (int c = 0; c < NPL; ++c) zacc[c] = 0.f;
+  double zl = 0.0;  // this warp's sum of logsumexp^2 (every lane holds the same value)
+  // Aux-Loss-Free selection bias of the lane's experts (0 where there is none)
+  const bool biased = a.sel_bias != nullptr;
+  float sb[NPL];
+#pragma unroll
+  for (int c = 0; c < NPL; ++c) {
+    const int e = lane + 32 * c;
+    sb[c] = (biased && e < N) ? a.sel_bias[e] : 0.f;
+  }
 
   for (int tl0 = warp * TPW; tl0 < BT; tl0 += NW * TPW) {
     float v[TPW][NPL], s[TPW][NPL];
@@ -231,6 +242,12 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
       for (int q = 0; q < TPW; ++q) sum[q] += __shfl_xor_sync(0xffffffffu, sum[q], o);
 #pragma unroll
     for (int q = 0; q < TPW; ++q)
+      if (valid[q]) {
+        const float lse = m[q] + logf(sum[q]);  // log-partition of the unbiased logits
+        zl += static_cast<double>(lse) * lse;
+      }
+#pragma unroll
+    for (int q = 0; q < TPW; ++q)
 #pragma unroll
       for (int c = 0; c < NPL; ++c) {
         if (valid[q]) {
@@ -240,19 +257,21 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
         if (isnan(v[q][c])) v[q][c] = -INFINITY;  // out of contract; keeps the selection defined
       }
 
-    // top-k on the logits.  Each (logit, expert) becomes one 64-bit key whose
-    // unsigned order is "larger logit first, then lower expert index" (-0.0 is
-    // taken as +0.0 so equal logits tie).  A lane sorts its few keys; each round
-    // is one warp-wide max over the lanes' leading keys, and the winning lane
-    // drops its leading key.  The winner's weight is recomputed from its logit
-    // with the softmax's own expression.
+    // top-k on the logits (plus the selection bias, in fp32, when there is
+    // one).  Each (score, expert) becomes one 64-bit key whose unsigned order
+    // is "larger score first, then lower expert index" (-0.0 is taken as +0.0
+    // so equal scores tie).  A lane sorts its few keys; each round is one
+    // warp-wide max over the lanes' leading keys, and the winning lane drops
+    // its leading key.  The winner's weight is recomputed from its unbiased
+    // logit with the softmax's own expression.
     uint64_t key[TPW][NPL];
 #pragma unroll
     for (int q = 0; q < TPW; ++q) {
 #pragma unroll
       for (int c = 0; c < NPL; ++c) {
         const int e = lane + 32 * c;
-        key[q][c] = e < N ? (static_cast<uint64_t>(order_key(v[q][c])) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(e))
+        const float sel = biased ? v[q][c] + sb[c] : v[q][c];
+        key[q][c] = e < N ? (static_cast<uint64_t>(order_key(sel)) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(e))
                           : 0ull;
       }
 #pragma unroll
@@ -292,7 +311,8 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
           key[q][NPL - 1] = 0ull;
         }
         const int e = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(best[q]));
-        const float sv = expf(key_value(static_cast<uint32_t>(best[q] >> 32)) - m[q]) / sum[q];
+        const float ve = biased ? sm.u.lg[tl0 + q][e] : key_value(static_cast<uint32_t>(best[q] >> 32));
+        const float sv = expf(ve - m[q]) / sum[q];
         ssum[q] += sv;
         if (lane == j) {
           my_idx[q] = e;
@@ -321,6 +341,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
     const int e = lane + 32 * c;
     if (e < NP) sm.zw[warp][e] = zacc[c];
   }
+  if (lane == 0) sm.zl[warp] = zl;
   __syncthreads();
   for (int e = tid; e < N; e += kRouteThreads) {
     float z = 0.f;
@@ -328,6 +349,12 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
     for (int w = 0; w < NW; ++w) z += sm.zw[w][e];
     atomicAdd(a.z_acc + e, static_cast<unsigned long long>(__double2ull_rn(static_cast<double>(z) * 4294967296.0)));
     if (sm.hist[e] != 0) atomicAdd(a.cnt_acc + e, sm.hist[e]);
+  }
+  if (tid == 0) {  // the block's z-loss partial, summed over its warps in order
+    double t = 0.0;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) t += sm.zl[w];
+    a.zl_part[blockIdx.x] = t;
   }
   __threadfence();
   __syncthreads();
@@ -337,27 +364,73 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
   if (!is_last) return;
   __threadfence();
   double* prod = reinterpret_cast<double*>(&sm.u);   // the logits tile is no longer needed
+  const double tk = static_cast<double>(T) * k;
   for (int e = tid; e < N; e += kRouteThreads) {
     const int cnt = __ldcg(a.cnt_acc + e);
     const double zsum = static_cast<double>(__ldcg(a.z_acc + e)) * (1.0 / 4294967296.0);
-    const double y = static_cast<double>(cnt) / (static_cast<double>(T) * k);
+    const double y = static_cast<double>(cnt) / tk;
     const double zm = zsum / static_cast<double>(T);
     if (a.stats.counts) a.stats.counts[e] = cnt;
     if (a.stats.y_frac) a.stats.y_frac[e] = static_cast<float>(y);
     if (a.stats.z_mean) a.stats.z_mean[e] = static_cast<float>(zm);
     prod[e] = y * zm;
+    sm.hist[e] = cnt;
   }
   __syncthreads();
   if (warp == 0) {
-    double acc = 0.0;
-    for (int e = lane; e < N; e += 32) acc += prod[e];
+    // L_aux, and the load figures: std of the shares f_i, the two largest counts
+    double acc = 0.0, fsum = 0.0;
+    int c1 = 0, c2 = 0;  // largest and second largest count seen by this lane
+    for (int e = lane; e < N; e += 32) {
+      acc += prod[e];
+      fsum += static_cast<double>(sm.hist[e]) / tk;
+      const int c = sm.hist[e];
+      if (c > c1) {
+        c2 = c1;
+        c1 = c;
+      } else if (c > c2) {
+        c2 = c;
+      }
+    }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    for (int o = 16; o > 0; o >>= 1) {
+      acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      fsum += __shfl_xor_sync(0xffffffffu, fsum, o);
+      const int o1 = __shfl_xor_sync(0xffffffffu, c1, o), o2 = __shfl_xor_sync(0xffffffffu, c2, o);
+      const int hi = max(c1, o1), lo = max(min(c1, o1), max(c2, o2));
+      c1 = hi;
+      c2 = lo;
+    }
+    const double fmean = fsum / N;
+    double var = 0.0;
+    for (int e = lane; e < N; e += 32) {
+      const double dv = static_cast<double>(sm.hist[e]) / tk - fmean;
+      var += dv * dv;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) var += __shfl_xor_sync(0xffffffffu, var, o);
     if (lane == 0) {
       if (a.stats.l_aux_p3) a.stats.l_aux_p3[0] = static_cast<float>(static_cast<double>(T) / N * acc);
       if (a.stats.l_aux_switch) a.stats.l_aux_switch[0] = static_cast<float>(N * acc);
+      if (a.stats.load_std) a.stats.load_std[0] = static_cast<float>(sqrt(var / N));
+      if (a.stats.top2_ratio) a.stats.top2_ratio[0] = static_cast<float>(static_cast<double>(c1 + c2) / tk);
     }
+  } else if (warp == 1 && a.stats.z_loss != nullptr) {
+    // z-loss: the blocks' partials in block order (a fixed reduction tree)
+    double t = 0.0;
+    for (unsigned b = lane; b < gridDim.x; b += 32) t += __ldcg(a.zl_part + b);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+    if (lane == 0) a.stats.z_loss[0] = static_cast<float>(t / static_cast<double>(T));
   }
+}
+
+__global__ void bias_update_kernel(float* b, const int32_t* counts, int64_t Tk, int N, float gamma) {
+  const int i = threadIdx.x;
+  if (i >= N) return;
+  const int64_t diff = Tk - static_cast<int64_t>(N) * counts[i];
+  const float sgn = diff > 0 ? 1.f : diff < 0 ? -1.f : 0.f;
+  b[i] = __fadd_rn(b[i], gamma * sgn);  // gamma * sgn is exact: one rounding, as written
 }
 
 template <int NP>
@@ -372,6 +445,11 @@ cudaError_t launch_np(const RouteArgs& a, cudaStream_t s) {
 }
 
 }  // namespace
+
+cudaError_t launch_bias_update(float* b, const int32_t* counts, int64_t Tk, int N, float gamma, cudaStream_t s) {
+  bias_update_kernel<<<1, 256, 0, s>>>(b, counts, Tk, N, gamma);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t s) {
   if (a.T == 0) return cudaSuccess;

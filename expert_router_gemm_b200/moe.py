@@ -39,12 +39,14 @@ class moe_config_t(ctypes.Structure):
 
 class moe_weights_t(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
-                ("w_router", "router_bias", "w1", "w3", "w2", "ws1", "ws3", "ws2")]
+                ("w_router", "router_bias", "w1", "w3", "w2", "ws1", "ws3", "ws2",
+                 "selection_bias")]
 
 
 class moe_stats_t(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
-                ("y_frac", "z_mean", "l_aux_p3", "l_aux_switch", "counts", "kept", "num_dropped")]
+                ("y_frac", "z_mean", "l_aux_p3", "l_aux_switch", "counts", "kept", "num_dropped",
+                 "z_loss", "load_std", "top2_ratio", "avg_tokens_per_expert")]
 
 
 _P = ctypes.c_void_p
@@ -56,10 +58,11 @@ _PROTOS = {
     "moe_capacity": (ctypes.c_int, [ctypes.POINTER(moe_config_t), ctypes.POINTER(ctypes.c_int32)]),
     "moe_workspace_size": (ctypes.c_int, [ctypes.POINTER(moe_config_t), ctypes.POINTER(_SZ),
                                           ctypes.POINTER(_SZ), ctypes.POINTER(ctypes.c_int64)]),
-    "moe_route": (ctypes.c_int, [ctypes.POINTER(moe_config_t), _P, _P, _P, _P, _P, _P,
+    "moe_route": (ctypes.c_int, [ctypes.POINTER(moe_config_t), _P, _P, _P, _P, _P, _P, _P,
                                  ctypes.POINTER(moe_stats_t), _P, _SZ, _P]),
-    "moe_route_from_logits": (ctypes.c_int, [ctypes.POINTER(moe_config_t), _P, _P, _P,
+    "moe_route_from_logits": (ctypes.c_int, [ctypes.POINTER(moe_config_t), _P, _P, _P, _P,
                                              ctypes.POINTER(moe_stats_t), _P, _SZ, _P]),
+    "moe_bias_update": (ctypes.c_int, [ctypes.POINTER(moe_config_t), _P, _P, ctypes.c_float, _P]),
     "moe_dispatch": (ctypes.c_int, [ctypes.POINTER(moe_config_t), _P, _P, _P, _P, _P, _P,
                                     ctypes.POINTER(moe_stats_t), _P, _SZ, _P]),
     "moe_dispatch_static": (ctypes.c_int, [ctypes.POINTER(moe_config_t), _P, _P, _P, _P, _P, _P,
@@ -134,14 +137,17 @@ def config_from_workload(w, T: Optional[int] = None, **over) -> moe_config_t:
 
 
 def make_weights(w_router, router_bias=None, w1=None, w3=None, w2=None, ws1=None, ws3=None,
-                 ws2=None) -> moe_weights_t:
-    return moe_weights_t(*[_ptr(t) for t in (w_router, router_bias, w1, w3, w2, ws1, ws3, ws2)])
+                 ws2=None, selection_bias=None) -> moe_weights_t:
+    return moe_weights_t(*[_ptr(t) for t in (w_router, router_bias, w1, w3, w2, ws1, ws3, ws2,
+                                            selection_bias)])
 
 
 def make_stats(y_frac=None, z_mean=None, l_aux_p3=None, l_aux_switch=None, counts=None,
-               kept=None, num_dropped=None) -> moe_stats_t:
+               kept=None, num_dropped=None, z_loss=None, load_std=None, top2_ratio=None,
+               avg_tokens_per_expert=None) -> moe_stats_t:
     return moe_stats_t(*[_ptr(t) for t in (y_frac, z_mean, l_aux_p3, l_aux_switch, counts, kept,
-                                            num_dropped)])
+                                            num_dropped, z_loss, load_std, top2_ratio,
+                                            avg_tokens_per_expert)])
 
 
 # ---------------------------------------------------------------- the C-ABI calls
@@ -171,19 +177,25 @@ def _stats_ref(stats: Optional[moe_stats_t]):
     return ctypes.byref(stats) if stats is not None else None
 
 
-def moe_route(cfg, x, w_router, router_bias, logits_out, topk_idx, topk_w, stats, ws,
-              stream=None):
+def moe_route(cfg, x, w_router, router_bias, selection_bias, logits_out, topk_idx, topk_w, stats,
+              ws, stream=None):
     _check(_lib.moe_route(ctypes.byref(cfg), _ptr(x), _ptr(w_router), _ptr(router_bias),
-                          _ptr(logits_out), _ptr(topk_idx), _ptr(topk_w), _stats_ref(stats),
-                          _ptr(ws), ws.numel() if ws is not None else 0, _stream(stream)),
+                          _ptr(selection_bias), _ptr(logits_out), _ptr(topk_idx), _ptr(topk_w),
+                          _stats_ref(stats), _ptr(ws), ws.numel() if ws is not None else 0,
+                          _stream(stream)),
            "moe_route")
 
 
-def moe_route_from_logits(cfg, logits, topk_idx, topk_w, stats, ws, stream=None):
-    _check(_lib.moe_route_from_logits(ctypes.byref(cfg), _ptr(logits), _ptr(topk_idx),
-                                      _ptr(topk_w), _stats_ref(stats), _ptr(ws),
+def moe_route_from_logits(cfg, logits, selection_bias, topk_idx, topk_w, stats, ws, stream=None):
+    _check(_lib.moe_route_from_logits(ctypes.byref(cfg), _ptr(logits), _ptr(selection_bias),
+                                      _ptr(topk_idx), _ptr(topk_w), _stats_ref(stats), _ptr(ws),
                                       ws.numel() if ws is not None else 0, _stream(stream)),
            "moe_route_from_logits")
+
+
+def moe_bias_update(cfg, selection_bias, counts, gamma: float, stream=None):
+    _check(_lib.moe_bias_update(ctypes.byref(cfg), _ptr(selection_bias), _ptr(counts),
+                                ctypes.c_float(gamma), _stream(stream)), "moe_bias_update")
 
 
 def moe_dispatch(cfg, x, topk_idx, row_map, seg_off, seg_count, xp, stats, ws, stream=None):
@@ -260,10 +272,11 @@ class DeviceLayer:
     ws1: Optional[torch.Tensor] = None
     ws3: Optional[torch.Tensor] = None
     ws2: Optional[torch.Tensor] = None
+    selection_bias: Optional[torch.Tensor] = None
 
     def weights(self) -> moe_weights_t:
         return make_weights(self.w_router, self.bias, self.w1, self.w3, self.w2,
-                            self.ws1, self.ws3, self.ws2)
+                            self.ws1, self.ws3, self.ws2, self.selection_bias)
 
 
 def to_device(inputs, cfg: moe_config_t, device="cuda") -> DeviceLayer:

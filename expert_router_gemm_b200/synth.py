@@ -27,7 +27,7 @@ import numpy as np
 from .configs import Workload
 
 # stream ids: tensor id in the high bits, expert index in the low 20 bits
-_X, _WR, _W1, _W3, _W2, _WS1, _WS3, _WS2, _LOGITS = range(1, 10)
+_X, _WR, _W1, _W3, _W2, _WS1, _WS3, _WS2, _LOGITS, _SELBIAS = range(1, 11)
 
 
 def _stream(tensor_id: int, sub: int = 0) -> int:
@@ -157,4 +157,23 @@ def make_logits(seed: int, T: int, N: int, pattern: str = "normal") -> np.ndarra
         g = normal_f32(seed, _stream(_LOGITS, 3), (T, N))
         g += np.linspace(2.0, -2.0, N, dtype=np.float32)[None, :]
         return g
+    raise ValueError(pattern)
+
+
+def make_selection_bias(seed: int, N: int, pattern: str = "normal") -> np.ndarray:
+    """Synthetic fp32 per-expert selection bias [N] (Aux-Loss-Free routing).
+
+    pattern:
+      "normal"  - N(0, 0.5^2)
+      "dyadic"  - multiples of 1/4 in [-1, 1] (exact sums with the "ties" logits,
+                  so biased scores tie too)
+      "zeros"   - all zero (must route exactly as without a bias)
+    """
+    if pattern == "normal":
+        return normal_f32(seed, _stream(_SELBIAS, 0), (N,)) * np.float32(0.5)
+    if pattern == "dyadic":
+        b = normal_f32(seed, _stream(_SELBIAS, 1), (N,))
+        return (np.clip(np.rint(b * 2.0), -4, 4) / 4.0).astype(np.float32)
+    if pattern == "zeros":
+        return np.zeros((N,), dtype=np.float32)
     raise ValueError(pattern)

@@ -96,6 +96,9 @@ typedef struct {
   const void* ws1;           /* [d][f_shared] act, shared expert gate; NULL if f_shared == 0 */
   const void* ws3;           /* [d][f_shared] act, shared expert up */
   const void* ws2;           /* [f_shared][d] act, shared expert down */
+  const float* selection_bias; /* [N] fp32 Aux-Loss-Free bias, added to g for the top-k
+                                  choice only (the weights use the unbiased softmax);
+                                  NULL = none.  Update it with moe_bias_update(). */
 } moe_weights_t;
 
 /* Load-balance and capacity statistics.  Device pointers; each may be NULL. */
@@ -107,6 +110,12 @@ typedef struct {
   int32_t* counts;      /* [N] top-k selections per expert before the drop */
   int32_t* kept;        /* [N] min(counts, C) */
   int32_t* num_dropped; /* [1] sum_i (counts_i - kept_i) */
+  /* Router z-loss and load-health figures ("负载均衡策略", hyper-parameter table,
+     z_loss_weight; "ms-swift + Megatron：MoE模型加速10倍实测" §3.3 "监控与诊断"). */
+  float* z_loss;        /* [1] mean over tokens of (log sum_i exp g_ti)^2 (unbiased g) */
+  float* load_std;      /* [1] population std over experts of counts_i / (T*k) */
+  float* top2_ratio;    /* [1] share of the T*k selections taken by the two busiest experts */
+  float* avg_tokens_per_expert; /* [1] sum_i kept_i / N (filled by the dispatch step) */
 } moe_stats_t;
 
 /* Human-readable name of a status. Never NULL. */
@@ -150,25 +159,43 @@ moe_status_t moe_workspace_size(const moe_config_t* cfg, size_t* layer_bytes,
  * weight_j = s_{idx_j} / sum_{j'} s_{idx_j'}.
  *   x          [T, d] act          input tokens (read)
  *   w_router   [d, N] fp32, bias [N] fp32 or NULL
- *   logits_out [T, N] fp32 or NULL: g including the bias
+ *   selection_bias [N] fp32 or NULL: Aux-Loss-Free bias ("MoE 训练加速实战" §5.3):
+ *              the experts are ranked on the fp32 sum g + selection_bias, while the
+ *              weights, z_i and the z-loss use the unbiased g
+ *   logits_out [T, N] fp32 or NULL: g including the bias (never the selection bias)
  *   topk_idx   [T, k] int32 (written), topk_w [T, k] fp32 (written)
- *   stats      may be NULL: fills y_frac, z_mean, l_aux_p3, l_aux_switch, counts
+ *   stats      may be NULL: fills y_frac, z_mean, l_aux_p3, l_aux_switch, counts,
+ *              z_loss, load_std, top2_ratio
  *   ws         op workspace (>= op_bytes); its flags word is cleared first.
  * Non-finite logits raise MOE_FLAG_NONFINITE_LOGITS (read with moe_read_flags).
  */
 moe_status_t moe_route(const moe_config_t* cfg, const void* x, const float* w_router,
-                       const float* router_bias, float* logits_out, int32_t* topk_idx,
-                       float* topk_w, moe_stats_t* stats, void* ws, size_t ws_bytes,
-                       moe_stream_t stream);
+                       const float* router_bias, const float* selection_bias, float* logits_out,
+                       int32_t* topk_idx, float* topk_w, moe_stats_t* stats, void* ws,
+                       size_t ws_bytes, moe_stream_t stream);
 
 /*
  * moe_route_from_logits - the same softmax / top-k / weights / statistics as
- * moe_route, starting from caller-supplied fp32 logits [T, N] (no GEMM).  This is
- * the entry point on which routing is compared bit-for-bit with a reference.
+ * moe_route, starting from caller-supplied fp32 logits [T, N] (no GEMM), with
+ * an optional selection_bias [N] as in moe_route.  This is the entry point on
+ * which routing is compared bit-for-bit with a reference.
  */
 moe_status_t moe_route_from_logits(const moe_config_t* cfg, const float* logits,
-                                   int32_t* topk_idx, float* topk_w, moe_stats_t* stats,
-                                   void* ws, size_t ws_bytes, moe_stream_t stream);
+                                   const float* selection_bias, int32_t* topk_idx,
+                                   float* topk_w, moe_stats_t* stats, void* ws,
+                                   size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * moe_bias_update - one Aux-Loss-Free bias step ("MoE 训练加速实战" §5.4):
+ *   selection_bias[i] += gamma * sign(1/N - f_i),   f_i = counts[i] / (T*k),
+ * with the sign taken exactly on integers, sign(T*k - N*counts[i]), and one fp32
+ * addition.  counts [N] int32 are a routing call's top-k selections before the
+ * capacity drop (moe_stats_t.counts of moe_route / moe_layer_fwd on the same
+ * cfg).  selection_bias [N] fp32 is read and written in place on `stream`.
+ * Errors: MOE_ERR_INVALID_ARG for NULL pointers, a bad cfg or a non-finite gamma.
+ */
+moe_status_t moe_bias_update(const moe_config_t* cfg, float* selection_bias, const int32_t* counts,
+                             float gamma, moe_stream_t stream);
 
 /*
  * moe_dispatch - capacity clip and permutation into expert-contiguous rows.
@@ -184,7 +211,7 @@ moe_status_t moe_route_from_logits(const moe_config_t* cfg, const float* logits,
  *   seg_count [N] int32 (written): kept rows of each expert = min(count, C)
  *   xp        [max_rows, d] act (written): xp[row_map[t][j]] = x[t] bit for bit;
  *             rows between segments are not written
- *   stats     may be NULL: fills counts, kept, num_dropped
+ *   stats     may be NULL: fills counts, kept, num_dropped, avg_tokens_per_expert
  * An index outside [0, N) or repeated in a row raises MOE_FLAG_BAD_EXPERT_INDEX;
  * that slot is dropped.
  */
@@ -265,8 +292,10 @@ moe_status_t moe_combine(const moe_config_t* cfg, const void* out_rows, const in
 /*
  * moe_layer_fwd - the whole layer: route, dispatch, routed experts, shared
  * expert (if cfg->f_shared > 0), combine.  x [T, d] act (read), y [T, d] act
- * (written), stats may be NULL, ws >= layer_bytes of moe_workspace_size.  The
- * permuted rows and the expert outputs share one workspace region.
+ * (written), stats may be NULL (every field is filled), ws >= layer_bytes of
+ * moe_workspace_size.  weights->selection_bias (may be NULL) steers the top-k
+ * choice as in moe_route; the layer does not update it.  The permuted rows and
+ * the expert outputs share one workspace region.
  */
 moe_status_t moe_layer_fwd(const moe_config_t* cfg, const moe_weights_t* weights,
                            const void* x, void* y, moe_stats_t* stats, void* ws,

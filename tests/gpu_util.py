@@ -30,7 +30,11 @@ def new_stats(N):
                 l_aux_switch=torch.full((1,), NAN, dtype=F32, device="cuda"),
                 counts=torch.full((N,), -9, dtype=I32, device="cuda"),
                 kept=torch.full((N,), -9, dtype=I32, device="cuda"),
-                num_dropped=torch.full((1,), -9, dtype=I32, device="cuda"))
+                num_dropped=torch.full((1,), -9, dtype=I32, device="cuda"),
+                z_loss=torch.full((1,), NAN, dtype=F32, device="cuda"),
+                load_std=torch.full((1,), NAN, dtype=F32, device="cuda"),
+                top2_ratio=torch.full((1,), NAN, dtype=F32, device="cuda"),
+                avg_tokens_per_expert=torch.full((1,), NAN, dtype=F32, device="cuda"))
     return bufs, moe.make_stats(**bufs)
 
 
@@ -43,14 +47,15 @@ def op_workspace(cfg):
     return torch.zeros(ob, dtype=U8, device="cuda")
 
 
-def route_from_logits(cfg, logits: np.ndarray):
+def route_from_logits(cfg, logits: np.ndarray, selection_bias=None):
     T, N, k = cfg.T, cfg.N, cfg.k
     lg = cuda_tensor(logits.astype(np.float32))
     idx = torch.full((T, k), -7, dtype=I32, device="cuda")
     w = torch.full((T, k), NAN, dtype=F32, device="cuda")
     ws = op_workspace(cfg)
     bufs, st = new_stats(N)
-    moe.moe_route_from_logits(cfg, lg, idx, w, st, ws)
+    sb = None if selection_bias is None else cuda_tensor(np.asarray(selection_bias, np.float32))
+    moe.moe_route_from_logits(cfg, lg, sb, idx, w, st, ws)
     flags = moe.moe_read_flags(ws)
     return host(idx), host(w), stats_host(bufs), flags
 
@@ -82,7 +87,7 @@ def staged_layer(dl: moe.DeviceLayer):
     idx = torch.full((T, k), -7, dtype=I32, device="cuda")
     w = torch.full((T, k), NAN, dtype=F32, device="cuda")
     bufs, st = new_stats(N)
-    moe.moe_route(cfg, dl.x, dl.w_router, dl.bias, logits, idx, w, st, ws)
+    moe.moe_route(cfg, dl.x, dl.w_router, dl.bias, dl.selection_bias, logits, idx, w, st, ws)
     row_map = torch.full((T, k), -7, dtype=I32, device="cuda")
     seg_off = torch.full((N + 1,), -7, dtype=I32, device="cuda")
     seg_count = torch.full((N,), -7, dtype=I32, device="cuda")

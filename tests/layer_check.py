@@ -36,23 +36,51 @@ def logit_bound(x, w_router, bias=None):
     return (3 * xa.shape[1] + 2) * U32 * s + 1e-7
 
 
-def oracle_routing(inp, w, align=128, cap=None):
+def z_loss_tolerance(g64, N):
+    """Bound on |z-loss(GPU) - z-loss(oracle)| for fp32 logits g64 (as float64).
+
+    Per token the GPU forms lse = m + log(sum_i exp(g_i - m)) in fp32: the sum of
+    at most N exponentials (each within 2 ulp) over at most N/32 + 5 sequential
+    and butterfly additions has relative error below (N/32 + 9) u, so log(sum)
+    is off by that much plus one ulp of log N; adding m rounds once more.  With
+    delta_t that bound, (lse + delta)^2 - lse^2 <= 2 |lse| delta + delta^2; the
+    mean over tokens then sums in double (negligible)."""
+    m = g64.max(axis=1)
+    lse = m + np.log(np.exp(g64 - m[:, None]).sum(axis=1))
+    delta = (N / 32 + 9) * U32 + 2 * U32 * (np.abs(lse) + np.log(N) + 1)
+    return float(np.mean(2 * np.abs(lse) * delta + delta ** 2)) * 2 + 1e-12
+
+
+def check_route_extras(st, g64, idx, T, k, N):
+    """The router z-loss and the load figures of a routing call's statistics."""
+    zl = orc.router_z_loss(g64)
+    assert abs(float(st["z_loss"][0]) - zl) <= z_loss_tolerance(g64, N), (st["z_loss"][0], zl)
+    counts = np.bincount(idx.reshape(-1), minlength=N)
+    ref = orc.load_metrics(counts, counts, T, k)
+    np.testing.assert_allclose(st["load_std"][0], ref.load_std, rtol=1e-6, atol=1e-9)
+    assert st["top2_ratio"][0] == np.float32(ref.top2_ratio), (st["top2_ratio"][0], ref.top2_ratio)
+
+
+def oracle_routing(inp, w, align=128, cap=None, selection_bias=None):
     return orc.layer_forward(inp.x, inp.w_router, inp.bias, inp.w1, inp.w3, inp.w2, k=w.k,
                              capacity_factor=w.capacity_factor, cap=cap, bf16=inp.bf16,
-                             align=align, tokens=[])
+                             align=align, tokens=[], selection_bias=selection_bias)
 
 
 def compare_layer(inp, w, gpu_y, gpu_idx, gpu_row_map, gpu_logits=None, tol=2e-2,
-                  sample=None, seed=0, align=128, cap=None):
-    """Returns (rel_frobenius, n_compared, n_flips)."""
+                  sample=None, seed=0, align=128, cap=None, selection_bias=None):
+    """Returns (rel_frobenius, n_compared, n_flips).  With a selection bias the
+    near-tie test runs on the biased scores that decide the choice."""
     T = inp.x.shape[0]
-    ref = oracle_routing(inp, w, align, cap)
+    ref = oracle_routing(inp, w, align, cap, selection_bias)
     bound = logit_bound(inp.x, inp.w_router, inp.bias)
     if gpu_logits is not None:
         err = np.abs(gpu_logits.astype(np.float64) - ref.logits)
         assert np.all(err <= bound), f"router logits differ by {err.max():.3g}"
 
     g = ref.logits
+    if selection_bias is not None:
+        g = g + np.asarray(selection_bias, np.float64)[None, :]
     o_sets = [set(r) for r in ref.idx.tolist()]
     g_sets = [set(r) for r in gpu_idx.tolist()]
     flips = [t for t in range(T) if o_sets[t] != g_sets[t]]
@@ -86,7 +114,7 @@ def compare_layer(inp, w, gpu_y, gpu_idx, gpu_row_map, gpu_logits=None, tol=2e-2
     res = orc.layer_forward(inp.x, inp.w_router, inp.bias, inp.w1, inp.w3, inp.w2, k=w.k,
                             capacity_factor=w.capacity_factor, cap=cap, bf16=inp.bf16,
                             ws1=inp.ws1, ws3=inp.ws3, ws2=inp.ws2, align=align, tokens=good,
-                            logits=ref.logits)
+                            logits=ref.logits, selection_bias=selection_bias)
     y = gpu_y[good]
     if y.dtype == np.uint16:
         y = (y.astype(np.uint32) << np.uint32(16)).view(np.float32)

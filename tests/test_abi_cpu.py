@@ -108,7 +108,7 @@ def test_workspace_size_and_shape_checks():
 def _route_status(cfg, x=0x10000, wr=0x20000, idx=0x30000, w=0x40000, ws=0x50000, ws_bytes=None):
     if ws_bytes is None:
         ws_bytes = moe.moe_workspace_size(cfg)[1]
-    return moe.raw_call("moe_route", ctypes.byref(cfg), x, wr, None, None, idx, w, None, ws,
+    return moe.raw_call("moe_route", ctypes.byref(cfg), x, wr, None, None, None, idx, w, None, ws,
                         ctypes.c_size_t(ws_bytes), None)
 
 
@@ -122,6 +122,20 @@ def test_route_argument_validation():
     assert _route_status(cfg, ws=0x50008) == MISAL
     bad = moe.make_config(T=256, d=128, N=8, k=9, f=256)
     assert _route_status(bad, ws_bytes=1 << 20) == INVALID
+
+
+def test_bias_update_argument_validation():
+    cfg = moe.make_config(T=256, d=128, N=8, k=2, f=256, capacity_factor=1.25)
+    f = ctypes.c_float
+
+    def call(c, b=0x10000, counts=0x20000, gamma=1e-3):
+        return moe.raw_call("moe_bias_update", ctypes.byref(c), b, counts, f(gamma), None)
+
+    assert call(cfg, b=None) == INVALID
+    assert call(cfg, counts=None) == INVALID
+    assert call(cfg, gamma=float("nan")) == INVALID
+    assert call(cfg, gamma=float("inf")) == INVALID
+    assert call(moe.make_config(T=256, d=128, N=8, k=9, f=256)) == INVALID
 
 
 def test_other_entry_points_validate():

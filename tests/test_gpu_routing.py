@@ -19,7 +19,7 @@ if not torch.cuda.is_available():
 
 from expert_router_gemm_b200 import moe  # noqa: E402
 from tests import gpu_util as gu  # noqa: E402
-from tests.layer_check import logit_bound  # noqa: E402
+from tests.layer_check import check_route_extras, logit_bound  # noqa: E402
 
 W_RTOL = 2e-6
 
@@ -40,6 +40,7 @@ def _check_route(T, N, k, pattern, seed=0):
     np.testing.assert_allclose(st["z_mean"], ref.z_mean, rtol=1e-5, atol=1e-7)
     np.testing.assert_allclose(st["l_aux_p3"][0], ref.l_aux_p3, rtol=1e-5)
     np.testing.assert_allclose(st["l_aux_switch"][0], ref.l_aux_switch, rtol=1e-5)
+    check_route_extras(st, g, want_idx, T, k, N)
 
 
 @pytest.mark.parametrize("N,k", [(8, 1), (8, 2), (8, 8), (5, 3), (16, 4), (33, 7), (64, 32),
@@ -80,7 +81,7 @@ def test_route_gemm_logits(T, d, N, k, dtype, bias):
     wt = torch.zeros((T, k), device="cuda")
     ws = gu.op_workspace(cfg)
     moe.moe_route(cfg, gu.cuda_tensor(x), gu.cuda_tensor(wr), None if b is None else gu.cuda_tensor(b),
-                  logits, idx, wt, None, ws)
+                  None, logits, idx, wt, None, ws)
     assert moe.moe_read_flags(ws) == 0
     g = gu.host(logits).astype(np.float64)
     ref = orc.router_logits(x, wr, b)
@@ -115,7 +116,7 @@ def test_route_gemm_exact_on_one_hot_tokens(d, N, bias):
     wt = torch.empty((T, cfg.k), device="cuda")
     ws = gu.op_workspace(cfg)
     moe.moe_route(cfg, gu.cuda_tensor(x), gu.cuda_tensor(wr), None if b is None else gu.cuda_tensor(b),
-                  logits, idx, wt, None, ws)
+                  None, logits, idx, wt, None, ws)
     want = wr[np.arange(T) % d]
     if b is not None:
         want = want + b[None, :]          # one fp32 addition, round to nearest
@@ -153,6 +154,8 @@ def _check_dispatch(T, N, k, d, cap, align, dtype, pattern, seed=0):
     np.testing.assert_array_equal(r["stats"]["counts"], want.counts)
     np.testing.assert_array_equal(r["stats"]["kept"], want.kept)
     assert int(r["stats"]["num_dropped"][0]) == want.num_dropped
+    avg = orc.load_metrics(want.counts, want.kept, T, k).avg_tokens_per_expert
+    assert r["stats"]["avg_tokens_per_expert"][0] == np.float32(avg)
     rows = orc.permuted_rows(x, want)
     for row, xr in rows.items():
         assert np.array_equal(r["xp"][row], xr), row
@@ -212,6 +215,8 @@ def test_empty_batch():
     idx, w, st, flags = gu.route_from_logits(cfg, np.zeros((0, 8), np.float32))
     assert flags == 0 and idx.shape == (0, 2)
     assert np.all(st["counts"] == 0) and np.all(st["y_frac"] == 0) and st["l_aux_p3"][0] == 0
+    assert st["z_loss"][0] == 0 and st["load_std"][0] == 0 and st["top2_ratio"][0] == 0
     r = gu.dispatch(cfg, torch.empty((0, 64), dtype=torch.int16, device="cuda"),
                     torch.empty((0, 2), dtype=torch.int32, device="cuda"))
     assert np.all(r["seg_off"] == 0) and np.all(r["seg_count"] == 0)
+    assert r["stats"]["avg_tokens_per_expert"][0] == 0

@@ -399,6 +399,28 @@ def check_bias_update_hand(o=orc):
     assert got.dtype == np.float32
 
 
+def check_aux_loss_free_balances(o=orc):
+    # the method's purpose: on logits with a per-expert ramp (experts 0..1 take
+    # most of the load), repeated sign updates of the selection bias drive the
+    # load std towards 0 and move the bias against the load ramp
+    from expert_router_gemm_b200 import synth
+    T, N, k = 4096, 8, 2
+    g = synth.make_logits(5, T, N, "skewed").astype(np.float64)
+    b = np.zeros(N, np.float32)
+    first = None
+    for _ in range(60):
+        counts = np.bincount(o.topk(g, k, b).reshape(-1), minlength=N)
+        m = o.load_metrics(counts, counts, T, k)
+        first = m.load_std if first is None else first
+        b = o.bias_update(b, counts, T, k, 0.05)
+    assert first > 0.1 and m.load_std < 0.1 * first, (first, m.load_std)
+    assert np.all(np.diff(b) > 0), b
+
+
+def test_aux_loss_free_balances():
+    check_aux_loss_free_balances()
+
+
 def test_selection_bias_hand():
     check_selection_bias_hand()
 
@@ -496,7 +518,7 @@ ALL_CHECKS = [check_capacity_worked_example, check_capacity_closed_forms, check_
               check_dropped_slots_contribute_zero, check_shared_expert_added, check_aux_hand,
               check_aux_uniform, check_bf16_rounding, check_bf16_decode, check_selection_bias_hand,
               check_selection_bias_bruteforce, check_bias_update_hand, check_z_loss,
-              check_load_metrics_hand]
+              check_load_metrics_hand, check_aux_loss_free_balances]
 
 
 def _mut_topk_high_index_ties(g, k, selection_bias=None):
