@@ -150,12 +150,14 @@ def oracle_threads() -> int:
         return os.cpu_count() or 1
 
 
-def oracle_expert_steps(w, inp, n_steps=None, budget_s=None):
+def oracle_expert_steps(w, inp, n_steps=None, budget_s=None, mx=False):
     """Time the fp64 oracle on a bounded sample of the workload: the routing of
     all T tokens once, then one expert per step (its kept rows through the SwiGLU
-    FFN and their weighted contributions to the combine).  Returns a list of
+    FFN and their weighted contributions to the combine; with mx the oracle's
+    block-scaled FP8 expert, quantization included).  Returns a list of
     (token_equivalents, seconds) per step and the routing time."""
     from oracle import moe_oracle as orc
+    from oracle import mxfp8 as mxo
     t0 = time.perf_counter()
     g = orc.router_logits(inp.x, inp.w_router, inp.bias)
     s = orc.softmax(g)
@@ -179,7 +181,11 @@ def oracle_expert_steps(w, inp, n_steps=None, budget_s=None):
         e = int(order[i % w.N])
         ts = time.perf_counter()
         ti, tj = np.nonzero((idx == e) & (disp.row_map >= 0))
-        if len(ti):
+        if len(ti) and mx:
+            o = mxo.swiglu_mx(mxo.mx_quantize(orc.as_f64(inp.x[ti])), mxo.quantize_weight(inp.w1[e]),
+                              mxo.quantize_weight(inp.w3[e]), mxo.quantize_weight(inp.w2[e]))
+            np.add.at(y, ti, wts[ti, tj][:, None] * o)
+        elif len(ti):
             o = orc.swiglu_ffn(orc.as_f64(inp.x[ti]), inp.w1[e], inp.w3[e], inp.w2[e], bf16)
             np.add.at(y, ti, wts[ti, tj][:, None] * o)
         steps.append((len(ti) / w.k, time.perf_counter() - ts))
@@ -238,6 +244,9 @@ def main():
     ap.add_argument("--aux-free", type=float, default=0.0, metavar="GAMMA",
                     help="Aux-Loss-Free routing: a selection bias, updated on the device with "
                          "this step size after every layer call (0 = off)")
+    ap.add_argument("--gemm", default="act", choices=["act", "mxfp8"],
+                    help="number format of the routed experts' GEMMs: the activation dtype, or "
+                         "block-scaled FP8 (weights quantized once before the timed region)")
     ap.add_argument("--shape", default="",
                     help="override workload fields for small profiling cases, e.g. T=2048,N=32")
     args = ap.parse_args()
@@ -270,8 +279,14 @@ def main():
     from expert_router_gemm_b200 import moe
 
     inp = synth.make_inputs(w)
-    cfg = moe.config_from_workload(w)
+    mx = args.gemm == "mxfp8"
+    cfg = moe.config_from_workload(w, gemm=args.gemm)
     dl = moe.to_device(inp, cfg)
+    if mx:
+        dl.quantize_mx()
+        torch.cuda.synchronize()
+        dl.w1 = dl.w3 = dl.w2 = None   # the FP8 layer reads only the quantized experts
+        torch.cuda.empty_cache()
     aux_free = args.aux_free > 0
     if aux_free:
         dl.selection_bias = torch.zeros(w.N, dtype=torch.float32, device="cuda")
@@ -344,9 +359,10 @@ def main():
                      "avg_tokens_per_expert")}
     line = {"metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "mxfp8 experts (e4m3, bf16 in/out)" if mx else w.dtype,
             "data": "synthetic",
-            "config": dict(workload_config(w), parallelism=f"replicas x{world}",
+            "config": dict(workload_config(w), expert_gemm=args.gemm, parallelism=f"replicas x{world}",
                            l2="inputs larger than L2: the expert weights read every step "
                               f"({(inp.w1.nbytes + inp.w3.nbytes + inp.w2.nbytes) / 1e9:.2f} GB) "
                               "exceed the 126 MB L2; no flush"),
@@ -368,6 +384,10 @@ def main():
         seg_count = torch.empty(N, dtype=torch.int32, device="cuda")
         xp = torch.empty((max_rows, d), dtype=act, device="cuda")
         h = torch.empty((max_rows, f), dtype=act, device="cuda")
+        if mx:
+            x8 = torch.empty((max_rows, d), dtype=torch.uint8, device="cuda")
+            x8sf = torch.empty(moe.mx_sf_bytes(max_rows, d), dtype=torch.uint8, device="cuda")
+            h8sf = torch.empty(moe.mx_sf_bytes(max_rows, f), dtype=torch.uint8, device="cuda")
         hs = torch.empty((T, w.f_shared), dtype=act, device="cuda") if w.f_shared else None
         sh = torch.empty((T, d), dtype=act, device="cuda") if w.f_shared else None
         names = ["route", "dispatch", "expert_ffn", "shared_ffn", "combine"] + (
@@ -377,9 +397,17 @@ def main():
             evs[0].record(stream)
             moe.moe_route(cfg, dl.x, dl.w_router, dl.bias, dl.selection_bias, None, idx, wt, stats, ws_op, stream)
             evs[1].record(stream)
-            moe.moe_dispatch(cfg, dl.x, idx, row_map, seg_off, seg_count, xp, stats, ws_op, stream)
+            if mx:
+                moe.moe_dispatch_mx(cfg, dl.x, idx, row_map, seg_off, seg_count, x8, x8sf, stats, ws_op,
+                                    stream)
+            else:
+                moe.moe_dispatch(cfg, dl.x, idx, row_map, seg_off, seg_count, xp, stats, ws_op, stream)
             evs[2].record(stream)
-            moe.moe_expert_ffn(cfg, xp, seg_off, seg_count, weights, h, xp, ws_op, stream)
+            if mx:
+                moe.moe_expert_ffn_mx(cfg, x8, x8sf, seg_off, seg_count, weights, h, h8sf, xp, ws_op,
+                                      stream)
+            else:
+                moe.moe_expert_ffn(cfg, xp, seg_off, seg_count, weights, h, xp, ws_op, stream)
             evs[3].record(stream)
             if w.f_shared:
                 moe.moe_shared_expert_ffn(cfg, dl.x, weights, hs, sh, ws_op, stream)
@@ -408,12 +436,18 @@ def main():
         peaks, peak_src = load_peaks()
         hbm = peaks["hbm_gbs"]
         tc_peak = peaks["bf16_tflops_sustained"]
+        # the FP8 GEMM's peak: the measured bf16 figure times the nominal FP8 : bf16
+        # dense ratio (4.5 : 2.25 PFLOP/s)
+        gemm_peak = 2.0 * tc_peak if mx else tc_peak
         x_bytes = T * d * elem
         route_bytes = x_bytes + d * N * 4 + T * k * 8
         route_flops = 2.0 * T * d * N
-        disp_bytes = x_bytes + a_kept * d * elem + T * k * 8
+        if mx:   # rows written as 1-byte codes plus one scale byte per 32 values
+            disp_bytes = x_bytes + a_kept * d * (1 + 1 / 32) + T * k * 8
+        else:
+            disp_bytes = x_bytes + a_kept * d * elem + T * k * 8
         ffn_flops = 6.0 * d * f * a_kept
-        ffn_wbytes = 3.0 * N * d * f * elem
+        ffn_wbytes = 3.0 * N * d * f * ((1 + 1 / 32) if mx else elem)
         comb_bytes = a_kept * d * elem + T * k * 8 + x_bytes + (x_bytes if w.f_shared else 0)
         sh_flops = 6.0 * T * d * w.f_shared
 
@@ -443,7 +477,7 @@ def main():
                          "frac_hbm": round(gbs(disp_bytes, stage_ms["dispatch"]) / hbm, 4)},
             "expert_ffn": {"ms": round(stage_ms["expert_ffn"], 4), "flops": ffn_flops,
                            "TFLOP/s": round(tfs(ffn_flops, stage_ms["expert_ffn"]), 1),
-                           "frac_tensor": round(tfs(ffn_flops, stage_ms["expert_ffn"]) / tc_peak, 4),
+                           "frac_tensor": round(tfs(ffn_flops, stage_ms["expert_ffn"]) / gemm_peak, 4),
                            "weight_bytes": ffn_wbytes,
                            "weight_GB/s": round(gbs(ffn_wbytes, stage_ms["expert_ffn"]), 1)},
             "combine": {"ms": round(stage_ms["combine"], 4), "bytes": comb_bytes,
@@ -458,14 +492,18 @@ def main():
         line["kernels"] = kern
         line["stage_sum_ms"] = round(sum(stage_ms.values()), 4)
         ffn_tf = tfs(ffn_flops, stage_ms["expert_ffn"])
-        tr = traffic_record("ffn_tc.cu")
+        tr = traffic_record("ffn_mx.cu" if mx else "ffn_tc.cu")
         line["roofline"] = {
-            "kernel": "tc_ffn_gemm_kernel (grouped SwiGLU GEMM + down GEMM, the two launches of "
-                      "moe_expert_ffn)",
-            "bound": "tensor", "achieved": round(ffn_tf, 1), "peak": tc_peak, "unit": "TFLOP/s",
-            "frac": round(ffn_tf / tc_peak, 4),
-            "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a seconds-long loop)",
-            "frac_of_burst_peak": round(ffn_tf / peaks["bf16_tflops"], 4),
+            "kernel": ("tc_mx_gemm_kernel (block-scaled FP8 grouped SwiGLU GEMM + down GEMM, the two "
+                       "launches of moe_expert_ffn_mx)") if mx else
+                      ("tc_ffn_gemm_kernel (grouped SwiGLU GEMM + down GEMM, the two launches of "
+                       "moe_expert_ffn)"),
+            "bound": "tensor", "achieved": round(ffn_tf, 1), "peak": gemm_peak, "unit": "TFLOP/s",
+            "frac": round(ffn_tf / gemm_peak, 4),
+            "peak_source": (f"{peak_src} bf16_tflops_sustained x 2 (nominal FP8 : bf16 dense ratio; "
+                            "kernel timed inside a seconds-long loop)") if mx else
+                           f"{peak_src} bf16_tflops_sustained (kernel timed inside a seconds-long loop)",
+            "frac_of_burst_peak": round(ffn_tf / (peaks["bf16_tflops"] * (2.0 if mx else 1.0)), 4),
             "algorithmic_flops_per_step": ffn_flops,
             "traffic": (tr["expert_ffn_per_step"] * 1.0 if tr and "expert_ffn_per_step" in tr else None)}
 
@@ -538,7 +576,7 @@ def main():
                        "serial_ms_per_step": round(serial_ms, 4)}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.quick:
-        steps, t_route = oracle_expert_steps(w, inp, budget_s=args.cpu_budget)
+        steps, t_route = oracle_expert_steps(w, inp, budget_s=args.cpu_budget, mx=mx)
         rate, tok, sec = cpu_rate(steps, t_route, w.T)
         line["cpu_baseline"] = {
             "value": round(rate, 3), "unit": "tokens/s", "cores": oracle_threads(), "kind": "oracle",

@@ -250,4 +250,69 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int b_mn_maj
          | (static_cast<uint32_t>(M >> 4) << 24);     // M / 16
 }
 
+// ------------------------------------------------------------------ block-scaled FP8
+// 1-D bulk copy global -> shared (16-byte aligned, size a multiple of 16),
+// completion counted on `bar` as transaction bytes.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
+// Shared-memory descriptor of an unswizzled K-major operand made of 8-row x
+// 16-byte core matrices: SBO = distance between 8-row groups, LBO = distance
+// between 16-byte K columns (layout field 0 = no swizzle).
+__device__ __forceinline__ uint64_t smem_desc_plain(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  return d;
+}
+
+// Copy a 32-row x 16-byte block of shared memory into 4 consecutive TMEM
+// columns of all 128 lanes (each 32-lane quarter receives the same 32 rows).
+__device__ __forceinline__ void tc_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// Instruction descriptor of tcgen05.mma kind::mxf8f6f4.block_scale: E4M3 A and
+// B (both K-major), E8M0 scales, fp32 accumulator, M x N tile, K = 32 per
+// instruction.  sf_id (bits 29-30 for A, 4-5 for B) selects which byte of the
+// 32-bit scale word (which 32-element K block of the stage) the MMA uses.
+__host__ __device__ constexpr uint32_t idesc_mxf8(int M, int N, uint32_t sf_id) {
+  return (sf_id << 4)                                // B scale-factor byte
+         | (0u << 7)                                 // A format: E4M3
+         | (0u << 10)                                // B format: E4M3
+         | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
+         | (1u << 23)                                // scale format: E8M0
+         | (static_cast<uint32_t>(M >> 4) << 24)     // M / 16
+         | (sf_id << 29);                            // A scale-factor byte
+}
+// D[tmem] (+)= (A * scaleA) x (B * scaleB), scales read from TMEM
+__device__ __forceinline__ void tc_mma_mxf8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+      : "memory");
+}
+
+// Shared exponent of a block of 32 values with largest magnitude `amax` (>= 0):
+// the smallest e in [-127, 127] with amax <= 448 * 2^e.  With amax = M 2^E,
+// M in [1, 2): e = E - 8 if M <= 1.75, else E - 7 (integer logic on the bits;
+// zero and fp32 subnormals give -127).
+__device__ __forceinline__ int mx_exponent(float amax) {
+  const uint32_t b = __float_as_uint(amax);
+  const int ef = static_cast<int>((b >> 23) & 0xFFu);
+  if (ef == 0) return -127;
+  const int e = ef - 127 - 8 + ((b & 0x7FFFFFu) > 0x600000u ? 1 : 0);
+  return e < -127 ? -127 : e;
+}
+// 2^-e as a float, for -127 <= e <= 126
+__device__ __forceinline__ float mx_inv_scale(int e) { return __uint_as_float(static_cast<uint32_t>(127 - e) << 23); }
+
 }  // namespace moe

@@ -17,6 +17,8 @@
 //   3. scatter: rank of (t, e) = base[block][e] + popcount of the mask bits below
 //               t, kept iff rank < C; row = seg_off[e] + rank; one warp per token
 //               copies x[t] with 16-byte vectors to each of its kept rows.
+#include <cuda_fp8.h>
+
 #include "device_utils.cuh"
 #include "internal.h"
 
@@ -193,6 +195,86 @@ __global__ void __launch_bounds__(kScatterThreads) dispatch_scatter_kernel(const
   }
 }
 
+// The same permutation with the rows quantized on the way: block-scaled FP8
+// (E4M3 codes, one E8M0 scale per 32 values of d, the smallest power of two
+// that keeps the block within 448).  A warp reads its bf16 token row once;
+// four lanes hold one block of 32 values (8 each), so the block maximum is two
+// shuffles.  Codes go to every kept row, the scale byte to the tile-interleaved
+// scale buffer of the rows.
+__device__ __forceinline__ uint32_t e4m3x4_rn(float a, float b, float c, float d) {
+  const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+  const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(c, d), __NV_SATFINITE, __NV_E4M3);
+  return lo | (hi << 16);
+}
+
+__global__ void __launch_bounds__(kScatterThreads) dispatch_scatter_mx_kernel(const DispatchArgs a) {
+  __shared__ uint32_t m[256];
+  __shared__ int base_s[256];
+  __shared__ int off_s[256];
+  __shared__ int rows_s[kScatterTokens][32];
+  const int N = a.N, k = a.k;
+  const int64_t t_first = static_cast<int64_t>(blockIdx.x) * kScatterTokens;
+  const int64_t blk = t_first / kDispatchTokens;
+  for (int e = threadIdx.x; e < N; e += kScatterThreads) {
+    m[e] = a.mask[blk * N + e];
+    base_s[e] = a.base[blk * N + e];
+    off_s[e] = a.seg_off[e];
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t t = t_first + warp;
+  const int pos = static_cast<int>(t - blk * kDispatchTokens);
+  if (t >= a.T) return;
+
+  if (lane < k) {
+    const int32_t* row = a.topk_idx + t * k;
+    const int e = row[lane];
+    int r = -1;
+    if (slot_valid(row, lane, e, N)) {
+      const int rank = base_s[e] + __popc(m[e] & ((1u << pos) - 1u));
+      if (rank < a.capacity) r = off_s[e] + rank;
+    }
+    a.row_map[t * k + lane] = r;
+    rows_s[warp][lane] = r;
+  }
+  __syncwarp();
+
+  const int d = a.d;
+  const int nvec = d / 8;                          // 16-byte vectors (8 bf16) per row
+  const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.x) + t * d);
+  uint8_t* codes = static_cast<uint8_t*>(a.xp);
+  for (int c0 = 0; c0 < nvec; c0 += 32 * kCopyUnroll) {
+    uint4 v[kCopyUnroll];
+#pragma unroll
+    for (int u = 0; u < kCopyUnroll; ++u) {
+      const int c = c0 + 32 * u + lane;
+      v[u] = c < nvec ? src[c] : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < kCopyUnroll; ++u) {
+      const int c = c0 + 32 * u + lane;           // d % 32 == 0: a block's 4 lanes are all in or all out
+      const float f[8] = {bf16_lo(v[u].x), bf16_hi(v[u].x), bf16_lo(v[u].y), bf16_hi(v[u].y),
+                          bf16_lo(v[u].z), bf16_hi(v[u].z), bf16_lo(v[u].w), bf16_hi(v[u].w)};
+      float amax = 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+      if (c >= nvec) continue;
+      const int ex = mx_exponent(amax);
+      const float inv = mx_inv_scale(ex);
+      const uint2 q = make_uint2(e4m3x4_rn(f[0] * inv, f[1] * inv, f[2] * inv, f[3] * inv),
+                                 e4m3x4_rn(f[4] * inv, f[5] * inv, f[6] * inv, f[7] * inv));
+      for (int j = 0; j < k; ++j) {
+        const int r = rows_s[warp][j];
+        if (r < 0) continue;
+        *reinterpret_cast<uint2*>(codes + static_cast<int64_t>(r) * d + 8 * c) = q;
+        if ((lane & 3) == 0) a.xp_sf[mx_sf_offset(r, c / 4, d / 32)] = static_cast<uint8_t>(ex + 127);
+      }
+    }
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t s) {
@@ -200,7 +282,10 @@ cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t s) {
   dispatch_mask_kernel<<<blocks, kMaskThreads, 0, s>>>(a);
   dispatch_scan_kernel<<<(a.N + 31) / 32, 1024, 0, s>>>(a, blocks);
   const unsigned sblocks = static_cast<unsigned>((a.T + kScatterTokens - 1) / kScatterTokens);
-  dispatch_scatter_kernel<<<sblocks, kScatterThreads, 0, s>>>(a);
+  if (a.xp_sf != nullptr)
+    dispatch_scatter_mx_kernel<<<sblocks, kScatterThreads, 0, s>>>(a);
+  else
+    dispatch_scatter_kernel<<<sblocks, kScatterThreads, 0, s>>>(a);
   return cudaGetLastError();
 }
 

@@ -68,6 +68,9 @@ cudaError_t launch_router_tc(const RouteArgs& a, void* split, float* partials, i
 // swizzle, zero fill outside the tensor.
 bool make_tma_2d_bf16(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint32_t box_inner,
                       uint32_t box_outer);
+// The same over bytes (FP8 codes).
+bool make_tma_2d_u8(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                    uint32_t box_outer);
 
 // --------------------------------------------------------------- dispatch
 constexpr int kDispatchTokens = 32;   // tokens per dispatch block (one bit each)
@@ -81,6 +84,8 @@ struct DispatchArgs {
   int32_t* seg_off;
   int32_t* seg_count;
   void* xp;
+  uint8_t* xp_sf;           // non-null: xp receives block-scaled FP8 codes and these
+                            // scale bytes (tile-interleaved, d/32 per row)
   uint32_t* mask;           // [blocks, N] scratch
   int32_t* base;            // [blocks, N] scratch
   int32_t* counts;          // [N] scratch
@@ -125,6 +130,49 @@ struct FfnArgs {
 };
 cudaError_t launch_ffn_bf16(const FfnArgs& a, cudaStream_t s);
 cudaError_t launch_ffn_f32(const FfnArgs& a, cudaStream_t s);
+
+// Block-scaled FP8 (E4M3 codes, one E8M0 scale byte per 32 values along K,
+// scales in the tile-interleaved layout of mx_sf_offset) grouped SwiGLU FFN:
+// a = FP8 codes of the permuted rows [rows, d] with a_sf; w1/w3 [G][f][d] and w2
+// [G][d][f] K-major codes with their scales; h = FP8 codes [rows, f] with h_sf
+// (written by GEMM1, read by GEMM2); out [rows, d] bf16.  d and f are
+// multiples of 128 and segments start at multiples of 128 rows.
+struct FfnMxArgs {
+  int G;
+  int64_t max_rows;
+  int d, f;
+  const int32_t* seg_off;
+  const int32_t* seg_count;
+  const uint8_t* a;
+  const uint8_t* a_sf;
+  const uint8_t* w1;
+  const uint8_t* w1_sf;
+  const uint8_t* w3;
+  const uint8_t* w3_sf;
+  const uint8_t* w2;
+  const uint8_t* w2_sf;
+  uint8_t* h;
+  uint8_t* h_sf;
+  void* out;
+  uint32_t* flags;
+};
+cudaError_t launch_ffn_mx(const FfnMxArgs& a, cudaStream_t s);
+
+// Quantize G weights [G][K][N] (bf16, N contiguous) to K-major FP8 codes
+// [G][N][K] and scale bytes [G][N/128][K/128][512]; K, N multiples of 128.
+cudaError_t launch_mx_quantize_weight(const uint16_t* w, int64_t G, int K, int N, uint8_t* codes, uint8_t* sf,
+                                      cudaStream_t s);
+
+// Byte offset of the scale of (row, 32-element block kb) in a tile-interleaved
+// scale buffer with n_kblocks blocks per row: 512-byte atoms of 128 rows x 4
+// blocks ordered (row tile, K tile); inside an atom 16 (m % 32) + 4 (m / 32) + j.
+__host__ __device__ inline int64_t mx_sf_offset(int64_t row, int kb, int n_kblocks) {
+  const int64_t atom = (row >> 7) * (n_kblocks >> 2) + (kb >> 2);
+  const int m = static_cast<int>(row & 127);
+  return atom * 512 + 16 * (m & 31) + 4 * (m >> 5) + (kb & 3);
+}
+// bytes of the scales of `rows` rows of K values
+__host__ __device__ inline int64_t mx_sf_bytes(int64_t rows, int K) { return (rows + 127) / 128 * 128 * (K / 32); }
 
 // ---------------------------------------------------------------- combine
 struct CombineArgs {

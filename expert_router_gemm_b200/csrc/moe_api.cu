@@ -47,6 +47,7 @@ struct Dims {
   int64_t T;
   int d, N, k, f, fs, C, align, elem;
   bool bf16;
+  bool mx;             // routed-expert GEMMs in block-scaled FP8
   int64_t max_rows;    // rows of xp / h / out buffers
   int64_t max_count;   // upper bound of one expert's kept rows: min(C, T)
 };
@@ -97,12 +98,15 @@ moe_status_t derive(const moe_config_t* cfg, Dims* D) {
   D->fs = cfg->f_shared;
   D->bf16 = cfg->act_dtype == MOE_BF16;
   D->elem = D->bf16 ? 2 : 4;
+  if (cfg->gemm_format != MOE_GEMM_ACT && cfg->gemm_format != MOE_GEMM_MXFP8) return MOE_ERR_INVALID_ARG;
+  D->mx = cfg->gemm_format == MOE_GEMM_MXFP8;
   D->align = cfg->seg_align == 0 ? 128 : cfg->seg_align;
   if (D->bf16) {
     if (D->d % 64 || D->f % 64 || D->fs % 64) return MOE_ERR_UNSUPPORTED;
   } else {
     if (D->d % 4) return MOE_ERR_UNSUPPORTED;  // rows are moved as 16-byte vectors
   }
+  if (D->mx && (!D->bf16 || D->d % 128 || D->f % 128 || D->align % 128)) return MOE_ERR_UNSUPPORTED;
   if (cfg->capacity >= 0) {
     D->C = cfg->capacity;
   } else {
@@ -118,9 +122,11 @@ moe_status_t derive(const moe_config_t* cfg, Dims* D) {
 
 // Workspace layout.  The first bytes (flags word, route ticket, route count and
 // z accumulators) are zeroed by one memset at the start of every routing call.
+// In an FP8 layer the xp region holds the bf16 expert outputs, h the FP8 codes
+// of h, and x8 / x8sf / h8sf the FP8 rows and the two scale buffers.
 struct Layout {
   size_t flags, rticket, rcnt, rz, zero_end, rzl, rsplit, rlogits, dmask, dbase, dcounts, dticket, op_end;
-  size_t idx, w, row_map, seg_off, seg_count, xp, h, hs, sh, layer_end;
+  size_t idx, w, row_map, seg_off, seg_count, xp, h, hs, sh, x8, x8sf, h8sf, layer_end;
 };
 
 Layout layout(const Dims& D) {
@@ -156,6 +162,9 @@ Layout layout(const Dims& D) {
   L.h = take(static_cast<size_t>(D.elem) * D.max_rows * D.f);
   L.hs = take(static_cast<size_t>(D.elem) * (D.fs ? D.T * D.fs : 0));
   L.sh = take(static_cast<size_t>(D.elem) * (D.fs ? D.T * D.d : 0));
+  L.x8 = take(D.mx ? static_cast<size_t>(D.max_rows) * D.d : 0);
+  L.x8sf = take(D.mx ? static_cast<size_t>(mx_sf_bytes(D.max_rows, D.d)) : 0);
+  L.h8sf = take(D.mx ? static_cast<size_t>(mx_sf_bytes(D.max_rows, D.f)) : 0);
   L.layer_end = o;
   return L;
 }
@@ -236,8 +245,8 @@ moe_status_t do_route(const Dims& D, const void* x, const float* w_router, const
 }
 
 moe_status_t do_dispatch(const Dims& D, const void* x, const int32_t* topk_idx, int32_t* row_map,
-                         int32_t* seg_off, int32_t* seg_count, void* xp, const moe_stats_t* stats,
-                         void* ws, cudaStream_t st) {
+                         int32_t* seg_off, int32_t* seg_count, void* xp, uint8_t* xp_sf,
+                         const moe_stats_t* stats, void* ws, cudaStream_t st) {
   const Layout L = layout(D);
   if (D.T == 0) {
     cudaError_t e = cudaMemsetAsync(seg_off, 0, sizeof(int32_t) * (D.N + 1), st);
@@ -263,6 +272,7 @@ moe_status_t do_dispatch(const Dims& D, const void* x, const int32_t* topk_idx, 
   a.seg_off = seg_off;
   a.seg_count = seg_count;
   a.xp = xp;
+  a.xp_sf = xp_sf;
   a.mask = at<uint32_t*>(ws, L.dmask);
   a.base = at<int32_t*>(ws, L.dbase);
   a.counts = at<int32_t*>(ws, L.dcounts);
@@ -295,6 +305,39 @@ moe_status_t do_ffn(const Dims& D, const void* a_rows, const int32_t* seg_off, c
   a.flags = at<uint32_t*>(ws, L.flags);
   if (D.T == 0) return MOE_OK;
   return cuda_status(D.bf16 ? launch_ffn_bf16(a, st) : launch_ffn_f32(a, st));
+}
+
+moe_status_t do_ffn_mx(const Dims& D, const void* xp, const void* xp_sf, const int32_t* seg_off,
+                       const int32_t* seg_count, const moe_weights_t* w, void* h, void* h_sf, void* out, void* ws,
+                       cudaStream_t st) {
+  const Layout L = layout(D);
+  FfnMxArgs a{};
+  a.G = D.N;
+  a.max_rows = D.max_rows;
+  a.d = D.d;
+  a.f = D.f;
+  a.seg_off = seg_off;
+  a.seg_count = seg_count;
+  a.a = static_cast<const uint8_t*>(xp);
+  a.a_sf = static_cast<const uint8_t*>(xp_sf);
+  a.w1 = static_cast<const uint8_t*>(w->w1_mx);
+  a.w1_sf = static_cast<const uint8_t*>(w->w1_sf);
+  a.w3 = static_cast<const uint8_t*>(w->w3_mx);
+  a.w3_sf = static_cast<const uint8_t*>(w->w3_sf);
+  a.w2 = static_cast<const uint8_t*>(w->w2_mx);
+  a.w2_sf = static_cast<const uint8_t*>(w->w2_sf);
+  a.h = static_cast<uint8_t*>(h);
+  a.h_sf = static_cast<uint8_t*>(h_sf);
+  a.out = out;
+  a.flags = at<uint32_t*>(ws, L.flags);
+  if (D.T == 0) return MOE_OK;
+  return cuda_status(launch_ffn_mx(a, st));
+}
+
+bool mx_weights_ok(const moe_weights_t* w) {
+  return w != nullptr && w->w1_mx && w->w1_sf && w->w3_mx && w->w3_sf && w->w2_mx && w->w2_sf &&
+         aligned16(w->w1_mx) && aligned16(w->w1_sf) && aligned16(w->w3_mx) && aligned16(w->w3_sf) &&
+         aligned16(w->w2_mx) && aligned16(w->w2_sf);
 }
 
 moe_status_t do_combine(const Dims& D, const void* out_rows, const int32_t* row_map, const float* topk_w,
@@ -344,6 +387,7 @@ moe_status_t dispatch_prepare(const moe_config_t* cfg, const void* x, const int3
   a->seg_off = seg_off;
   a->seg_count = seg_count;
   a->xp = xp;
+  a->xp_sf = nullptr;
   if (stats) a->stats = *stats;
   *blocks = (D.T + kDispatchTokens - 1) / kDispatchTokens;
   return MOE_OK;
@@ -452,7 +496,7 @@ moe_status_t moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t*
     return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(xp)) return MOE_ERR_MISALIGNED;
   if ((s = check_ws(ws, ws_bytes, layout(D).op_end)) != MOE_OK) return s;
-  return do_dispatch(D, x, topk_idx, row_map, seg_off, seg_count, xp, stats, ws,
+  return do_dispatch(D, x, topk_idx, row_map, seg_off, seg_count, xp, nullptr, stats, ws,
                      reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -505,11 +549,15 @@ moe_status_t moe_layer_fwd(const moe_config_t* cfg, const moe_weights_t* weights
   Dims D;
   moe_status_t s = derive(cfg, &D);
   if (s != MOE_OK) return s;
-  if (weights == nullptr || weights->w_router == nullptr || !weights->w1 || !weights->w3 || !weights->w2 ||
-      (D.T > 0 && (x == nullptr || y == nullptr)))
+  if (weights == nullptr || weights->w_router == nullptr || (D.T > 0 && (x == nullptr || y == nullptr)))
+    return MOE_ERR_INVALID_ARG;
+  if (D.mx ? !(weights->w1_mx && weights->w1_sf && weights->w3_mx && weights->w3_sf && weights->w2_mx &&
+               weights->w2_sf)
+           : !(weights->w1 && weights->w3 && weights->w2))
     return MOE_ERR_INVALID_ARG;
   if (D.fs > 0 && (!weights->ws1 || !weights->ws3 || !weights->ws2)) return MOE_ERR_INVALID_ARG;
-  if (!aligned16(x) || !aligned16(y) || !ffn_weights_ok(weights)) return MOE_ERR_MISALIGNED;
+  if (!aligned16(x) || !aligned16(y) || !(D.mx ? mx_weights_ok(weights) : ffn_weights_ok(weights)))
+    return MOE_ERR_MISALIGNED;
   if (D.fs > 0 && (!aligned16(weights->ws1) || !aligned16(weights->ws3) || !aligned16(weights->ws2)))
     return MOE_ERR_MISALIGNED;
   const Layout L = layout(D);
@@ -529,14 +577,69 @@ moe_status_t moe_layer_fwd(const moe_config_t* cfg, const moe_weights_t* weights
   if ((s = do_route(D, x, weights->w_router, weights->router_bias, weights->selection_bias, nullptr, nullptr, idx, w,
                     stats, ws, st)) != MOE_OK)
     return s;
-  if ((s = do_dispatch(D, x, idx, row_map, seg_off, seg_count, xp, stats, ws, st)) != MOE_OK) return s;
-  if ((s = do_ffn(D, xp, seg_off, seg_count, weights->w1, weights->w3, weights->w2, D.f, false, h, out_rows, ws,
-                  st)) != MOE_OK)
-    return s;
+  if (D.mx) {
+    void* x8 = at<void*>(ws, L.x8);
+    uint8_t* x8sf = at<uint8_t*>(ws, L.x8sf);
+    if ((s = do_dispatch(D, x, idx, row_map, seg_off, seg_count, x8, x8sf, stats, ws, st)) != MOE_OK) return s;
+    if ((s = do_ffn_mx(D, x8, x8sf, seg_off, seg_count, weights, h, at<void*>(ws, L.h8sf), out_rows, ws, st)) !=
+        MOE_OK)
+      return s;
+  } else {
+    if ((s = do_dispatch(D, x, idx, row_map, seg_off, seg_count, xp, nullptr, stats, ws, st)) != MOE_OK) return s;
+    if ((s = do_ffn(D, xp, seg_off, seg_count, weights->w1, weights->w3, weights->w2, D.f, false, h, out_rows, ws,
+                    st)) != MOE_OK)
+      return s;
+  }
   if (D.fs > 0 && (s = do_ffn(D, x, nullptr, nullptr, weights->ws1, weights->ws3, weights->ws2, D.fs, true,
                               at<void*>(ws, L.hs), shared_out, ws, st)) != MOE_OK)
     return s;
   return do_combine(D, out_rows, row_map, w, shared_out, y, st);
+}
+
+moe_status_t moe_mx_quantize_weight(const void* w, int64_t G, int32_t K, int32_t N, void* codes, void* sf,
+                                    moe_stream_t stream) {
+  if (G < 0 || K < 1 || N < 1 || G > 65535) return MOE_ERR_INVALID_ARG;
+  if (K % 128 || N % 128 || N / 128 > 65535) return MOE_ERR_UNSUPPORTED;
+  if (G > 0 && (w == nullptr || codes == nullptr || sf == nullptr)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(w) || !aligned16(codes) || !aligned16(sf)) return MOE_ERR_MISALIGNED;
+  return cuda_status(launch_mx_quantize_weight(static_cast<const uint16_t*>(w), G, K, N, static_cast<uint8_t*>(codes),
+                                               static_cast<uint8_t*>(sf), reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_dispatch_mx(const moe_config_t* cfg, const void* x, const int32_t* topk_idx, int32_t* row_map,
+                             int32_t* seg_off, int32_t* seg_count, void* xp_codes, void* xp_sf, moe_stats_t* stats,
+                             void* ws, size_t ws_bytes, moe_stream_t stream) {
+  Dims D;
+  moe_status_t s = derive(cfg, &D);
+  if (s != MOE_OK) return s;
+  if (!D.mx) return MOE_ERR_INVALID_ARG;
+  if (seg_off == nullptr || seg_count == nullptr) return MOE_ERR_INVALID_ARG;
+  if (D.T > 0 && (x == nullptr || topk_idx == nullptr || row_map == nullptr || xp_codes == nullptr || xp_sf == nullptr))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(xp_codes) || !aligned16(xp_sf)) return MOE_ERR_MISALIGNED;
+  if ((s = check_ws(ws, ws_bytes, layout(D).op_end)) != MOE_OK) return s;
+  return do_dispatch(D, x, topk_idx, row_map, seg_off, seg_count, xp_codes, static_cast<uint8_t*>(xp_sf), stats, ws,
+                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_expert_ffn_mx(const moe_config_t* cfg, const void* xp_codes, const void* xp_sf, const int32_t* seg_off,
+                               const int32_t* seg_count, const moe_weights_t* weights, void* h_codes, void* h_sf,
+                               void* out_rows, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  Dims D;
+  moe_status_t s = derive(cfg, &D);
+  if (s != MOE_OK) return s;
+  if (!D.mx || weights == nullptr) return MOE_ERR_INVALID_ARG;
+  if (!(weights->w1_mx && weights->w1_sf && weights->w3_mx && weights->w3_sf && weights->w2_mx && weights->w2_sf))
+    return MOE_ERR_INVALID_ARG;
+  if (D.T > 0 && (xp_codes == nullptr || xp_sf == nullptr || seg_off == nullptr || seg_count == nullptr ||
+                  h_codes == nullptr || h_sf == nullptr || out_rows == nullptr))
+    return MOE_ERR_INVALID_ARG;
+  if (!mx_weights_ok(weights) || !aligned16(xp_codes) || !aligned16(xp_sf) || !aligned16(h_codes) ||
+      !aligned16(h_sf) || !aligned16(out_rows))
+    return MOE_ERR_MISALIGNED;
+  if ((s = check_ws(ws, ws_bytes, layout(D).op_end)) != MOE_OK) return s;
+  return do_ffn_mx(D, xp_codes, xp_sf, seg_off, seg_count, weights, h_codes, h_sf, out_rows, ws,
+                   reinterpret_cast<cudaStream_t>(stream));
 }
 
 moe_status_t moe_read_flags(const void* ws, size_t ws_bytes, uint32_t* flags, moe_stream_t stream) {

@@ -27,6 +27,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_MISALIGNED = 0, 1, 2, 3
 MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_NONFINITE, MOE_ERR_DEVICE = 4, 5, 6, 7
 MOE_F32, MOE_BF16 = 0, 1
+MOE_GEMM_ACT, MOE_GEMM_MXFP8 = 0, 1
 MOE_FLAG_NONFINITE_LOGITS, MOE_FLAG_BAD_EXPERT_INDEX, MOE_FLAG_WAIT_TIMEOUT = 1, 2, 4
 
 
@@ -34,13 +35,14 @@ class moe_config_t(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int64), ("d", ctypes.c_int32), ("N", ctypes.c_int32),
                 ("k", ctypes.c_int32), ("f", ctypes.c_int32), ("f_shared", ctypes.c_int32),
                 ("capacity_factor", ctypes.c_double), ("capacity", ctypes.c_int32),
-                ("act_dtype", ctypes.c_int), ("seg_align", ctypes.c_int32)]
+                ("act_dtype", ctypes.c_int), ("seg_align", ctypes.c_int32),
+                ("gemm_format", ctypes.c_int32)]
 
 
 class moe_weights_t(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("w_router", "router_bias", "w1", "w3", "w2", "ws1", "ws3", "ws2",
-                 "selection_bias")]
+                 "selection_bias", "w1_mx", "w1_sf", "w3_mx", "w3_sf", "w2_mx", "w2_sf")]
 
 
 class moe_stats_t(ctypes.Structure):
@@ -63,6 +65,12 @@ _PROTOS = {
     "moe_route_from_logits": (ctypes.c_int, [ctypes.POINTER(moe_config_t), _P, _P, _P, _P,
                                              ctypes.POINTER(moe_stats_t), _P, _SZ, _P]),
     "moe_bias_update": (ctypes.c_int, [ctypes.POINTER(moe_config_t), _P, _P, ctypes.c_float, _P]),
+    "moe_mx_quantize_weight": (ctypes.c_int, [_P, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, _P, _P,
+                                              _P]),
+    "moe_dispatch_mx": (ctypes.c_int, [ctypes.POINTER(moe_config_t), _P, _P, _P, _P, _P, _P, _P,
+                                       ctypes.POINTER(moe_stats_t), _P, _SZ, _P]),
+    "moe_expert_ffn_mx": (ctypes.c_int, [ctypes.POINTER(moe_config_t), _P, _P, _P, _P,
+                                         ctypes.POINTER(moe_weights_t), _P, _P, _P, _P, _SZ, _P]),
     "moe_dispatch": (ctypes.c_int, [ctypes.POINTER(moe_config_t), _P, _P, _P, _P, _P, _P,
                                     ctypes.POINTER(moe_stats_t), _P, _SZ, _P]),
     "moe_dispatch_static": (ctypes.c_int, [ctypes.POINTER(moe_config_t), _P, _P, _P, _P, _P, _P,
@@ -124,9 +132,10 @@ def _stream(stream) -> Optional[int]:
 
 def make_config(T: int, d: int, N: int, k: int, f: int, f_shared: int = 0,
                 capacity_factor: float = 1.0, capacity: int = -1, dtype: str = "bf16",
-                seg_align: int = 0) -> moe_config_t:
+                seg_align: int = 0, gemm: str = "act") -> moe_config_t:
     return moe_config_t(T, d, N, k, f, f_shared, capacity_factor, capacity,
-                        MOE_BF16 if dtype == "bf16" else MOE_F32, seg_align)
+                        MOE_BF16 if dtype == "bf16" else MOE_F32, seg_align,
+                        MOE_GEMM_MXFP8 if gemm == "mxfp8" else MOE_GEMM_ACT)
 
 
 def config_from_workload(w, T: Optional[int] = None, **over) -> moe_config_t:
@@ -137,9 +146,11 @@ def config_from_workload(w, T: Optional[int] = None, **over) -> moe_config_t:
 
 
 def make_weights(w_router, router_bias=None, w1=None, w3=None, w2=None, ws1=None, ws3=None,
-                 ws2=None, selection_bias=None) -> moe_weights_t:
+                 ws2=None, selection_bias=None, w1_mx=None, w1_sf=None, w3_mx=None, w3_sf=None,
+                 w2_mx=None, w2_sf=None) -> moe_weights_t:
     return moe_weights_t(*[_ptr(t) for t in (w_router, router_bias, w1, w3, w2, ws1, ws3, ws2,
-                                            selection_bias)])
+                                            selection_bias, w1_mx, w1_sf, w3_mx, w3_sf, w2_mx,
+                                            w2_sf)])
 
 
 def make_stats(y_frac=None, z_mean=None, l_aux_p3=None, l_aux_switch=None, counts=None,
@@ -215,6 +226,32 @@ def moe_dispatch_static(cfg, x, topk_idx, row_map, seg_off, seg_count, xp, stats
 MOE_DISPATCH_STATIC_MAX_CELLS = 131072
 
 
+def moe_mx_quantize_weight(w, G: int, K: int, N: int, codes, sf, stream=None):
+    _check(_lib.moe_mx_quantize_weight(_ptr(w), G, K, N, _ptr(codes), _ptr(sf), _stream(stream)),
+           "moe_mx_quantize_weight")
+
+
+def moe_dispatch_mx(cfg, x, topk_idx, row_map, seg_off, seg_count, xp_codes, xp_sf, stats, ws,
+                    stream=None):
+    _check(_lib.moe_dispatch_mx(ctypes.byref(cfg), _ptr(x), _ptr(topk_idx), _ptr(row_map),
+                                _ptr(seg_off), _ptr(seg_count), _ptr(xp_codes), _ptr(xp_sf),
+                                _stats_ref(stats), _ptr(ws), ws.numel() if ws is not None else 0,
+                                _stream(stream)), "moe_dispatch_mx")
+
+
+def moe_expert_ffn_mx(cfg, xp_codes, xp_sf, seg_off, seg_count, weights: moe_weights_t, h_codes,
+                      h_sf, out_rows, ws, stream=None):
+    _check(_lib.moe_expert_ffn_mx(ctypes.byref(cfg), _ptr(xp_codes), _ptr(xp_sf), _ptr(seg_off),
+                                  _ptr(seg_count), ctypes.byref(weights), _ptr(h_codes), _ptr(h_sf),
+                                  _ptr(out_rows), _ptr(ws), ws.numel() if ws is not None else 0,
+                                  _stream(stream)), "moe_expert_ffn_mx")
+
+
+def mx_sf_bytes(rows: int, K: int) -> int:
+    """Bytes of the scales of `rows` rows of K values (tile-interleaved layout)."""
+    return (rows + 127) // 128 * 128 * (K // 32)
+
+
 def moe_expert_ffn(cfg, xp, seg_off, seg_count, weights: moe_weights_t, h, out_rows, ws,
                    stream=None):
     _check(_lib.moe_expert_ffn(ctypes.byref(cfg), _ptr(xp), _ptr(seg_off), _ptr(seg_count),
@@ -273,10 +310,28 @@ class DeviceLayer:
     ws3: Optional[torch.Tensor] = None
     ws2: Optional[torch.Tensor] = None
     selection_bias: Optional[torch.Tensor] = None
+    mx: Optional[dict] = None      # block-scaled FP8 weights (quantize_mx)
 
     def weights(self) -> moe_weights_t:
+        m = self.mx or {}
         return make_weights(self.w_router, self.bias, self.w1, self.w3, self.w2,
-                            self.ws1, self.ws3, self.ws2, self.selection_bias)
+                            self.ws1, self.ws3, self.ws2, self.selection_bias,
+                            m.get("w1_mx"), m.get("w1_sf"), m.get("w3_mx"), m.get("w3_sf"),
+                            m.get("w2_mx"), m.get("w2_sf"))
+
+    def quantize_mx(self, stream=None) -> dict:
+        """Quantize the routed experts' bf16 weights to block-scaled FP8 on the
+        device (moe_mx_quantize_weight) and keep them for weights()."""
+        N, d, f = self.cfg.N, self.cfg.d, self.cfg.f
+        dev = self.w1.device
+        out = {}
+        for name, w, K, Nn in (("w1", self.w1, d, f), ("w3", self.w3, d, f), ("w2", self.w2, f, d)):
+            codes = torch.empty((N, Nn, K), dtype=torch.uint8, device=dev)
+            sf = torch.empty(N * Nn * K // 32, dtype=torch.uint8, device=dev)
+            moe_mx_quantize_weight(w, N, K, Nn, codes, sf, stream)
+            out[name + "_mx"], out[name + "_sf"] = codes, sf
+        self.mx = out
+        return out
 
 
 def to_device(inputs, cfg: moe_config_t, device="cuda") -> DeviceLayer:

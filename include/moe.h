@@ -69,6 +69,12 @@ typedef enum {
 
 typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype_t;
 
+/* Number format of the routed experts' GEMMs (moe_config_t.gemm_format). */
+typedef enum {
+  MOE_GEMM_ACT = 0,    /* the act_dtype (bf16 or fp32), the default */
+  MOE_GEMM_MXFP8 = 1,  /* block-scaled FP8: E4M3 codes, one E8M0 scale per 32 values along K */
+} moe_gemm_format_t;
+
 /* Bits of the device flags word (moe_read_flags). */
 #define MOE_FLAG_NONFINITE_LOGITS 0x1u  /* some router logit was NaN or +-Inf */
 #define MOE_FLAG_BAD_EXPERT_INDEX 0x2u  /* topk_idx outside [0,N) or repeated in a row */
@@ -85,6 +91,8 @@ typedef struct {
   int32_t capacity;        /* >= 0: use this C instead of the formula; < 0: derive */
   moe_dtype_t act_dtype;   /* MOE_F32 or MOE_BF16 */
   int32_t seg_align;       /* expert segments start at multiples of this many rows; 0 -> 128 */
+  int32_t gemm_format;     /* moe_gemm_format_t; MOE_GEMM_MXFP8 needs act_dtype MOE_BF16,
+                              d % 128 == 0, f % 128 == 0 and seg_align % 128 == 0 */
 } moe_config_t;
 
 typedef struct {
@@ -99,6 +107,14 @@ typedef struct {
   const float* selection_bias; /* [N] fp32 Aux-Loss-Free bias, added to g for the top-k
                                   choice only (the weights use the unbiased softmax);
                                   NULL = none.  Update it with moe_bias_update(). */
+  /* Block-scaled FP8 copies of the routed experts (gemm_format MOE_GEMM_MXFP8;
+     written by moe_mx_quantize_weight): K-major codes and their scales. */
+  const void* w1_mx;         /* [N][f][d] E4M3 codes of W1 (K = d) */
+  const void* w1_sf;         /* scales of w1_mx: N * f * d / 32 bytes */
+  const void* w3_mx;         /* [N][f][d] codes of W3 */
+  const void* w3_sf;
+  const void* w2_mx;         /* [N][d][f] codes of W2 (K = f) */
+  const void* w2_sf;         /* N * d * f / 32 bytes */
 } moe_weights_t;
 
 /* Load-balance and capacity statistics.  Device pointers; each may be NULL. */
@@ -253,6 +269,55 @@ moe_status_t moe_dispatch_static(const moe_config_t* cfg, const void* x, const i
                                  moe_stats_t* stats, uint32_t* device_flags, moe_stream_t stream);
 
 /*
+ * Block-scaled FP8 ("MoE 训练加速实战" §9.1: FP8 forward with bf16 activations;
+ * the pages fix no format).  A tensor of R rows by K values (K a multiple of
+ * 128) is stored as R x K E4M3 codes (row-major) plus one E8M0 scale byte per
+ * 32 consecutive values of a row: the value of code c in block b is
+ * e4m3(c) * 2^(scale_b - 127), where scale_b - 127 is the smallest exponent e
+ * with max|v| <= 448 * 2^e over the block, and each code is v / 2^e rounded to
+ * the nearest E4M3 value (ties to even).  The scale bytes use the layout the
+ * tensor cores read: 512-byte atoms for 128 rows x 4 blocks, atoms in order
+ * (row / 128, block / 4), and inside an atom row m, block j at byte
+ * 16 * (m % 32) + 4 * (m / 32) + j % 4; a buffer for R rows holds
+ * ceil(R / 128) * 128 * K / 32 bytes.
+ */
+
+/*
+ * moe_mx_quantize_weight - quantize G matrices w [G][K][N] (bf16, N contiguous,
+ * the layout of W1/W3 with K = d, N = f, or of W2 with K = f, N = d) along K:
+ * codes [G][N][K] (K-major) and sf (G * N * K / 32 bytes, N counting rows).
+ * K and N multiples of 128 (MOE_ERR_UNSUPPORTED otherwise); every buffer
+ * 16-byte aligned.  Bit-exact and deterministic.
+ */
+moe_status_t moe_mx_quantize_weight(const void* w, int64_t G, int32_t K, int32_t N, void* codes, void* sf,
+                                    moe_stream_t stream);
+
+/*
+ * moe_dispatch_mx - moe_dispatch for a MOE_GEMM_MXFP8 layer: the same row map,
+ * segments and statistics, with each kept row quantized on the way: xp_codes
+ * [max_rows, d] E4M3 codes and xp_sf (scales of max_rows rows, K = d).  x is
+ * bf16.  Rows between segments are not written.
+ */
+moe_status_t moe_dispatch_mx(const moe_config_t* cfg, const void* x, const int32_t* topk_idx,
+                             int32_t* row_map, int32_t* seg_off, int32_t* seg_count, void* xp_codes,
+                             void* xp_sf, moe_stats_t* stats, void* ws, size_t ws_bytes,
+                             moe_stream_t stream);
+
+/*
+ * moe_expert_ffn_mx - the routed experts of a MOE_GEMM_MXFP8 layer as one
+ * grouped GEMM pair on the tcgen05 block-scaled FP8 tensor cores
+ * (kind::mxf8f6f4, scales applied inside the MMA, fp32 accumulation):
+ *   h[r] = silu(xp[r] W1_e) * (xp[r] W3_e), written as FP8 codes h_codes
+ *          [max_rows, f] + h_sf (blocks of 32 along f)
+ *   out_rows[r] = h[r] W2_e, bf16 [max_rows, d]
+ * Inputs: xp_codes / xp_sf from moe_dispatch_mx, weights->w{1,3,2}_mx/_sf.
+ */
+moe_status_t moe_expert_ffn_mx(const moe_config_t* cfg, const void* xp_codes, const void* xp_sf,
+                               const int32_t* seg_off, const int32_t* seg_count,
+                               const moe_weights_t* weights, void* h_codes, void* h_sf,
+                               void* out_rows, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
  * moe_expert_ffn - all routed experts as one grouped GEMM pair, SwiGLU fused.
  * "MoE 训练加速实战" §4.1-4.2: one kernel serves every expert, y_i = W_i x_i.
  * For every expert e and row r in [seg_off[e], seg_off[e] + seg_count[e]):
@@ -291,7 +356,10 @@ moe_status_t moe_combine(const moe_config_t* cfg, const void* out_rows, const in
 
 /*
  * moe_layer_fwd - the whole layer: route, dispatch, routed experts, shared
- * expert (if cfg->f_shared > 0), combine.  x [T, d] act (read), y [T, d] act
+ * expert (if cfg->f_shared > 0), combine.  With gemm_format MOE_GEMM_MXFP8 the
+ * dispatch quantizes the rows and the routed experts run in block-scaled FP8
+ * from weights->w*_mx (the bf16 w1/w3/w2 are not read; the shared expert stays
+ * bf16).  x [T, d] act (read), y [T, d] act
  * (written), stats may be NULL (every field is filled), ws >= layer_bytes of
  * moe_workspace_size.  weights->selection_bias (may be NULL) steers the top-k
  * choice as in moe_route; the layer does not update it.  The permuted rows and

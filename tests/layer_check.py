@@ -68,9 +68,10 @@ def oracle_routing(inp, w, align=128, cap=None, selection_bias=None):
 
 
 def compare_layer(inp, w, gpu_y, gpu_idx, gpu_row_map, gpu_logits=None, tol=2e-2,
-                  sample=None, seed=0, align=128, cap=None, selection_bias=None):
+                  sample=None, seed=0, align=128, cap=None, selection_bias=None, mxfp8=False):
     """Returns (rel_frobenius, n_compared, n_flips).  With a selection bias the
-    near-tie test runs on the biased scores that decide the choice."""
+    near-tie test runs on the biased scores that decide the choice; with mxfp8
+    the reference output is the block-scaled FP8 layer of oracle.mxfp8."""
     T = inp.x.shape[0]
     ref = oracle_routing(inp, w, align, cap, selection_bias)
     bound = logit_bound(inp.x, inp.w_router, inp.bias)
@@ -111,10 +112,17 @@ def compare_layer(inp, w, gpu_y, gpu_idx, gpu_row_map, gpu_logits=None, tol=2e-2
     good = np.array(sorted(set(range(T)) - flip_set - set(cascade)), dtype=np.int64)
     if sample is not None and sample < len(good):
         good = np.sort(np.random.default_rng(seed).choice(good, size=sample, replace=False))
-    res = orc.layer_forward(inp.x, inp.w_router, inp.bias, inp.w1, inp.w3, inp.w2, k=w.k,
-                            capacity_factor=w.capacity_factor, cap=cap, bf16=inp.bf16,
-                            ws1=inp.ws1, ws3=inp.ws3, ws2=inp.ws2, align=align, tokens=good,
-                            logits=ref.logits, selection_bias=selection_bias)
+    if mxfp8:
+        from oracle import mxfp8 as mxo
+        res = mxo.layer_forward_mxfp8(inp.x, inp.w_router, inp.bias, inp.w1, inp.w3, inp.w2, k=w.k,
+                                      capacity_factor=w.capacity_factor, cap=cap, ws1=inp.ws1,
+                                      ws3=inp.ws3, ws2=inp.ws2, align=align, tokens=good,
+                                      logits=ref.logits, selection_bias=selection_bias)
+    else:
+        res = orc.layer_forward(inp.x, inp.w_router, inp.bias, inp.w1, inp.w3, inp.w2, k=w.k,
+                                capacity_factor=w.capacity_factor, cap=cap, bf16=inp.bf16,
+                                ws1=inp.ws1, ws3=inp.ws3, ws2=inp.ws2, align=align, tokens=good,
+                                logits=ref.logits, selection_bias=selection_bias)
     y = gpu_y[good]
     if y.dtype == np.uint16:
         y = (y.astype(np.uint32) << np.uint32(16)).view(np.float32)

@@ -182,3 +182,50 @@ def test_header_documents_every_entry_point():
     for f in ("moe_route", "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_capacity"):
         block = text[text.index(" * " + f + " "):]
         assert "§" in block[:900] or "section" in block[:900], f
+
+
+def test_mxfp8_config_validation():
+    ok = moe.make_config(T=256, d=256, N=8, k=2, f=384, gemm="mxfp8")
+    lb_mx, ob_mx, rows = moe.moe_workspace_size(ok)
+    lb, ob, rows2 = moe.moe_workspace_size(moe.make_config(T=256, d=256, N=8, k=2, f=384))
+    assert rows == rows2 and ob_mx == ob and lb_mx > lb
+    for bad in (moe.make_config(T=256, d=320, N=8, k=2, f=384, gemm="mxfp8"),    # d % 128
+                moe.make_config(T=256, d=256, N=8, k=2, f=192, gemm="mxfp8"),    # f % 128
+                moe.make_config(T=256, d=256, N=8, k=2, f=384, gemm="mxfp8", seg_align=64),
+                moe.make_config(T=256, d=256, N=8, k=2, f=384, gemm="mxfp8", dtype="f32")):
+        with pytest.raises(moe.MoeError) as ei:
+            moe.moe_workspace_size(bad)
+        assert ei.value.status == moe.MOE_ERR_UNSUPPORTED
+    weird = moe.make_config(T=256, d=256, N=8, k=2, f=384)
+    weird.gemm_format = 7
+    with pytest.raises(moe.MoeError) as ei:
+        moe.moe_workspace_size(weird)
+    assert ei.value.status == INVALID
+
+
+def test_mx_entry_validation():
+    q = lambda w=0x1000, G=2, K=256, N=128, c=0x2000, s=0x3000: moe.raw_call(  # noqa: E731
+        "moe_mx_quantize_weight", w, ctypes.c_int64(G), K, N, c, s, None)
+    assert q(K=100) == moe.MOE_ERR_UNSUPPORTED
+    assert q(N=200) == moe.MOE_ERR_UNSUPPORTED
+    assert q(w=None) == INVALID
+    assert q(G=-1) == INVALID
+    assert q(c=0x2008) == MISAL
+    assert q(G=0, w=None, c=None, s=None) == moe.MOE_OK   # nothing to do, nothing launched
+    plain = moe.make_config(T=256, d=256, N=8, k=2, f=384)
+    mx = moe.make_config(T=256, d=256, N=8, k=2, f=384, gemm="mxfp8")
+    _, ob, _ = moe.moe_workspace_size(mx)
+    sz = ctypes.c_size_t(ob)
+    d = lambda c: moe.raw_call("moe_dispatch_mx", ctypes.byref(c), 0x1000, 0x2000, 0x3000, 0x4000,  # noqa: E731
+                               0x5000, 0x6000, 0x7000, None, 0x8000, sz, None)
+    assert d(plain) == INVALID                              # needs an FP8 config
+    w = moe.make_weights(0x100, w1=0x200, w3=0x300, w2=0x400)  # bf16 weights only
+    f = lambda c, wt: moe.raw_call("moe_expert_ffn_mx", ctypes.byref(c), 0x1000, 0x2000, 0x3000,  # noqa: E731
+                                   0x4000, ctypes.byref(wt), 0x5000, 0x6000, 0x7000, 0x8000, sz, None)
+    assert f(mx, w) == INVALID                              # FP8 weights missing
+    wmx = moe.make_weights(0x100, w1_mx=0x200, w1_sf=0x300, w3_mx=0x400, w3_sf=0x500, w2_mx=0x600,
+                           w2_sf=0x708)
+    assert f(mx, wmx) == MISAL
+    layer = lambda wt: moe.raw_call("moe_layer_fwd", ctypes.byref(mx), ctypes.byref(wt), 0x1000,  # noqa: E731
+                                    0x2000, None, 0x3000, ctypes.c_size_t(1 << 40), None)
+    assert layer(w) == INVALID
