@@ -250,6 +250,11 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int b_mn_maj
          | (static_cast<uint32_t>(M >> 4) << 24);     // M / 16
 }
 
+// kind::f16 descriptor with the majorness of both operands selectable.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_ab(int M, int N, int a_mn_major, int b_mn_major) {
+  return idesc_bf16_f32(M, N, b_mn_major) | (static_cast<uint32_t>(a_mn_major) << 15);
+}
+
 // ------------------------------------------------------------------ block-scaled FP8
 // 1-D bulk copy global -> shared (16-byte aligned, size a multiple of 16),
 // completion counted on `bar` as transaction bytes.

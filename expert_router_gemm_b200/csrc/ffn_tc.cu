@@ -75,6 +75,8 @@ struct TcParams {
   int K;                     // reduction length (multiple of 64)
   int n_out;                 // output columns
   uint16_t* out;             // [max_rows, n_out] bf16
+  uint16_t* save_g;          // SwiGLU, optional: gate and up pre-activations [max_rows, n_out]
+  uint16_t* save_u;          //   (bf16), kept for the backward pass
   uint32_t* flags;
 };
 
@@ -389,6 +391,17 @@ __global__ void __launch_bounds__(kThreads, 1)
               pk[i] = pack_bf16x2(h0, h1);
             }
             store_row32(orow, tile.n0 + c, p.n_out, pk);
+            if (p.save_g != nullptr) {
+              const int64_t off = (static_cast<int64_t>(tl.row0[tile.g]) + row) * p.n_out;
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                pk[i] = pack_bf16x2(__uint_as_float(gv[2 * i]), __uint_as_float(gv[2 * i + 1]));
+              store_row32(p.save_g + off, tile.n0 + c, p.n_out, pk);
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                pk[i] = pack_bf16x2(__uint_as_float(uv[2 * i]), __uint_as_float(uv[2 * i + 1]));
+              store_row32(p.save_u + off, tile.n0 + c, p.n_out, pk);
+            }
           }
         }
       } else {
@@ -501,8 +514,11 @@ cudaError_t launch_pair(const FfnArgs& a, const CUtensorMap& mA1, const CUtensor
   p.K = a.d;
   p.n_out = a.f;
   p.out = static_cast<uint16_t*>(a.h);
+  p.save_g = static_cast<uint16_t*>(a.save_g);
+  p.save_u = static_cast<uint16_t*>(a.save_u);
   cudaError_t e = launch_gemm<MODE_SWIGLU, CG>(mA1, mW1, mW3, p, m_bound * ((a.f + 127) / 128), s);
   if (e != cudaSuccess) return e;
+  p.save_g = p.save_u = nullptr;
   p.K = a.f;
   p.n_out = a.d;
   p.out = static_cast<uint16_t*>(a.out);

@@ -126,6 +126,8 @@ struct FfnArgs {
   const void* w2;           // [G][f][d]
   void* h;                  // [rows, f]
   void* out;                // [rows, d]
+  void* save_g;             // bf16 path, optional: [rows, f] gate / up pre-activations of GEMM1
+  void* save_u;
   uint32_t* flags;
 };
 cudaError_t launch_ffn_bf16(const FfnArgs& a, cudaStream_t s);
@@ -173,6 +175,70 @@ __host__ __device__ inline int64_t mx_sf_offset(int64_t row, int kb, int n_kbloc
 }
 // bytes of the scales of `rows` rows of K values
 __host__ __device__ inline int64_t mx_sf_bytes(int64_t rows, int K) { return (rows + 127) / 128 * 128 * (K / 32); }
+
+// --------------------------------------------------------------- backward
+// Row groups of the backward GEMMs: the experts' segments (seg_off [G+1],
+// seg_count [G]) or, with seg_off == nullptr, one dense group of dense_rows rows.
+struct BwdGroups {
+  int G;
+  int dense_rows;
+  int64_t max_rows;
+  const int32_t* seg_off;
+  const int32_t* seg_count;
+  uint32_t* flags;
+};
+// dH = dO W2^T per group, then dG = dH * u * silu'(g), dU = dH * silu(g) (bf16;
+// rows of a segment past its kept count are written as zeros).
+cudaError_t launch_dgrad_swiglu(const BwdGroups& s, int d, int f, const void* dO, const void* w2, const void* g,
+                                const void* u, void* dG, void* dU, cudaStream_t st);
+// dXp = dG W1^T + dU W3^T per group (bf16, kept rows).
+cudaError_t launch_dgrad_plain2(const BwdGroups& s, int d, int f, const void* dG, const void* dU, const void* w1,
+                                const void* w3, void* dXp, cudaStream_t st);
+// out[g] = A_g^T B_g over the rows of group g (its padded segment, whose extra
+// rows are zero): A [rows][M], B [rows][N] bf16, out [G][M][N] fp32.
+cudaError_t launch_wgrad(const BwdGroups& s, int M, int N, const void* a, const void* b, float* out, cudaStream_t st);
+
+struct BwdSmallArgs {
+  int64_t T;
+  int d, N, k, f;
+  float aux_weight, z_weight;
+  const uint16_t* dy;        // [T, d]
+  const float* logits;       // [T, N] (router logits incl. the router bias)
+  const int32_t* topk_idx;   // [T, k]
+  const float* topk_w;       // [T, k]
+  const int32_t* row_map;    // [T, k]
+  const int32_t* counts;     // [N] top-k selections per expert
+  const uint16_t* out_rows;  // [rows, d] expert outputs o
+  uint16_t* dO;              // [rows, d]
+  float* dw;                 // [T, k] gradient of the routing weights
+  float* dg;                 // [T, N] gradient of the logits
+};
+// dO[row] = w * dy[t] and dw[t][j] = <dy[t], o[row]> for kept slots (dw = 0 for
+// dropped ones).
+cudaError_t launch_combine_bwd(const BwdSmallArgs& a, cudaStream_t s);
+// Router backward: renormalised weights, softmax, Switch auxiliary loss and
+// z-loss gradients -> dg.
+cudaError_t launch_router_bwd(const BwdSmallArgs& a, cudaStream_t s);
+// Zero the rows [seg_off[e] + seg_count[e], seg_off[e+1]) of up to four bf16
+// row buffers (row widths cols[i], multiples of 8).
+struct PadBufs {
+  void* buf[4];
+  int cols[4];
+  int n;
+};
+cudaError_t launch_zero_pad_rows(int N, const int32_t* seg_off, const int32_t* seg_count, const PadBufs& b,
+                                 cudaStream_t s);
+// dW_r = x^T dg (fp32 [d, N]) and dbias = sum_t dg[t] (may be null), with
+// per-chunk partials summed in a fixed order (scratch: n_chunks * (d + 1) * N floats).
+size_t router_wgrad_scratch_floats(int64_t T, int d, int N);
+cudaError_t launch_router_wgrad(int64_t T, int d, int N, const uint16_t* x, const float* dg, float* dw_router,
+                                float* dbias, float* scratch, cudaStream_t s);
+// dxr = dg W_r^T (fp32 [T, d]).
+cudaError_t launch_router_dgrad(int64_t T, int d, int N, const float* dg, const float* w_router, float* dxr,
+                                cudaStream_t s);
+// dx[t] = sum over kept slots of dXp[row] + dxr[t] (+ dxs[t]), one rounding to bf16.
+cudaError_t launch_dx_gather(int64_t T, int d, int k, const int32_t* row_map, const uint16_t* dXp, const float* dxr,
+                             const uint16_t* dxs, uint16_t* dx, cudaStream_t s);
 
 // ---------------------------------------------------------------- combine
 struct CombineArgs {

@@ -169,6 +169,47 @@ Layout layout(const Dims& D) {
   return L;
 }
 
+// Workspace of the backward pass: the op head (flags, routing and dispatch
+// scratch) of the forward layout, then its own arrays.  Row buffers are reused
+// in place: o becomes dO, g and u become dG and dU, xp becomes dXp.
+struct BwdLayout {
+  size_t idx, w, row_map, seg_off, seg_count, logits, counts, dw, dg, dxr, rws, xp, g, u, h, o, gs, us, hs, dxs, end;
+};
+
+BwdLayout bwd_layout(const Dims& D) {
+  const Layout L = layout(D);
+  BwdLayout B{};
+  size_t o = L.op_end;
+  auto take = [&](size_t bytes) {
+    const size_t at_ = o;
+    o = round_up(o + bytes, kAlign);
+    return at_;
+  };
+  const size_t T = static_cast<size_t>(D.T), R = static_cast<size_t>(D.max_rows);
+  B.idx = take(4 * T * D.k);
+  B.w = take(4 * T * D.k);
+  B.row_map = take(4 * T * D.k);
+  B.seg_off = take(4 * (D.N + 1));
+  B.seg_count = take(4 * D.N);
+  B.logits = take(4 * T * D.N);
+  B.counts = take(4 * D.N);
+  B.dw = take(4 * T * D.k);
+  B.dg = take(4 * T * D.N);
+  B.dxr = take(4 * T * D.d);
+  B.rws = take(4 * router_wgrad_scratch_floats(D.T, D.d, D.N));
+  B.xp = take(2 * R * D.d);
+  B.g = take(2 * R * D.f);
+  B.u = take(2 * R * D.f);
+  B.h = take(2 * R * D.f);
+  B.o = take(2 * R * D.d);
+  B.gs = take(D.fs ? 2 * T * D.fs : 0);
+  B.us = take(D.fs ? 2 * T * D.fs : 0);
+  B.hs = take(D.fs ? 2 * T * D.fs : 0);
+  B.dxs = take(D.fs ? 2 * T * D.d : 0);
+  B.end = o;
+  return B;
+}
+
 template <typename P>
 P at(void* ws, size_t off) {
   return reinterpret_cast<P>(static_cast<uint8_t*>(ws) + off);
@@ -284,7 +325,7 @@ moe_status_t do_dispatch(const Dims& D, const void* x, const int32_t* topk_idx, 
 
 moe_status_t do_ffn(const Dims& D, const void* a_rows, const int32_t* seg_off, const int32_t* seg_count,
                     const void* w1, const void* w3, const void* w2, int f, bool dense, void* h, void* out,
-                    void* ws, cudaStream_t st) {
+                    void* ws, cudaStream_t st, void* save_g = nullptr, void* save_u = nullptr) {
   const Layout L = layout(D);
   FfnArgs a{};
   a.G = dense ? 1 : D.N;
@@ -302,6 +343,8 @@ moe_status_t do_ffn(const Dims& D, const void* a_rows, const int32_t* seg_off, c
   a.w2 = w2;
   a.h = h;
   a.out = out;
+  a.save_g = save_g;
+  a.save_u = save_u;
   a.flags = at<uint32_t*>(ws, L.flags);
   if (D.T == 0) return MOE_OK;
   return cuda_status(D.bf16 ? launch_ffn_bf16(a, st) : launch_ffn_f32(a, st));
@@ -640,6 +683,156 @@ moe_status_t moe_expert_ffn_mx(const moe_config_t* cfg, const void* xp_codes, co
   if ((s = check_ws(ws, ws_bytes, layout(D).op_end)) != MOE_OK) return s;
   return do_ffn_mx(D, xp_codes, xp_sf, seg_off, seg_count, weights, h_codes, h_sf, out_rows, ws,
                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_backward_workspace_size(const moe_config_t* cfg, size_t* bytes) {
+  Dims D;
+  moe_status_t s = derive(cfg, &D);
+  if (s != MOE_OK) return s;
+  if (!D.bf16 || D.mx || D.align % 64) return MOE_ERR_UNSUPPORTED;
+  if (bytes) *bytes = bwd_layout(D).end;
+  return MOE_OK;
+}
+
+moe_status_t moe_layer_bwd(const moe_config_t* cfg, const moe_weights_t* weights, const void* x, const void* dy,
+                           float aux_weight, float z_weight, moe_grads_t* grads, void* ws, size_t ws_bytes,
+                           moe_stream_t stream) {
+  Dims D;
+  moe_status_t s = derive(cfg, &D);
+  if (s != MOE_OK) return s;
+  if (!D.bf16 || D.mx || D.align % 64) return MOE_ERR_UNSUPPORTED;
+  if (weights == nullptr || grads == nullptr || weights->w_router == nullptr || !weights->w1 || !weights->w3 ||
+      !weights->w2 || !grads->dw_router || !grads->dw1 || !grads->dw3 || !grads->dw2 || !std::isfinite(aux_weight) ||
+      !std::isfinite(z_weight))
+    return MOE_ERR_INVALID_ARG;
+  if (D.T > 0 && (x == nullptr || dy == nullptr || grads->dx == nullptr)) return MOE_ERR_INVALID_ARG;
+  if (D.fs > 0 && (!weights->ws1 || !weights->ws3 || !weights->ws2 || !grads->dws1 || !grads->dws3 || !grads->dws2))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(dy) || !aligned16(grads->dx) || !ffn_weights_ok(weights) ||
+      !aligned16(grads->dw1) || !aligned16(grads->dw3) || !aligned16(grads->dw2))
+    return MOE_ERR_MISALIGNED;
+  if (D.fs > 0 && (!aligned16(weights->ws1) || !aligned16(weights->ws3) || !aligned16(weights->ws2) ||
+                   !aligned16(grads->dws1) || !aligned16(grads->dws3) || !aligned16(grads->dws2)))
+    return MOE_ERR_MISALIGNED;
+  const BwdLayout B = bwd_layout(D);
+  if ((s = check_ws(ws, ws_bytes, B.end)) != MOE_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t T = D.T;
+  const int d = D.d, N = D.N, k = D.k, f = D.f, fs = D.fs;
+  float* dbias = weights->router_bias != nullptr ? grads->drouter_bias : nullptr;
+
+  if (T == 0) {  // no tokens: every weight gradient is zero
+    cudaError_t e = cudaMemsetAsync(grads->dw_router, 0, sizeof(float) * d * N, st);
+    if (e == cudaSuccess && dbias) e = cudaMemsetAsync(dbias, 0, sizeof(float) * N, st);
+    const size_t we = static_cast<size_t>(N) * d * f * sizeof(float);
+    if (e == cudaSuccess) e = cudaMemsetAsync(grads->dw1, 0, we, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(grads->dw3, 0, we, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(grads->dw2, 0, we, st);
+    if (fs > 0) {
+      const size_t se = static_cast<size_t>(d) * fs * sizeof(float);
+      if (e == cudaSuccess) e = cudaMemsetAsync(grads->dws1, 0, se, st);
+      if (e == cudaSuccess) e = cudaMemsetAsync(grads->dws3, 0, se, st);
+      if (e == cudaSuccess) e = cudaMemsetAsync(grads->dws2, 0, se, st);
+    }
+    return cuda_status(e);
+  }
+
+  int32_t* idx = at<int32_t*>(ws, B.idx);
+  float* w = at<float*>(ws, B.w);
+  int32_t* row_map = at<int32_t*>(ws, B.row_map);
+  int32_t* seg_off = at<int32_t*>(ws, B.seg_off);
+  int32_t* seg_count = at<int32_t*>(ws, B.seg_count);
+  float* logits = at<float*>(ws, B.logits);
+  void* xp = at<void*>(ws, B.xp);
+  void* g = at<void*>(ws, B.g);
+  void* u = at<void*>(ws, B.u);
+  void* h = at<void*>(ws, B.h);
+  void* o = at<void*>(ws, B.o);
+  uint32_t* flags = at<uint32_t*>(ws, layout(D).flags);
+
+  // forward recompute: routing (logits and counts kept), permutation, experts
+  // with the SwiGLU pre-activations saved
+  moe_stats_t rs{};
+  rs.counts = at<int32_t*>(ws, B.counts);
+  if ((s = do_route(D, x, weights->w_router, weights->router_bias, weights->selection_bias, nullptr, logits, idx, w,
+                    &rs, ws, st)) != MOE_OK)
+    return s;
+  if ((s = do_dispatch(D, x, idx, row_map, seg_off, seg_count, xp, nullptr, nullptr, ws, st)) != MOE_OK) return s;
+  if ((s = do_ffn(D, xp, seg_off, seg_count, weights->w1, weights->w3, weights->w2, f, false, h, o, ws, st, g, u)) !=
+      MOE_OK)
+    return s;
+
+  BwdSmallArgs a{};
+  a.T = T;
+  a.d = d;
+  a.N = N;
+  a.k = k;
+  a.f = f;
+  a.aux_weight = aux_weight;
+  a.z_weight = z_weight;
+  a.dy = static_cast<const uint16_t*>(dy);
+  a.logits = logits;
+  a.topk_idx = idx;
+  a.topk_w = w;
+  a.row_map = row_map;
+  a.counts = rs.counts;
+  a.out_rows = static_cast<const uint16_t*>(o);
+  a.dO = static_cast<uint16_t*>(o);   // in place: each row is read, then overwritten, by one block
+  a.dw = at<float*>(ws, B.dw);
+  a.dg = at<float*>(ws, B.dg);
+  cudaError_t e = launch_combine_bwd(a, st);
+  PadBufs pb{};
+  pb.buf[0] = xp;
+  pb.cols[0] = d;
+  pb.buf[1] = h;
+  pb.cols[1] = f;
+  pb.buf[2] = o;
+  pb.cols[2] = d;
+  pb.n = 3;
+  if (e == cudaSuccess) e = launch_zero_pad_rows(N, seg_off, seg_count, pb, st);
+  if (e == cudaSuccess) e = launch_router_bwd(a, st);
+
+  BwdGroups grp{};
+  grp.G = N;
+  grp.max_rows = D.max_rows;
+  grp.seg_off = seg_off;
+  grp.seg_count = seg_count;
+  grp.flags = flags;
+  if (e == cudaSuccess) e = launch_dgrad_swiglu(grp, d, f, o, weights->w2, g, u, g, u, st);   // dG, dU in place
+  if (e == cudaSuccess) e = launch_wgrad(grp, d, f, xp, g, grads->dw1, st);
+  if (e == cudaSuccess) e = launch_wgrad(grp, d, f, xp, u, grads->dw3, st);
+  if (e == cudaSuccess) e = launch_wgrad(grp, f, d, h, o, grads->dw2, st);
+  if (e == cudaSuccess) e = launch_dgrad_plain2(grp, d, f, g, u, weights->w1, weights->w3, xp, st);   // dXp over xp
+  if (e == cudaSuccess)
+    e = launch_router_wgrad(T, d, N, static_cast<const uint16_t*>(x), a.dg, grads->dw_router, dbias,
+                            at<float*>(ws, B.rws), st);
+  float* dxr = at<float*>(ws, B.dxr);
+  if (e == cudaSuccess) e = launch_router_dgrad(T, d, N, a.dg, weights->w_router, dxr, st);
+  if (e != cudaSuccess) return cuda_status(e);
+
+  void* dxs = nullptr;
+  if (fs > 0) {  // the shared expert: one dense group of T rows, weight 1
+    void* gs = at<void*>(ws, B.gs);
+    void* us = at<void*>(ws, B.us);
+    void* hs = at<void*>(ws, B.hs);
+    dxs = at<void*>(ws, B.dxs);
+    if ((s = do_ffn(D, x, nullptr, nullptr, weights->ws1, weights->ws3, weights->ws2, fs, true, hs, dxs, ws, st, gs,
+                    us)) != MOE_OK)
+      return s;
+    BwdGroups dense{};
+    dense.G = 1;
+    dense.dense_rows = static_cast<int>(T);
+    dense.max_rows = T;
+    dense.flags = flags;
+    e = launch_dgrad_swiglu(dense, d, fs, dy, weights->ws2, gs, us, gs, us, st);
+    if (e == cudaSuccess) e = launch_wgrad(dense, d, fs, x, gs, grads->dws1, st);
+    if (e == cudaSuccess) e = launch_wgrad(dense, d, fs, x, us, grads->dws3, st);
+    if (e == cudaSuccess) e = launch_wgrad(dense, fs, d, hs, dy, grads->dws2, st);
+    if (e == cudaSuccess) e = launch_dgrad_plain2(dense, d, fs, gs, us, weights->ws1, weights->ws3, dxs, st);
+    if (e != cudaSuccess) return cuda_status(e);
+  }
+  return cuda_status(launch_dx_gather(T, d, k, row_map, static_cast<const uint16_t*>(xp), dxr,
+                                      static_cast<const uint16_t*>(dxs), static_cast<uint16_t*>(grads->dx), st));
 }
 
 moe_status_t moe_read_flags(const void* ws, size_t ws_bytes, uint32_t* flags, moe_stream_t stream) {

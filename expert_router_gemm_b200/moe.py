@@ -51,6 +51,11 @@ class moe_stats_t(ctypes.Structure):
                  "z_loss", "load_std", "top2_ratio", "avg_tokens_per_expert")]
 
 
+class moe_grads_t(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("dx", "dw_router", "drouter_bias", "dw1", "dw3", "dw2", "dws1", "dws3", "dws2")]
+
+
 _P = ctypes.c_void_p
 _SZ = ctypes.c_size_t
 _PROTOS = {
@@ -83,6 +88,10 @@ _PROTOS = {
     "moe_layer_fwd": (ctypes.c_int, [ctypes.POINTER(moe_config_t), ctypes.POINTER(moe_weights_t),
                                      _P, _P, ctypes.POINTER(moe_stats_t), _P, _SZ, _P]),
     "moe_read_flags": (ctypes.c_int, [_P, _SZ, ctypes.POINTER(ctypes.c_uint32), _P]),
+    "moe_backward_workspace_size": (ctypes.c_int, [ctypes.POINTER(moe_config_t), ctypes.POINTER(_SZ)]),
+    "moe_layer_bwd": (ctypes.c_int, [ctypes.POINTER(moe_config_t), ctypes.POINTER(moe_weights_t), _P, _P,
+                                     ctypes.c_float, ctypes.c_float, ctypes.POINTER(moe_grads_t), _P, _SZ,
+                                     _P]),
 }
 for _name, (_res, _args) in _PROTOS.items():
     _fn = getattr(_lib, _name)
@@ -279,6 +288,27 @@ def moe_layer_fwd(cfg, weights: moe_weights_t, x, y, stats, ws, stream=None):
     _check(_lib.moe_layer_fwd(ctypes.byref(cfg), ctypes.byref(weights), _ptr(x), _ptr(y),
                               _stats_ref(stats), _ptr(ws), ws.numel() if ws is not None else 0,
                               _stream(stream)), "moe_layer_fwd")
+
+
+def make_grads(dx=None, dw_router=None, drouter_bias=None, dw1=None, dw3=None, dw2=None, dws1=None,
+               dws3=None, dws2=None) -> moe_grads_t:
+    return moe_grads_t(*[_ptr(t) for t in (dx, dw_router, drouter_bias, dw1, dw3, dw2, dws1, dws3,
+                                           dws2)])
+
+
+def moe_backward_workspace_size(cfg) -> int:
+    b = _SZ()
+    _check(_lib.moe_backward_workspace_size(ctypes.byref(cfg), ctypes.byref(b)),
+           "moe_backward_workspace_size")
+    return b.value
+
+
+def moe_layer_bwd(cfg, weights: moe_weights_t, x, dy, aux_weight: float, z_weight: float,
+                  grads: moe_grads_t, ws, stream=None):
+    _check(_lib.moe_layer_bwd(ctypes.byref(cfg), ctypes.byref(weights), _ptr(x), _ptr(dy),
+                              ctypes.c_float(aux_weight), ctypes.c_float(z_weight),
+                              ctypes.byref(grads), _ptr(ws), ws.numel() if ws is not None else 0,
+                              _stream(stream)), "moe_layer_bwd")
 
 
 def moe_read_flags(ws, stream=None) -> int:

@@ -370,6 +370,41 @@ moe_status_t moe_layer_fwd(const moe_config_t* cfg, const moe_weights_t* weights
                            size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * Backward pass of one layer ("MoE 训练加速实战" §5.2: the training loss is the
+ * main loss plus a weighted auxiliary loss; "负载均衡策略": z_loss_weight;
+ * "ms-swift + Megatron：MoE模型加速10倍实测" §2.3: only the experts a token was
+ * routed to receive its gradient).  moe_layer_bwd returns the gradient of
+ *   L = <dy, y> + aux_weight * L_aux + z_weight * z_loss
+ * with y the output of moe_layer_fwd on the same inputs, L_aux = N sum_i f_i P_i
+ * (the l_aux_switch statistic: f_i the selection share, a count without
+ * gradient; P_i the mean softmax score) and z_loss the z_loss statistic.  The
+ * routing decisions (top-k set, capacity drops) carry no gradient, nor does the
+ * selection bias.  The call recomputes the forward pass from x (activation
+ * recomputation) and needs nothing saved from it.  bf16 layers with
+ * gemm_format MOE_GEMM_ACT and seg_align a multiple of 64 (MOE_ERR_UNSUPPORTED
+ * otherwise).  Weight gradients are fp32 and overwrite their buffers; dx is
+ * bf16.  Deterministic.
+ */
+typedef struct {
+  void* dx;              /* [T, d] bf16 */
+  float* dw_router;      /* [d, N] */
+  float* drouter_bias;   /* [N], or NULL; written only when weights->router_bias is set */
+  float* dw1;            /* [N][d][f] */
+  float* dw3;            /* [N][d][f] */
+  float* dw2;            /* [N][f][d] */
+  float* dws1;           /* [d][f_shared] (f_shared > 0), else NULL */
+  float* dws3;           /* [d][f_shared] */
+  float* dws2;           /* [f_shared][d] */
+} moe_grads_t;
+
+/* Bytes of the workspace of moe_layer_bwd. */
+moe_status_t moe_backward_workspace_size(const moe_config_t* cfg, size_t* bytes);
+
+moe_status_t moe_layer_bwd(const moe_config_t* cfg, const moe_weights_t* weights, const void* x,
+                           const void* dy, float aux_weight, float z_weight, moe_grads_t* grads,
+                           void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
  * moe_read_flags - wait for `stream`, then copy the workspace's device flags
  * word (MOE_FLAG_* bits, cleared by moe_route / moe_route_from_logits /
  * moe_layer_fwd) to *flags.  Returns MOE_ERR_NONFINITE or MOE_ERR_DEVICE when a
