@@ -244,6 +244,8 @@ def main():
     ap.add_argument("--aux-free", type=float, default=0.0, metavar="GAMMA",
                     help="Aux-Loss-Free routing: a selection bias, updated on the device with "
                          "this step size after every layer call (0 = off)")
+    ap.add_argument("--backward", action="store_true",
+                    help="also time moe_layer_bwd (forward recompute + backward) and report it")
     ap.add_argument("--gemm", default="act", choices=["act", "mxfp8"],
                     help="number format of the routed experts' GEMMs: the activation dtype, or "
                          "block-scaled FP8 (weights quantized once before the timed region)")
@@ -574,6 +576,55 @@ def main():
                        "copies": "overlapped with the neighbouring steps' compute (2 copy streams)",
                        "serial_value": round(world * T / (serial_ms / 1e3), 1),
                        "serial_ms_per_step": round(serial_ms, 4)}
+
+    if args.backward and not mx:
+        # -------------------------------------------- the layer backward
+        # One step = moe_layer_bwd: the forward recomputed from x (routing, permutation,
+        # GEMM1 saving g and u, GEMM2), then the gradients of every input and weight.
+        T, N, k, d, f, fs = w.T, w.N, w.k, w.d, w.f, w.f_shared
+        gb = dict(dx=torch.empty((T, d), dtype=act, device="cuda"),
+                  dw_router=torch.empty((d, N), device="cuda"),
+                  drouter_bias=torch.empty(N, device="cuda") if dl.bias is not None else None,
+                  dw1=torch.empty((N, d, f), device="cuda"), dw3=torch.empty((N, d, f), device="cuda"),
+                  dw2=torch.empty((N, f, d), device="cuda"))
+        if fs:
+            gb.update(dws1=torch.empty((d, fs), device="cuda"), dws3=torch.empty((d, fs), device="cuda"),
+                      dws2=torch.empty((fs, d), device="cuda"))
+        grads = moe.make_grads(**gb)
+        ws_b = torch.empty(moe.moe_backward_workspace_size(cfg), dtype=torch.uint8, device="cuda")
+        dy = torch.randn((T, d), generator=torch.Generator().manual_seed(5)).to(torch.bfloat16).view(
+            torch.int16).cuda()
+
+        def bwd_step():
+            moe.moe_layer_bwd(cfg, weights, dl.x, dy, 0.01, 1e-3, grads, ws_b, stream)
+
+        for _ in range(max(3, args.warmup)):
+            bwd_step()
+        torch.cuda.synchronize()
+        bflags = moe.moe_read_flags(ws_b)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_b = max(1, args.steps // 2)
+        bsampler = ClockSampler(local)
+        barrier()
+        torch.cuda.synchronize()
+        with bsampler:
+            e0.record(stream)
+            for _ in range(n_b):
+                bwd_step()
+            e1.record(stream)
+            torch.cuda.synchronize()
+        barrier()
+        bms = max_over_ranks(e0.elapsed_time(e1)) / n_b
+        # GEMM work of one step: forward recompute (6 d f per kept row), dgrad (6 d f)
+        # and weight gradients (6 d f), plus the shared expert's 2 + 4 + 6 d fs per token
+        gemm_fl = 18.0 * d * f * a_kept + (12.0 + 6.0) * T * d * fs
+        peaks, peak_src = load_peaks()
+        line["backward"] = {
+            "what": "moe_layer_bwd: forward recomputed from x, then dx and every weight gradient (fp32)",
+            "steps": n_b, "ms_per_step": round(bms, 4), "tokens/s": round(world * T / (bms / 1e3), 1),
+            "gemm_flops_per_step": gemm_fl, "gemm_TFLOP/s": round(gemm_fl / (bms / 1e3) / 1e12, 1),
+            "frac_of_sustained_bf16_peak": round(gemm_fl / (bms / 1e3) / 1e12 / peaks["bf16_tflops_sustained"], 4),
+            "peak_source": peak_src, "device_flags": bflags, "clocks": bsampler.summary()}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.quick:
         steps, t_route = oracle_expert_steps(w, inp, budget_s=args.cpu_budget, mx=mx)

@@ -29,7 +29,7 @@ workload gets the gradient sum_t dg_t like any additive bias.
 from __future__ import annotations
 
 from dataclasses import dataclass
-from typing import Optional
+from typing import Optional, Sequence
 
 import numpy as np
 
@@ -74,7 +74,11 @@ def expert_backward(x64, w1, w3, w2, dout):
 def layer_backward(x, w_router, bias, w1, w3, w2, dy, k: int, capacity_factor: float = 1.0,
                    cap: Optional[int] = None, ws1=None, ws3=None, ws2=None, align: int = 128,
                    aux_weight: float = 0.0, z_weight: float = 0.0,
-                   selection_bias: Optional[np.ndarray] = None) -> LayerGrads:
+                   selection_bias: Optional[np.ndarray] = None,
+                   weight_experts: Optional[Sequence[int]] = None) -> LayerGrads:
+    """With weight_experts, dw1 / dw3 / dw2 hold only those experts' gradients,
+    in that order (the full arrays of a large layer do not fit in memory); every
+    other gradient is complete."""
     T, d = x.shape
     N = w_router.shape[1]
     fwd = orc.layer_forward(x, w_router, bias, w1, w3, w2, k=k, capacity_factor=capacity_factor,
@@ -86,9 +90,11 @@ def layer_backward(x, w_router, bias, w1, w3, w2, dy, k: int, capacity_factor: f
     kept = fwd.disp.row_map >= 0
 
     dx = np.zeros((T, d))
-    dw1 = np.zeros(np.shape(w1))
-    dw3 = np.zeros(np.shape(w3))
-    dw2 = np.zeros(np.shape(w2))
+    keep_w = list(range(N)) if weight_experts is None else [int(e) for e in weight_experts]
+    slot = {e: i for i, e in enumerate(keep_w)}
+    dw1 = np.zeros((len(keep_w),) + np.shape(w1)[1:])
+    dw3 = np.zeros((len(keep_w),) + np.shape(w3)[1:])
+    dw2 = np.zeros((len(keep_w),) + np.shape(w2)[1:])
     dwt = np.zeros((T, k))
     for e in range(N):
         ti, tj = np.nonzero((idx == e) & kept)
@@ -97,8 +103,10 @@ def layer_backward(x, w_router, bias, w1, w3, w2, dy, k: int, capacity_factor: f
         xe = x64[ti]
         o = orc.swiglu_ffn(xe, w1[e], w3[e], w2[e], False)
         dwt[ti, tj] = np.sum(dy[ti] * o, axis=1)            # y = sum_j w_j o_j
-        dxe, dw1[e], dw3[e], dw2[e] = expert_backward(xe, w1[e], w3[e], w2[e], w[ti, tj][:, None] * dy[ti])
+        dxe, g1, g3, g2 = expert_backward(xe, w1[e], w3[e], w2[e], w[ti, tj][:, None] * dy[ti])
         np.add.at(dx, ti, dxe)
+        if e in slot:
+            dw1[slot[e]], dw3[slot[e]], dw2[slot[e]] = g1, g3, g2
 
     dws1 = dws3 = dws2 = None
     if ws1 is not None:                    # shared expert, weight 1
