@@ -160,8 +160,8 @@ constexpr int kChunkRows = 512;  // rows of T per partial of the weight gradient
 // partial holds sum_t dg[t][i] (the bias), computed as x = 1.
 __global__ void __launch_bounds__(256) router_wgrad_kernel(int64_t T, int d, int N, const uint16_t* __restrict__ x,
                                                           const float* __restrict__ dg, float* __restrict__ part) {
-  __shared__ float xs[RK][RT + 4];
-  __shared__ float gs[RK][RT + 4];
+  __shared__ __align__(16) float xs[RK][RT + 4];
+  __shared__ __align__(16) float gs[RK][RT + 4];
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;   // 16 x 16 threads, 4 x 4 outputs each
   const int c0 = blockIdx.x * RT, i0 = blockIdx.y * RT;
   const bool bias_tile = c0 >= d;
@@ -186,12 +186,10 @@ __global__ void __launch_bounds__(256) router_wgrad_kernel(int64_t T, int d, int
     __syncthreads();
 #pragma unroll 8
     for (int r = 0; r < RK; ++r) {
-      float xa[4], ga[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        xa[q] = xs[r][ty * 4 + q];
-        ga[q] = gs[r][tx * 4 + q];
-      }
+      const float4 x4 = *reinterpret_cast<const float4*>(&xs[r][ty * 4]);
+      const float4 g4 = *reinterpret_cast<const float4*>(&gs[r][tx * 4]);
+      const float xa[4] = {x4.x, x4.y, x4.z, x4.w};
+      const float ga[4] = {g4.x, g4.y, g4.z, g4.w};
 #pragma unroll
       for (int a = 0; a < 4; ++a)
 #pragma unroll
@@ -229,8 +227,8 @@ __global__ void router_wgrad_reduce_kernel(int n_chunks, int d, int N, const flo
 // dxr[t][c] = sum_i dg[t][i] W_r[c][i]
 __global__ void __launch_bounds__(256) router_dgrad_kernel(int64_t T, int d, int N, const float* __restrict__ dg,
                                                           const float* __restrict__ wr, float* __restrict__ dxr) {
-  __shared__ float gs[RK][RT + 4];   // [i][t]
-  __shared__ float ws[RK][RT + 4];   // [i][c]
+  __shared__ __align__(16) float gs[RK][RT + 4];   // [i][t]
+  __shared__ __align__(16) float ws[RK][RT + 4];   // [i][c]
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
   const int64_t t0 = static_cast<int64_t>(blockIdx.x) * RT;
   const int c0 = blockIdx.y * RT;
@@ -246,12 +244,10 @@ __global__ void __launch_bounds__(256) router_dgrad_kernel(int64_t T, int d, int
     __syncthreads();
 #pragma unroll 8
     for (int i = 0; i < RK; ++i) {
-      float ga[4], wa[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        ga[q] = gs[i][ty * 4 + q];
-        wa[q] = ws[i][tx * 4 + q];
-      }
+      const float4 g4 = *reinterpret_cast<const float4*>(&gs[i][ty * 4]);
+      const float4 w4 = *reinterpret_cast<const float4*>(&ws[i][tx * 4]);
+      const float ga[4] = {g4.x, g4.y, g4.z, g4.w};
+      const float wa[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
       for (int a = 0; a < 4; ++a)
 #pragma unroll

@@ -70,7 +70,11 @@ struct Tail {
   int32_t count[kMaxGroups];   // dgrad: kept rows; wgrad: padded rows (the reduction length)
 };
 
-constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(STAGES) * STAGE_BYTES + sizeof(Tail);
+// fp32 output staging of the weight-gradient epilogue: one 32 x 32 block
+// (4 KB, 128-byte swizzled as the TMA store reads it) per epilogue warp
+constexpr int kStageBlock = 32 * 32 * 4;
+constexpr size_t kStagingBytes = 4 * kStageBlock;
+constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(STAGES) * STAGE_BYTES + kStagingBytes + sizeof(Tail);
 
 struct Tile {
   int g, m0, n0;
@@ -136,7 +140,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = base;
   uint8_t* sB = base + STAGES * A_BYTES;
-  Tail& tl = *reinterpret_cast<Tail*>(base + STAGES * STAGE_BYTES);
+  uint8_t* sStage = base + STAGES * STAGE_BYTES;   // 1024-byte aligned
+  Tail& tl = *reinterpret_cast<Tail*>(sStage + kStagingBytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int unit = static_cast<int>(blockIdx.x), n_units = static_cast<int>(gridDim.x);
@@ -330,14 +335,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (col >= p.n_out) continue;
         if (KIND == KIND_WGRAD) {
-          const int m = tile.m0 + r_in_tile;
-          if (m >= p.M) continue;
-          float* dst = static_cast<float*>(p.out0) + (static_cast<int64_t>(tile.g) * p.M + m) * p.n_out + col;
-          float4* d4 = reinterpret_cast<float4*>(dst);
+          // the warp's 32 rows x 32 columns go to its staging block in the
+          // 128-byte swizzled layout (16-byte chunk q of row r at chunk q ^ (r % 8):
+          // conflict-free), then one TMA store writes the block to dW[g]; the
+          // 3-D tensor map clips rows past M and columns past n_out
+          const int m_first = tile.m0 + quad * 32;
+          if (m_first < p.M) {
+            uint8_t* stg = sStage + quad * kStageBlock;
+            if (lane == 0) bulk_wait_read_all();   // this warp's previous store has read the block
+            __syncwarp();
 #pragma unroll
-          for (int q = 0; q < 8; ++q)
-            d4[q] = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]), __uint_as_float(v[4 * q + 2]),
-                                __uint_as_float(v[4 * q + 3]));
+            for (int q = 0; q < 8; ++q)
+              *reinterpret_cast<float4*>(stg + lane * 128 + ((q ^ (lane & 7)) << 4)) =
+                  make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]), __uint_as_float(v[4 * q + 2]),
+                              __uint_as_float(v[4 * q + 3]));
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_3d(&tmA1, smem_addr(stg), col, m_first, tile.g);
+              bulk_commit();
+            }
+          }
         } else {
           const int row = tile.m0 + r_in_tile;
           const bool valid = row < tl.count[tile.g];
@@ -381,6 +399,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         acc_phase ^= 1u;
       }
     }
+    if (KIND == KIND_WGRAD && lane == 0) bulk_wait_all();   // every store issued by this warp has landed
   }
 
   __syncwarp();
@@ -463,14 +482,15 @@ cudaError_t launch_wgrad(const BwdGroups& s, int M, int N, const void* a, const 
                          cudaStream_t st) {
   if (s.max_rows <= 0) return cudaSuccess;
   const int G = s.seg_off != nullptr ? s.G : 1;
-  CUtensorMap mA, mB;
-  if (!make_tma_2d_bf16(&mA, a, M, s.max_rows, 64, BK) || !make_tma_2d_bf16(&mB, b, N, s.max_rows, 64, BK))
+  CUtensorMap mA, mB, mOut;
+  if (!make_tma_2d_bf16(&mA, a, M, s.max_rows, 64, BK) || !make_tma_2d_bf16(&mB, b, N, s.max_rows, 64, BK) ||
+      !make_tma_3d_f32_sw128(&mOut, out, N, M, G, 32, 32))
     return cudaErrorInvalidValue;
   BwdParams p = base_params(s);
   p.M = M;
   p.n_out = N;
   p.out0 = out;
-  return launch<KIND_WGRAD>(mA, mA, mB, mB, p,
+  return launch<KIND_WGRAD>(mA, mOut, mB, mB, p,
                             static_cast<int64_t>(G) * ((M + BM - 1) / BM) * ((N + MMA_N - 1) / MMA_N), st);
 }
 

@@ -68,6 +68,10 @@ cudaError_t launch_router_tc(const RouteArgs& a, void* split, float* partials, i
 // swizzle, zero fill outside the tensor.
 bool make_tma_2d_bf16(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint32_t box_inner,
                       uint32_t box_outer);
+// 3-D fp32 tensor map [outer][mid][inner] (inner contiguous), 128-byte swizzle,
+// for tiled stores of [box_mid x box_inner] blocks (box_inner * 4 == 128).
+bool make_tma_3d_f32_sw128(CUtensorMap* m, void* ptr, uint64_t inner, uint64_t mid, uint64_t outer, uint32_t box_inner,
+                           uint32_t box_mid);
 // The same over bytes (FP8 codes).
 bool make_tma_2d_u8(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint32_t box_inner,
                     uint32_t box_outer);

@@ -49,6 +49,19 @@ bool make_tma_2d_bf16(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t 
   return make_2d(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ptr, inner, outer, box_inner, box_outer);
 }
 
+bool make_tma_3d_f32_sw128(CUtensorMap* m, void* ptr, uint64_t inner, uint64_t mid, uint64_t outer, uint32_t box_inner,
+                           uint32_t box_mid) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[3] = {inner, mid, outer};
+  const cuuint64_t strides[2] = {inner * 4, inner * mid * 4};
+  const cuuint32_t box[3] = {box_inner, box_mid, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, ptr, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool make_tma_2d_u8(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint32_t box_inner,
                     uint32_t box_outer) {
   return make_2d(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ptr, inner, outer, box_inner, box_outer);
