@@ -323,6 +323,23 @@ __device__ __forceinline__ void tc_mma_mxf8(uint32_t d_tmem, uint64_t adesc, uin
       : "memory");
 }
 
+// CTA-pair forms (issued by the even CTA): the copy moves each CTA's 32x128b
+// block from its own shared memory (same offset) into its own TMEM; the MMA
+// computes a 256-row tile, each CTA holding its 128 rows' scales of A and the
+// scales of all B columns.
+__device__ __forceinline__ void tc_cp_32x128b_x4_pair(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+__device__ __forceinline__ void tc_mma_mxf8_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                                 uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+      : "memory");
+}
+
 // Shared exponent of a block of 32 values with largest magnitude `amax` (>= 0):
 // the smallest e in [-127, 127] with amax <= 448 * 2^e.  With amax = M 2^E,
 // M in [1, 2): e = E - 8 if M <= 1.75, else E - 7 (integer logic on the bits;

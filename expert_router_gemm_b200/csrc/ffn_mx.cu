@@ -10,14 +10,23 @@
 //                   (blocks of 32 along f) in the epilogue -> codes + scales
 //   GEMM2 (PLAIN):  out[r] = h[r] W2_e -> bf16
 //
-// Per CTA (one per SM, 192 threads), one 128 x 256 tile at a time:
+// Persistent, 192 threads per CTA, one CTA per SM:
 //   warp 0 lane 0   producer: per K stage of 128 values (128 bytes per row),
-//                   TMA loads of A (128 rows) and B (256 K-major weight rows,
-//                   two boxes), plus three 512-byte scale atoms (bulk copies);
-//   warp 1          allocates all 512 TMEM columns; lane 0 copies the stage's
-//                   scale atoms into TMEM (tcgen05.cp) and issues four K=32 MMAs
-//                   whose scale-factor id picks the 32-value block;
+//                   TMA loads of A and of the K-major weight rows, plus the
+//                   stage's 512-byte scale atoms (A, and B rows 0-127 / 128-255);
+//   warp 1          allocates all 512 TMEM columns; lane 0 copies the scale
+//                   atoms into TMEM (tcgen05.cp) and issues four K=32 MMAs whose
+//                   scale-factor id picks the 32-value block;
 //   warps 2-5       epilogue (tcgen05.ld, SwiGLU + FP8 quantization or bf16).
+// CG = 1: a CTA computes a 128 x 256 tile alone (M=128 MMA), four stages of
+//   16 KB A + 32 KB B + 1.5 KB scales.
+// CG = 2: a cluster of two CTAs computes a 256 x 256 tile with one
+//   cta_group::2 MMA issued by the even CTA; each CTA stages its own 128 rows of
+//   A, its own 128 rows of B (SwiGLU: CTA 0 the W1 rows, CTA 1 the W3 rows) and
+//   the scales of its A rows and of all 256 B rows (the B scales are needed by
+//   both halves of the tile), six stages of 33.5 KB.  Every load is a TMA tensor
+//   load counted on the even CTA's barrier; the MMA commits to both CTAs'
+//   barriers; both epilogues release the accumulator on the even CTA's barrier.
 // TMEM: accumulator 0 at columns [0, 256), accumulator 1 at [224, 480) and the
 // scales at [480, 492).  The two accumulators share 32 columns so that both fit
 // beside the scales; the epilogue drains buffer 0 from its last 32 columns
@@ -29,6 +38,7 @@
 #include <cuda_fp8.h>
 
 #include <algorithm>
+#include <cstdlib>
 #include <mutex>
 
 #include "device_utils.cuh"
@@ -37,17 +47,14 @@
 namespace moe {
 namespace {
 
-constexpr int BM = 128;                    // rows per tile
+constexpr int BM = 128;                    // rows per CTA
 constexpr int BK = 128;                    // K per stage (bytes per row)
 constexpr int MMA_N = 256;
 constexpr int MMA_K = 32;
 constexpr int A_BYTES = BM * BK;           // 16 KB
 constexpr int B_HALF = 128 * BK;           // 16 KB: 128 weight rows
-constexpr int B_BYTES = 2 * B_HALF;        // 32 KB
 constexpr int SF_ATOM = 512;               // scales of 128 rows x 4 K blocks
 constexpr int SF_BYTES = 3 * SF_ATOM;      // A atom + two B atoms
-constexpr int STAGES = 4;
-constexpr int STAGE_TX = A_BYTES + B_BYTES + SF_BYTES;
 constexpr int kThreads = 192;
 constexpr int kTmemCols = 512;
 constexpr uint32_t kAcc1Col = 224;         // accumulator 1 starts here (shares [224, 256))
@@ -57,6 +64,14 @@ constexpr int kMaxGroups = 256;
 
 enum { MODE_SWIGLU = 0, MODE_PLAIN = 1 };
 
+template <int CG>
+struct Cfg {
+  static constexpr int B_BYTES = CG == 1 ? 2 * B_HALF : B_HALF;   // B rows staged by one CTA
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SF_BYTES;
+  static constexpr int STAGES = CG == 1 ? 4 : 6;
+  static constexpr int TILE_M = BM * CG;
+};
+
 struct MxParams {
   const int32_t* seg_off;
   const int32_t* seg_count;
@@ -64,7 +79,7 @@ struct MxParams {
   int64_t max_rows;
   int K;                     // reduction length (multiple of 128)
   int n_out;                 // output columns (multiple of 128)
-  const uint8_t* a_sf;       // scales of A
+  const uint8_t* a_sf;       // scales of A (CG = 1: bulk copies; CG = 2: TMA maps)
   const uint8_t* b0_sf;      // scales of B (W1 or W2)
   const uint8_t* b1_sf;      // scales of W3 (SwiGLU)
   uint8_t* out8;             // SwiGLU: h codes [max_rows, n_out]
@@ -74,8 +89,8 @@ struct MxParams {
 };
 
 struct MxTail {
-  uint64_t full[STAGES];
-  uint64_t empty[STAGES];
+  uint64_t full[6];
+  uint64_t empty[6];
   uint64_t tfull[2];
   uint64_t drained;          // epilogue read the columns shared with the next tile's accumulator
   uint64_t drain;
@@ -86,13 +101,16 @@ struct MxTail {
   int32_t count[kMaxGroups];
 };
 
-constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(STAGES) * (A_BYTES + B_BYTES + SF_BYTES) + sizeof(MxTail);
+template <int CG>
+constexpr size_t smem_bytes() {
+  return 1024 + static_cast<size_t>(Cfg<CG>::STAGES) * Cfg<CG>::STAGE_BYTES + sizeof(MxTail);
+}
 
 struct Tile {
   int g, m0, n0;
 };
 
-__device__ __forceinline__ Tile decode_tile(const MxTail& s, int G, int bn, int t) {
+__device__ __forceinline__ Tile decode_tile(const MxTail& s, int G, int bn, int tile_m, int t) {
   int lo = 0, hi = G;  // largest g with tile_start[g] <= t
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
@@ -102,11 +120,11 @@ __device__ __forceinline__ Tile decode_tile(const MxTail& s, int G, int bn, int 
       hi = mid;
   }
   const int local = t - s.tile_start[lo];
-  const int mt = (s.count[lo] + BM - 1) / BM;
+  const int mt = (s.count[lo] + tile_m - 1) / tile_m;
   Tile r;
   r.g = lo;
   r.n0 = (local / mt) * bn;
-  r.m0 = (local % mt) * BM;
+  r.m0 = (local % mt) * tile_m;
   return r;
 }
 
@@ -120,34 +138,40 @@ __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
   return lo | (hi << 16);
 }
 
-template <int MODE>
+// Scale atoms as TMA tensors (CG = 2): the scale buffer viewed as [atoms * 4]
+// rows of 128 bytes, one atom = a 4-row box.
+template <int MODE, int CG>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_mx_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
-                      const __grid_constant__ CUtensorMap tmB1, const MxParams p) {
+                      const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmSA,
+                      const __grid_constant__ CUtensorMap tmSB0, const __grid_constant__ CUtensorMap tmSB1,
+                      const MxParams p) {
+  using C = Cfg<CG>;
   constexpr int BN = MODE == MODE_SWIGLU ? MMA_N / 2 : MMA_N;  // output columns per tile
   extern __shared__ uint8_t dsmem[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = base;
-  uint8_t* sB = base + STAGES * A_BYTES;
-  uint8_t* sSF = sB + STAGES * B_BYTES;
-  MxTail& tl = *reinterpret_cast<MxTail*>(sSF + STAGES * SF_BYTES);
+  uint8_t* sB = base + C::STAGES * A_BYTES;
+  uint8_t* sSF = sB + C::STAGES * C::B_BYTES;
+  MxTail& tl = *reinterpret_cast<MxTail*>(sSF + C::STAGES * SF_BYTES);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int unit = static_cast<int>(blockIdx.x);
-  const int n_units = static_cast<int>(gridDim.x);
+  const uint32_t rank = CG == 2 ? cluster_ctarank() : 0u;   // 0: this CTA issues the MMAs
+  const int unit = CG == 2 ? static_cast<int>(blockIdx.x) / 2 : static_cast<int>(blockIdx.x);
+  const int n_units = CG == 2 ? static_cast<int>(gridDim.x) / 2 : static_cast<int>(gridDim.x);
   const int G = p.G;
   const int n_tiles = (p.n_out + BN - 1) / BN;
   const int KT = p.K / BK;            // K stages (= scale atoms per 128-row tile)
   const int NT = p.n_out / 128;       // 128-row tiles of one expert's weight
 
   if (warp == 0 && lane == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(smem_addr(&tl.full[s]), 1);
       mbar_init(smem_addr(&tl.empty[s]), 1);
     }
     mbar_init(smem_addr(&tl.tfull[0]), 1);
     mbar_init(smem_addr(&tl.tfull[1]), 1);
-    mbar_init(smem_addr(&tl.drained), 128);
+    mbar_init(smem_addr(&tl.drained), 128 * CG);
     mbar_init(smem_addr(&tl.drain), 1);
     tl.abort = 0u;
     fence_mbar_init();
@@ -156,8 +180,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (MODE == MODE_SWIGLU) tma_prefetch_desc(&tmB1);
   }
   if (warp == 1) {
-    tmem_alloc(smem_addr(&tl.tmem_base), kTmemCols);
-    tmem_relinquish();
+    if (CG == 2) {
+      tmem_alloc_pair(smem_addr(&tl.tmem_base), kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_addr(&tl.tmem_base), kTmemCols);
+      tmem_relinquish();
+    }
   }
   if (warp == 2) {
     const int per = (G + 31) / 32;
@@ -172,7 +201,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tl.row0[g] = r0;
       tl.count[g] = c;
-      local += (c + BM - 1) / BM * n_tiles;
+      local += (c + C::TILE_M - 1) / C::TILE_M * n_tiles;
     }
     int incl = local;
 #pragma unroll
@@ -183,12 +212,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     int run = incl - local;
     for (int g = g_lo; g < g_hi; ++g) {
       tl.tile_start[g] = run;
-      run += (tl.count[g] + BM - 1) / BM * n_tiles;
+      run += (tl.count[g] + C::TILE_M - 1) / C::TILE_M * n_tiles;
     }
     if (lane == 31) tl.tile_start[G] = incl;
   }
   tc_fence_before();
-  __syncthreads();
+  if (CG == 2)
+    cluster_sync();  // both CTAs' barriers are initialised before any cross-CTA signal
+  else
+    __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = tl.tmem_base;
   const int total = tl.tile_start[G];
@@ -200,52 +232,72 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t stage = 0, phase = 0, issued = 0, last_par = 0;
       bool ok = true;
       for (int t = unit; ok && t < total; t += n_units) {
-        const Tile tile = decode_tile(tl, G, BN, t);
-        const int a_row = tl.row0[tile.g] + tile.m0;
-        const int b_row = tile.g * p.n_out + tile.n0;
-        const uint8_t* sfa = p.a_sf + static_cast<int64_t>(a_row / BM) * KT * SF_ATOM;
+        const Tile tile = decode_tile(tl, G, BN, C::TILE_M, t);
+        const int a_row = tl.row0[tile.g] + tile.m0 + static_cast<int>(rank) * BM;
+        // B rows this CTA stages: CG = 1 all 256; CG = 2 its 128
+        const int b_row = tile.g * p.n_out + tile.n0 + (MODE == MODE_PLAIN ? static_cast<int>(rank) * 128 : 0);
         const int nt0 = tile.n0 / 128;
         const int nt1 = MODE == MODE_SWIGLU ? nt0 : min(nt0 + 1, NT - 1);
-        const uint8_t* sfb0 = p.b0_sf + (static_cast<int64_t>(tile.g) * NT + nt0) * KT * SF_ATOM;
-        const uint8_t* sfb1 = (MODE == MODE_SWIGLU ? p.b1_sf : p.b0_sf) +
-                              (static_cast<int64_t>(tile.g) * NT + nt1) * KT * SF_ATOM;
+        const int64_t sfa_atom = static_cast<int64_t>(a_row / BM) * KT;
+        const int64_t sfb0_atom = (static_cast<int64_t>(tile.g) * NT + nt0) * KT;
+        const int64_t sfb1_atom = (static_cast<int64_t>(tile.g) * NT + nt1) * KT;
         for (int kb = 0; kb < KT; ++kb) {
           if (!mbar_wait(smem_addr(&tl.empty[stage]), phase ^ 1u, abort, p.flags, kFlagTimeout)) {
             ok = false;
             break;
           }
-          const uint32_t fb = smem_addr(&tl.full[stage]);
+          const uint32_t fb_local = smem_addr(&tl.full[stage]);
           const uint32_t a_dst = smem_addr(sA + stage * A_BYTES);
-          const uint32_t b_dst = smem_addr(sB + stage * B_BYTES);
+          const uint32_t b_dst = smem_addr(sB + stage * C::B_BYTES);
           const uint32_t sf_dst = smem_addr(sSF + stage * SF_BYTES);
-          mbar_arrive_expect_tx(fb, STAGE_TX);
-          tma_load_2d(a_dst, &tmA, fb, kb * BK, a_row);
-          if (MODE == MODE_SWIGLU) {
-            tma_load_2d(b_dst, &tmB0, fb, kb * BK, b_row);           // W1 rows n0 .. n0+127
-            tma_load_2d(b_dst + B_HALF, &tmB1, fb, kb * BK, b_row);  // W3 rows n0 .. n0+127
+          if (CG == 1) {
+            mbar_arrive_expect_tx(fb_local, C::STAGE_BYTES);
+            tma_load_2d(a_dst, &tmA, fb_local, kb * BK, a_row);
+            if (MODE == MODE_SWIGLU) {
+              tma_load_2d(b_dst, &tmB0, fb_local, kb * BK, b_row);           // W1 rows n0 .. n0+127
+              tma_load_2d(b_dst + B_HALF, &tmB1, fb_local, kb * BK, b_row);  // W3 rows n0 .. n0+127
+            } else {
+              tma_load_2d(b_dst, &tmB0, fb_local, kb * BK, b_row);
+              tma_load_2d(b_dst + B_HALF, &tmB0, fb_local, kb * BK, b_row + 128);
+            }
+            bulk_load(sf_dst, p.a_sf + (sfa_atom + kb) * SF_ATOM, SF_ATOM, fb_local);
+            bulk_load(sf_dst + SF_ATOM, p.b0_sf + (sfb0_atom + kb) * SF_ATOM, SF_ATOM, fb_local);
+            bulk_load(sf_dst + 2 * SF_ATOM, (MODE == MODE_SWIGLU ? p.b1_sf : p.b0_sf) + (sfb1_atom + kb) * SF_ATOM,
+                      SF_ATOM, fb_local);
           } else {
-            tma_load_2d(b_dst, &tmB0, fb, kb * BK, b_row);
-            tma_load_2d(b_dst + B_HALF, &tmB0, fb, kb * BK, b_row + 128);
+            // both CTAs' bytes complete on the even CTA's barrier
+            const uint32_t fb = rank == 0 ? fb_local : mapa_shared(fb_local, 0);
+            if (rank == 0) mbar_arrive_expect_tx(fb_local, 2 * C::STAGE_BYTES);
+            tma_load_2d_pair(a_dst, &tmA, fb, kb * BK, a_row);
+            tma_load_2d_pair(b_dst, (MODE == MODE_SWIGLU && rank == 1) ? &tmB1 : &tmB0, fb, kb * BK, b_row);
+            tma_load_2d_pair(sf_dst, &tmSA, fb, 0, static_cast<int>((sfa_atom + kb) * 4));
+            tma_load_2d_pair(sf_dst + SF_ATOM, &tmSB0, fb, 0, static_cast<int>((sfb0_atom + kb) * 4));
+            tma_load_2d_pair(sf_dst + 2 * SF_ATOM, MODE == MODE_SWIGLU ? &tmSB1 : &tmSB0, fb, 0,
+                             static_cast<int>((sfb1_atom + kb) * 4));
           }
-          bulk_load(sf_dst, sfa + kb * SF_ATOM, SF_ATOM, fb);
-          bulk_load(sf_dst + SF_ATOM, sfb0 + kb * SF_ATOM, SF_ATOM, fb);
-          bulk_load(sf_dst + 2 * SF_ATOM, sfb1 + kb * SF_ATOM, SF_ATOM, fb);
           issued |= 1u << stage;
           last_par = (last_par & ~(1u << stage)) | (phase << stage);
-          if (++stage == STAGES) {
+          if (++stage == C::STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
       }
-      // every copy issued by this thread has landed before the CTA may exit
-      for (int s = 0; s < STAGES; ++s)
-        if ((issued >> s) & 1u) mbar_wait(smem_addr(&tl.full[s]), (last_par >> s) & 1u, nullptr, p.flags, kFlagTimeout);
+      // Every copy issued by this thread has landed before the CTA may exit: the
+      // even CTA sees its barrier complete; the odd CTA sees the MMA that
+      // consumed the load release the stage.
+      for (int s = 0; s < C::STAGES; ++s)
+        if ((issued >> s) & 1u) {
+          if (rank == 0)
+            mbar_wait(smem_addr(&tl.full[s]), (last_par >> s) & 1u, nullptr, p.flags, kFlagTimeout);
+          else
+            mbar_wait(smem_addr(&tl.empty[s]), (last_par >> s) & 1u, nullptr, p.flags, kFlagTimeout);
+        }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    if (lane == 0 && rank == 0) {
       // ---------------------------------------------------------------- MMA issuer
-      uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0, j = 0;
+      uint32_t stage = 0, phase = 0, acc = 0, j = 0;
       bool ok = true, issued_any = false;
       for (int t = unit; ok && t < total; t += n_units, ++j) {
         // the previous tile's epilogue has read the columns this accumulator shares with it
@@ -260,47 +312,70 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
           const uint32_t a_addr = smem_addr(sA + stage * A_BYTES);
-          const uint32_t b_addr = smem_addr(sB + stage * B_BYTES);
+          const uint32_t b_addr = smem_addr(sB + stage * C::B_BYTES);
           const uint32_t sf_addr = smem_addr(sSF + stage * SF_BYTES);
           // scale atoms -> TMEM (executed in order with the MMAs issued around them)
-          tc_cp_32x128b_x4(tmem_base + kSfaCol, smem_desc_plain(sf_addr, 16, 128));
-          tc_cp_32x128b_x4(tmem_base + kSfbCol, smem_desc_plain(sf_addr + SF_ATOM, 16, 128));
-          tc_cp_32x128b_x4(tmem_base + kSfbCol + 4, smem_desc_plain(sf_addr + 2 * SF_ATOM, 16, 128));
+          if (CG == 2) {
+            tc_cp_32x128b_x4_pair(tmem_base + kSfaCol, smem_desc_plain(sf_addr, 16, 128));
+            tc_cp_32x128b_x4_pair(tmem_base + kSfbCol, smem_desc_plain(sf_addr + SF_ATOM, 16, 128));
+            tc_cp_32x128b_x4_pair(tmem_base + kSfbCol + 4, smem_desc_plain(sf_addr + 2 * SF_ATOM, 16, 128));
+          } else {
+            tc_cp_32x128b_x4(tmem_base + kSfaCol, smem_desc_plain(sf_addr, 16, 128));
+            tc_cp_32x128b_x4(tmem_base + kSfbCol, smem_desc_plain(sf_addr + SF_ATOM, 16, 128));
+            tc_cp_32x128b_x4(tmem_base + kSfbCol + 4, smem_desc_plain(sf_addr + 2 * SF_ATOM, 16, 128));
+          }
 #pragma unroll
           for (int kk = 0; kk < BK / MMA_K; ++kk) {
             // A and B K-major: advance 32 values (32 bytes) inside the swizzle row
             const uint64_t adesc = smem_desc_sw128(a_addr + kk * 32, 16, 1024);
             const uint64_t bdesc = smem_desc_sw128(b_addr + kk * 32, 16, 1024);
             const uint32_t sel = static_cast<uint32_t>(kk) << 30;   // scale byte kk of each word
-            tc_mma_mxf8(d_tmem, adesc, bdesc, idesc_mxf8(BM, MMA_N, static_cast<uint32_t>(kk)),
-                        (tmem_base + kSfaCol) | sel, (tmem_base + kSfbCol) | sel, (kb | kk) != 0 ? 1u : 0u);
+            const uint32_t idesc = idesc_mxf8(C::TILE_M, MMA_N, static_cast<uint32_t>(kk));
+            if (CG == 2)
+              tc_mma_mxf8_pair(d_tmem, adesc, bdesc, idesc, (tmem_base + kSfaCol) | sel, (tmem_base + kSfbCol) | sel,
+                               (kb | kk) != 0 ? 1u : 0u);
+            else
+              tc_mma_mxf8(d_tmem, adesc, bdesc, idesc, (tmem_base + kSfaCol) | sel, (tmem_base + kSfbCol) | sel,
+                          (kb | kk) != 0 ? 1u : 0u);
           }
-          tc_commit(smem_addr(&tl.empty[stage]));
-          if (++stage == STAGES) {
+          if (CG == 2) {
+            const uint32_t e = smem_addr(&tl.empty[stage]);
+            tc_commit_pair(e);
+            tc_commit_pair(mapa_shared(e, 1));
+          } else {
+            tc_commit(smem_addr(&tl.empty[stage]));
+          }
+          if (++stage == C::STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        tc_commit(smem_addr(&tl.tfull[acc]));
-        if (++acc == 2) {
-          acc = 0;
-          acc_phase ^= 1u;
+        if (CG == 2) {
+          const uint32_t f = smem_addr(&tl.tfull[acc]);
+          tc_commit_pair(f);
+          tc_commit_pair(mapa_shared(f, 1));
+        } else {
+          tc_commit(smem_addr(&tl.tfull[acc]));
         }
+        acc ^= 1u;
       }
-      (void)acc_phase;
       if (issued_any) {
-        tc_commit(smem_addr(&tl.drain));
+        if (CG == 2)
+          tc_commit_pair(smem_addr(&tl.drain));
+        else
+          tc_commit(smem_addr(&tl.drain));
         mbar_wait(smem_addr(&tl.drain), 0u, nullptr, p.flags, kFlagTimeout);
       }
     }
   } else {
     // ------------------------------------------------------------------ epilogue
     const int quad = warp & 3;  // TMEM lanes 32*quad .. 32*quad+31 belong to this warp
-    const int r_in_tile = quad * 32 + lane;
+    const int r_in_tile = static_cast<int>(rank) * BM + quad * 32 + lane;
+    const uint32_t drained = smem_addr(&tl.drained);
     uint32_t acc = 0, acc_phase = 0;
     for (int t = unit; t < total; t += n_units) {
-      const Tile tile = decode_tile(tl, G, BN, t);
+      const Tile tile = decode_tile(tl, G, BN, C::TILE_M, t);
       if (!mbar_wait(smem_addr(&tl.tfull[acc]), acc_phase, abort, p.flags, kFlagTimeout)) break;
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + (acc ? kAcc1Col : 0u);
@@ -319,7 +394,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld_wait();
           if (it == 0) {
             tc_fence_before();
-            mbar_arrive(smem_addr(&tl.drained));
+            if (CG == 2 && rank != 0)
+              mbar_arrive_cluster(mapa_shared(drained, 0));
+            else
+              mbar_arrive(drained);
           }
           if (valid) {
             float h[32];
@@ -352,7 +430,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld_wait();
           if (it == 0) {
             tc_fence_before();
-            mbar_arrive(smem_addr(&tl.drained));
+            if (CG == 2 && rank != 0)
+              mbar_arrive_cluster(mapa_shared(drained, 0));
+            else
+              mbar_arrive(drained);
           }
           const int col = tile.n0 + c;
           if (valid && col < p.n_out) {
@@ -374,10 +455,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   __syncwarp();
   tc_fence_before();
-  __syncthreads();
+  if (CG == 2)
+    cluster_sync();  // the even CTA's MMAs (which write both CTAs' TMEM) have drained
+  else
+    __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, kTmemCols);
+    if (CG == 2)
+      tmem_dealloc_pair(tmem_base, kTmemCols);
+    else
+      tmem_dealloc(tmem_base, kTmemCols);
   }
 }
 
@@ -415,41 +502,76 @@ __global__ void __launch_bounds__(128) mx_quantize_weight_kernel(const uint16_t*
 }
 
 // ---------------------------------------------------------------- host side
-template <int MODE>
-cudaError_t launch_gemm(const CUtensorMap& A, const CUtensorMap& B0, const CUtensorMap& B1, const MxParams& p,
-                        int64_t bound_units, cudaStream_t s) {
+// scale buffer of `rows` x K values as a TMA tensor: [atoms * 4 rows][128 bytes]
+bool make_sf_map(CUtensorMap* m, const void* sf, int64_t rows, int K) {
+  const uint64_t atoms = static_cast<uint64_t>((rows + 127) / 128) * (K / 128);
+  return make_tma_2d_u8_plain(m, sf, 128, atoms * 4, 128, 4);
+}
+
+template <int MODE, int CG>
+cudaError_t launch_gemm(const CUtensorMap* maps, const MxParams& p, int64_t bound_units, cudaStream_t s) {
   static std::once_flag once[64];
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   cudaError_t r = cudaSuccess;
   std::call_once(once[dev & 63], [&] {
-    r = cudaFuncSetAttribute(tc_mx_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kSmemBytes));
+    r = cudaFuncSetAttribute(tc_mx_gemm_kernel<MODE, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem_bytes<CG>()));
   });
   if (r != cudaSuccess) return r;
-  const int units = static_cast<int>(std::min<int64_t>(device_sm_count(), std::max<int64_t>(bound_units, 1)));
-  tc_mx_gemm_kernel<MODE><<<units, kThreads, kSmemBytes, s>>>(A, B0, B1, p);
+  int units = device_sm_count() / CG;
+  units = static_cast<int>(std::min<int64_t>(units, std::max<int64_t>(bound_units, 1)));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(units * CG), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem_bytes<CG>();
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  if (CG == 2) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int max_clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&max_clusters, tc_mx_gemm_kernel<MODE, CG>, &cfg) == cudaSuccess &&
+        max_clusters > 0 && max_clusters < units)
+      cfg.gridDim.x = static_cast<unsigned>(max_clusters * 2);
+  }
+  e = cudaLaunchKernelEx(&cfg, tc_mx_gemm_kernel<MODE, CG>, maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
-}  // namespace
+// CTA pairs halve the B operand each SM stages, but measured no faster here
+// (Qwen3-shaped layer: 1.32 vs 1.23-1.32 ms; tensor pipe 52 % vs 58 % busy):
+// the limit is the hand-over between tiles (the next tile's MMA waits until
+// the epilogue has read the 32 accumulator columns the two buffers share), not
+// the operand stream.  Single CTAs are the default; MOE_FFN_CTA_GROUP=1|2
+// forces one variant (tests run both).
+int choose_cta_group(const FfnMxArgs& a) {
+  static int forced = [] {
+    const char* v = std::getenv("MOE_FFN_CTA_GROUP");
+    return v ? std::atoi(v) : 0;
+  }();
+  (void)a;
+  if (forced == 1 || forced == 2) return forced;
+  return 1;
+}
 
-cudaError_t launch_ffn_mx(const FfnMxArgs& a, cudaStream_t s) {
-  if (a.max_rows <= 0 || a.G <= 0) return cudaSuccess;
-  const uint64_t G = static_cast<uint64_t>(a.G);
-  CUtensorMap mA1, mW1, mW3, mA2, mW2;
-  if (!make_tma_2d_u8(&mA1, a.a, a.d, a.max_rows, BK, BM) || !make_tma_2d_u8(&mW1, a.w1, a.d, G * a.f, BK, 128) ||
-      !make_tma_2d_u8(&mW3, a.w3, a.d, G * a.f, BK, 128) || !make_tma_2d_u8(&mA2, a.h, a.f, a.max_rows, BK, BM) ||
-      !make_tma_2d_u8(&mW2, a.w2, a.f, G * a.d, BK, 128))
-    return cudaErrorInvalidValue;
+template <int CG>
+cudaError_t launch_pair(const FfnMxArgs& a, const CUtensorMap& mA1, const CUtensorMap& mW1, const CUtensorMap& mW3,
+                        const CUtensorMap& mA2, const CUtensorMap& mW2, cudaStream_t s) {
   MxParams p{};
   p.seg_off = a.seg_off;
   p.seg_count = a.seg_count;
   p.G = a.G;
   p.max_rows = a.max_rows;
   p.flags = a.flags;
-  const int64_t m_bound = (a.max_rows + BM - 1) / BM + a.G;
+  const int64_t m_bound = (a.max_rows + Cfg<CG>::TILE_M - 1) / Cfg<CG>::TILE_M + a.G;
+  CUtensorMap maps[6];
   // GEMM1: K = d, n_out = f, h codes and scales out
   p.K = a.d;
   p.n_out = a.f;
@@ -458,7 +580,15 @@ cudaError_t launch_ffn_mx(const FfnMxArgs& a, cudaStream_t s) {
   p.b1_sf = a.w3_sf;
   p.out8 = a.h;
   p.out8_sf = a.h_sf;
-  cudaError_t e = launch_gemm<MODE_SWIGLU>(mA1, mW1, mW3, p, m_bound * (a.f / 128), s);
+  maps[0] = mA1;
+  maps[1] = mW1;
+  maps[2] = mW3;
+  if (CG == 2 && (!make_sf_map(&maps[3], a.a_sf, a.max_rows, a.d) ||
+                  !make_sf_map(&maps[4], a.w1_sf, static_cast<int64_t>(a.G) * a.f, a.d) ||
+                  !make_sf_map(&maps[5], a.w3_sf, static_cast<int64_t>(a.G) * a.f, a.d)))
+    return cudaErrorInvalidValue;
+  if (CG == 1) maps[3] = maps[4] = maps[5] = mA1;   // unused
+  cudaError_t e = launch_gemm<MODE_SWIGLU, CG>(maps, p, m_bound * (a.f / 128), s);
   if (e != cudaSuccess) return e;
   // GEMM2: K = f, n_out = d, bf16 out
   p.K = a.f;
@@ -469,7 +599,30 @@ cudaError_t launch_ffn_mx(const FfnMxArgs& a, cudaStream_t s) {
   p.out8 = nullptr;
   p.out8_sf = nullptr;
   p.out16 = static_cast<uint16_t*>(a.out);
-  return launch_gemm<MODE_PLAIN>(mA2, mW2, mW2, p, m_bound * ((a.d + 255) / 256), s);
+  maps[0] = mA2;
+  maps[1] = mW2;
+  maps[2] = mW2;
+  if (CG == 2 && (!make_sf_map(&maps[3], a.h_sf, a.max_rows, a.f) ||
+                  !make_sf_map(&maps[4], a.w2_sf, static_cast<int64_t>(a.G) * a.d, a.f)))
+    return cudaErrorInvalidValue;
+  if (CG == 2) maps[5] = maps[4];
+  if (CG == 1) maps[3] = maps[4] = maps[5] = mA2;
+  return launch_gemm<MODE_PLAIN, CG>(maps, p, m_bound * ((a.d + 255) / 256), s);
+}
+
+}  // namespace
+
+cudaError_t launch_ffn_mx(const FfnMxArgs& a, cudaStream_t s) {
+  if (a.max_rows <= 0 || a.G <= 0) return cudaSuccess;
+  const uint64_t G = static_cast<uint64_t>(a.G);
+  const int cg = choose_cta_group(a);
+  CUtensorMap mA1, mW1, mW3, mA2, mW2;   // B boxes are 128 weight rows
+  if (!make_tma_2d_u8(&mA1, a.a, a.d, a.max_rows, BK, BM) || !make_tma_2d_u8(&mW1, a.w1, a.d, G * a.f, BK, 128) ||
+      !make_tma_2d_u8(&mW3, a.w3, a.d, G * a.f, BK, 128) || !make_tma_2d_u8(&mA2, a.h, a.f, a.max_rows, BK, BM) ||
+      !make_tma_2d_u8(&mW2, a.w2, a.f, G * a.d, BK, 128))
+    return cudaErrorInvalidValue;
+  if (cg == 2) return launch_pair<2>(a, mA1, mW1, mW3, mA2, mW2, s);
+  return launch_pair<1>(a, mA1, mW1, mW3, mA2, mW2, s);
 }
 
 cudaError_t launch_mx_quantize_weight(const uint16_t* w, int64_t G, int K, int N, uint8_t* codes, uint8_t* sf,

@@ -75,6 +75,9 @@ bool make_tma_3d_f32_sw128(CUtensorMap* m, void* ptr, uint64_t inner, uint64_t m
 // The same over bytes (FP8 codes).
 bool make_tma_2d_u8(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint32_t box_inner,
                     uint32_t box_outer);
+// Bytes without swizzle (boxes copied as laid out, e.g. 512-byte scale atoms).
+bool make_tma_2d_u8_plain(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                          uint32_t box_outer);
 
 // --------------------------------------------------------------- dispatch
 constexpr int kDispatchTokens = 32;   // tokens per dispatch block (one bit each)
@@ -145,6 +148,7 @@ cudaError_t launch_ffn_f32(const FfnArgs& a, cudaStream_t s);
 // multiples of 128 and segments start at multiples of 128 rows.
 struct FfnMxArgs {
   int G;
+  int64_t mean_rows;        // expected rows per expert (tile-shape choice)
   int64_t max_rows;
   int d, f;
   const int32_t* seg_off;

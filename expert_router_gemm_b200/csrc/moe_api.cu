@@ -356,6 +356,7 @@ moe_status_t do_ffn_mx(const Dims& D, const void* xp, const void* xp_sf, const i
   const Layout L = layout(D);
   FfnMxArgs a{};
   a.G = D.N;
+  a.mean_rows = std::min<int64_t>(D.max_count, D.T * D.k / D.N);
   a.max_rows = D.max_rows;
   a.d = D.d;
   a.f = D.f;

@@ -30,16 +30,16 @@ EncodeTiledFn encode_fn() {
 namespace {
 
 bool make_2d(CUtensorMap* m, CUtensorMapDataType type, uint32_t elem_bytes, const void* ptr, uint64_t inner,
-             uint64_t outer, uint32_t box_inner, uint32_t box_outer) {
+             uint64_t outer, uint32_t box_inner, uint32_t box_outer,
+             CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
   const cuuint64_t dims[2] = {inner, outer};
   const cuuint64_t strides[1] = {inner * elem_bytes};
   const cuuint32_t box[2] = {box_inner, box_outer};
   const cuuint32_t estr[2] = {1, 1};
-  return fn(m, type, 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return fn(m, type, 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
@@ -65,6 +65,12 @@ bool make_tma_3d_f32_sw128(CUtensorMap* m, void* ptr, uint64_t inner, uint64_t m
 bool make_tma_2d_u8(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint32_t box_inner,
                     uint32_t box_outer) {
   return make_2d(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ptr, inner, outer, box_inner, box_outer);
+}
+
+bool make_tma_2d_u8_plain(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                          uint32_t box_outer) {
+  return make_2d(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ptr, inner, outer, box_inner, box_outer,
+                 CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 }  // namespace moe

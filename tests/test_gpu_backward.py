@@ -112,3 +112,37 @@ def test_layer_backward_deterministic_and_empty():
     z0 = _gpu_backward(dl0, np.zeros((0, w.d), np.uint16), aux, z)
     for key in ("dw_router", "dw1", "dw3", "dw2", "dws1", "dws3", "dws2", "drouter_bias"):
         assert not np.any(z0[key]), key
+
+
+EDGE = [
+    # capacity 0: every slot dropped, only the router path carries gradient
+    (Workload("bwd-cap0", T=128, d=128, N=4, k=2, f=128, capacity_factor=0.0), 0.05, 0.01, None),
+    # k = N: every expert chosen by every token
+    (Workload("bwd-topN", T=200, d=128, N=4, k=4, f=128, capacity_factor=1.0), 0.05, 0.01, None),
+    # one expert: the softmax is constant, the router gets only the z-loss gradient
+    (Workload("bwd-one-expert", T=96, d=128, N=1, k=1, f=128, capacity_factor=1.0), 0.05, 0.01, None),
+    # Aux-Loss-Free selection bias steering the choice (no gradient of its own)
+    (Workload("bwd-selbias", T=256, d=256, N=8, k=2, f=256, capacity_factor=1.0), 0.01, 1e-3, "normal"),
+]
+
+
+@pytest.mark.parametrize("w,aux,z,sel", EDGE, ids=[c[0].name for c in EDGE])
+def test_layer_backward_edge_cases(w, aux, z, sel):
+    inp = synth.make_inputs(w)
+    cfg = moe.config_from_workload(w)
+    dl = moe.to_device(inp, cfg)
+    sb = synth.make_selection_bias(3, w.N, sel) if sel else None
+    if sb is not None:
+        dl.selection_bias = gu.cuda_tensor(sb)
+    dy = synth.f32_to_bf16_bits(synth.normal_f32(13, 77, (w.T, w.d)))
+    got = _gpu_backward(dl, dy, aux, z)
+    ref = bwd.layer_backward(inp.x, inp.w_router, inp.bias, inp.w1, inp.w3, inp.w2, orc.as_f64(dy), k=w.k,
+                             capacity_factor=w.capacity_factor, aux_weight=aux, z_weight=z, selection_bias=sb)
+    for name, a, b in (("dx", gu.y_as_f64(got["dx"]), ref.dx), ("dw_router", got["dw_router"], ref.dw_router),
+                       ("dw1", got["dw1"], ref.dw1), ("dw3", got["dw3"], ref.dw3), ("dw2", got["dw2"], ref.dw2)):
+        assert np.all(np.isfinite(a)), name
+        if not np.any(b):
+            assert not np.any(a), name          # exactly zero where the oracle is zero
+            continue
+        rel = orc.rel_frobenius(np.asarray(a, np.float64), b)
+        assert rel <= TOL, (w.name, name, rel)

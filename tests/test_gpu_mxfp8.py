@@ -196,3 +196,55 @@ def test_mx_h_codes_match_oracle():
         same_sf += int(np.sum(hsf[rows] == hq.scale_bytes()))
     assert same >= 0.999 * total, (same, total)
     assert same_sf >= 0.999 * nblk, (same_sf, nblk)
+
+
+_MX_VARIANT_SCRIPT = r"""
+import sys
+sys.path.insert(0, {root!r})
+import numpy as np
+import torch
+from expert_router_gemm_b200 import synth, moe
+from expert_router_gemm_b200.configs import Workload
+from tests import gpu_util as gu
+from tests.layer_check import compare_layer
+for w in (Workload("mxv-ragged", T=1500, d=384, N=6, k=2, f=384, capacity_factor=1.1),
+          Workload("mxv-shared", T=700, d=256, N=8, k=2, f=256, f_shared=128, capacity_factor=1.25)):
+    inp = synth.make_inputs(w)
+    cfg = moe.config_from_workload(w, gemm="mxfp8")
+    dl = moe.to_device(inp, cfg)
+    dl.quantize_mx()
+    y, st, flags = gu.layer_fwd(dl)
+    assert flags == 0, flags
+    ws = gu.op_workspace(cfg)
+    logits = torch.empty((w.T, w.N), device="cuda")
+    idx = torch.empty((w.T, w.k), dtype=torch.int32, device="cuda")
+    wt = torch.empty((w.T, w.k), device="cuda")
+    moe.moe_route(cfg, dl.x, dl.w_router, dl.bias, None, logits, idx, wt, None, ws)
+    rm = np.asarray(gu.host(idx))   # routing only; the row map comes from the layer's own dispatch
+    _, _, max_rows = moe.moe_workspace_size(cfg)
+    row_map = torch.empty((w.T, w.k), dtype=torch.int32, device="cuda")
+    seg_off = torch.empty(w.N + 1, dtype=torch.int32, device="cuda")
+    seg_count = torch.empty(w.N, dtype=torch.int32, device="cuda")
+    codes = torch.empty((max_rows, w.d), dtype=torch.uint8, device="cuda")
+    sf = torch.empty(moe.mx_sf_bytes(max_rows, w.d), dtype=torch.uint8, device="cuda")
+    moe.moe_dispatch_mx(cfg, dl.x, idx, row_map, seg_off, seg_count, codes, sf, None, ws)
+    rel, n, flips = compare_layer(inp, w, y, rm, gu.host(row_map), gu.host(logits), tol=1e-2, mxfp8=True)
+    print("REL", w.name, rel, n, flips)
+"""
+
+
+@pytest.mark.parametrize("cta_group", ["1", "2"])
+def test_mx_gemm_cta_group_variants(cta_group):
+    """Both tile shapes of the FP8 grouped GEMM (single CTAs with 128-row tiles,
+    CTA pairs with 256-row tiles), each in its own process (the choice is made
+    once per process)."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, MOE_FFN_CTA_GROUP=cta_group)
+    r = subprocess.run([sys.executable, "-c", _MX_VARIANT_SCRIPT.format(root=root)], env=env,
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert r.stdout.count("REL") == 2, r.stdout
+    print(r.stdout)
