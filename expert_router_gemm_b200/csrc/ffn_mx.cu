@@ -27,8 +27,9 @@
 //   both halves of the tile), six stages of 33.5 KB.  Every load is a TMA tensor
 //   load counted on the even CTA's barrier; the MMA commits to both CTAs'
 //   barriers; both epilogues release the accumulator on the even CTA's barrier.
-// TMEM: accumulator 0 at columns [0, 256), accumulator 1 at [224, 480) and the
-// scales at [480, 492).  The two accumulators share 32 columns so that both fit
+// TMEM: accumulator 0 at columns [0, 256), accumulator 1 at [224, 480) and two
+// scale sets at [480, 504), used by alternate stages so that the copy of a
+// stage's scales need not wait for the previous stage's MMAs to read theirs.  The two accumulators share 32 columns so that both fit
 // beside the scales; the epilogue drains buffer 0 from its last 32 columns
 // down and buffer 1 from its first 32 columns up, and releases the next tile's
 // MMA as soon as the shared columns are read.
@@ -58,8 +59,9 @@ constexpr int SF_BYTES = 3 * SF_ATOM;      // A atom + two B atoms
 constexpr int kThreads = 192;
 constexpr int kTmemCols = 512;
 constexpr uint32_t kAcc1Col = 224;         // accumulator 1 starts here (shares [224, 256))
-constexpr uint32_t kSfaCol = 480;
+constexpr uint32_t kSfaCol = 480;          // scale set 0; set 1 is 12 columns further
 constexpr uint32_t kSfbCol = 484;          // two atoms: rows 0-127 then 128-255 of B
+constexpr uint32_t kSfSet = 12;            // columns of one scale set (two sets: [480, 504))
 constexpr int kMaxGroups = 256;
 
 enum { MODE_SWIGLU = 0, MODE_PLAIN = 1 };
@@ -297,7 +299,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     if (lane == 0 && rank == 0) {
       // ---------------------------------------------------------------- MMA issuer
-      uint32_t stage = 0, phase = 0, acc = 0, j = 0;
+      uint32_t stage = 0, phase = 0, acc = 0, j = 0, sfset = 0;
       bool ok = true, issued_any = false;
       for (int t = unit; ok && t < total; t += n_units, ++j) {
         // the previous tile's epilogue has read the columns this accumulator shares with it
@@ -314,15 +316,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t a_addr = smem_addr(sA + stage * A_BYTES);
           const uint32_t b_addr = smem_addr(sB + stage * C::B_BYTES);
           const uint32_t sf_addr = smem_addr(sSF + stage * SF_BYTES);
-          // scale atoms -> TMEM (executed in order with the MMAs issued around them)
+          // scale atoms -> this stage's TMEM scale set (executed in order with
+          // the MMAs issued around them)
+          const uint32_t sfa_col = tmem_base + kSfaCol + sfset * kSfSet;
+          const uint32_t sfb_col = tmem_base + kSfbCol + sfset * kSfSet;
+          sfset ^= 1u;
           if (CG == 2) {
-            tc_cp_32x128b_x4_pair(tmem_base + kSfaCol, smem_desc_plain(sf_addr, 16, 128));
-            tc_cp_32x128b_x4_pair(tmem_base + kSfbCol, smem_desc_plain(sf_addr + SF_ATOM, 16, 128));
-            tc_cp_32x128b_x4_pair(tmem_base + kSfbCol + 4, smem_desc_plain(sf_addr + 2 * SF_ATOM, 16, 128));
+            tc_cp_32x128b_x4_pair(sfa_col, smem_desc_plain(sf_addr, 16, 128));
+            tc_cp_32x128b_x4_pair(sfb_col, smem_desc_plain(sf_addr + SF_ATOM, 16, 128));
+            tc_cp_32x128b_x4_pair(sfb_col + 4, smem_desc_plain(sf_addr + 2 * SF_ATOM, 16, 128));
           } else {
-            tc_cp_32x128b_x4(tmem_base + kSfaCol, smem_desc_plain(sf_addr, 16, 128));
-            tc_cp_32x128b_x4(tmem_base + kSfbCol, smem_desc_plain(sf_addr + SF_ATOM, 16, 128));
-            tc_cp_32x128b_x4(tmem_base + kSfbCol + 4, smem_desc_plain(sf_addr + 2 * SF_ATOM, 16, 128));
+            tc_cp_32x128b_x4(sfa_col, smem_desc_plain(sf_addr, 16, 128));
+            tc_cp_32x128b_x4(sfb_col, smem_desc_plain(sf_addr + SF_ATOM, 16, 128));
+            tc_cp_32x128b_x4(sfb_col + 4, smem_desc_plain(sf_addr + 2 * SF_ATOM, 16, 128));
           }
 #pragma unroll
           for (int kk = 0; kk < BK / MMA_K; ++kk) {
@@ -332,11 +338,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t sel = static_cast<uint32_t>(kk) << 30;   // scale byte kk of each word
             const uint32_t idesc = idesc_mxf8(C::TILE_M, MMA_N, static_cast<uint32_t>(kk));
             if (CG == 2)
-              tc_mma_mxf8_pair(d_tmem, adesc, bdesc, idesc, (tmem_base + kSfaCol) | sel, (tmem_base + kSfbCol) | sel,
-                               (kb | kk) != 0 ? 1u : 0u);
+              tc_mma_mxf8_pair(d_tmem, adesc, bdesc, idesc, sfa_col | sel, sfb_col | sel, (kb | kk) != 0 ? 1u : 0u);
             else
-              tc_mma_mxf8(d_tmem, adesc, bdesc, idesc, (tmem_base + kSfaCol) | sel, (tmem_base + kSfbCol) | sel,
-                          (kb | kk) != 0 ? 1u : 0u);
+              tc_mma_mxf8(d_tmem, adesc, bdesc, idesc, sfa_col | sel, sfb_col | sel, (kb | kk) != 0 ? 1u : 0u);
           }
           if (CG == 2) {
             const uint32_t e = smem_addr(&tl.empty[stage]);
