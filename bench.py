@@ -255,9 +255,9 @@ def main():
     if args.warmup < 3 and not args.quick:
         ap.error("--warmup must be >= 3")
 
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    from expert_router_gemm_b200 import replicas
+    ranks = replicas.from_env()
+    rank, world, local = ranks.rank, ranks.world, ranks.local
     w = configs.get(args.config)
     if args.shape:
         from dataclasses import replace
@@ -270,13 +270,7 @@ def main():
 
     import torch
     torch.cuda.set_device(local)
-    dist = None
-    if world > 1:
-        import datetime
-
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+    replicas.init(ranks, "nccl", torch.device("cuda", local))
 
     from expert_router_gemm_b200 import moe
 
@@ -317,16 +311,10 @@ def main():
     def layer():
         layer_call(dl.x, y)
 
-    def barrier():
-        if dist is not None:
-            dist.barrier()
+    barrier = replicas.barrier
 
     def max_over_ranks(v: float) -> float:
-        if dist is None:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return replicas.max_over_ranks(v, torch.device("cuda", local))
 
     for _ in range(args.warmup):
         layer()
@@ -348,7 +336,7 @@ def main():
         torch.cuda.synchronize()
     barrier()
     ms = max_over_ranks(ev0.elapsed_time(ev1)) / args.steps
-    value = world * w.T / (ms / 1e3)
+    value = replicas.job_throughput(w.T, world, ms / 1e3)
     clocks = sampler.summary()
 
     # route: bf16 splits W_r, runs the tensor-core router GEMM and the softmax /
@@ -637,9 +625,7 @@ def main():
 
     if rank == 0:
         print(json.dumps(line), flush=True)
-    if dist is not None:
-        dist.barrier()
-        dist.destroy_process_group()
+    replicas.finish()
 
 
 if __name__ == "__main__":
