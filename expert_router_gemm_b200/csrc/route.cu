@@ -165,17 +165,57 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
   } else {
     // logits = partial sums added in order (one for caller-supplied logits), + bias
     const int64_t pstride = T * N;
-    for (int v = tid; v < BT * NP; v += kRouteThreads) {
-      const int r = v / NP, e = v % NP;
-      float g = -INFINITY;
-      if (e < N && t0 + r < T) {
-        const float* src = a.logits_in + (t0 + r) * N + e;
-        g = src[0];
-        for (int z = 1; z < a.n_partials; ++z) g += src[z * pstride];
-        if (a.bias != nullptr) g += a.bias[e];
-        if (a.logits_out != nullptr) a.logits_out[(t0 + r) * N + e] = g;
+    if ((N & 3) == 0 && (reinterpret_cast<uintptr_t>(a.logits_in) & 15) == 0 &&
+        (a.logits_out == nullptr || (reinterpret_cast<uintptr_t>(a.logits_out) & 15) == 0)) {
+      // 16-byte vectors, every load of a thread issued before the adds (the
+      // same additions, in the same order, as the scalar path below)
+      const int nq = N >> 2;
+#pragma unroll 4
+      for (int v = tid; v < BT * nq; v += kRouteThreads) {
+        const int r = v / nq, e = (v % nq) * 4;
+        float4 g = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+        if (t0 + r < T) {
+          const float4* src = reinterpret_cast<const float4*>(a.logits_in + (t0 + r) * N + e);
+          float4 part[kRouterMaxPartials];
+#pragma unroll
+          for (int z = 0; z < kRouterMaxPartials; ++z)
+            if (z < a.n_partials) part[z] = src[z * (pstride >> 2)];
+          g = part[0];
+#pragma unroll
+          for (int z = 1; z < kRouterMaxPartials; ++z)
+            if (z < a.n_partials) {
+              g.x += part[z].x;
+              g.y += part[z].y;
+              g.z += part[z].z;
+              g.w += part[z].w;
+            }
+          if (a.bias != nullptr) {
+            g.x += a.bias[e];
+            g.y += a.bias[e + 1];
+            g.z += a.bias[e + 2];
+            g.w += a.bias[e + 3];
+          }
+          if (a.logits_out != nullptr) *reinterpret_cast<float4*>(a.logits_out + (t0 + r) * N + e) = g;
+        }
+        sm.u.lg[r][e] = g.x;
+        sm.u.lg[r][e + 1] = g.y;
+        sm.u.lg[r][e + 2] = g.z;
+        sm.u.lg[r][e + 3] = g.w;
       }
-      sm.u.lg[r][e] = g;
+      for (int v = tid; v < BT * (NP - N); v += kRouteThreads) sm.u.lg[v / (NP - N)][N + v % (NP - N)] = -INFINITY;
+    } else {
+      for (int v = tid; v < BT * NP; v += kRouteThreads) {
+        const int r = v / NP, e = v % NP;
+        float g = -INFINITY;
+        if (e < N && t0 + r < T) {
+          const float* src = a.logits_in + (t0 + r) * N + e;
+          g = src[0];
+          for (int z = 1; z < a.n_partials; ++z) g += src[z * pstride];
+          if (a.bias != nullptr) g += a.bias[e];
+          if (a.logits_out != nullptr) a.logits_out[(t0 + r) * N + e] = g;
+        }
+        sm.u.lg[r][e] = g;
+      }
     }
     __syncthreads();
   }
