@@ -22,7 +22,7 @@
 //   cta_group::2 MMA (M=256) issued by the even CTA: each CTA stages its own 128
 //   rows of A and its own 128 columns of B (for SwiGLU: CTA 0 the W1 columns,
 //   CTA 1 the W3 columns), so per SM the operand traffic per flop is 2/3 of
-//   CG = 1 and six 32 KB stages fit instead of four 48 KB ones.  Both CTAs'
+//   CG = 1 and seven 32 KB stages fit instead of four 48 KB ones.  Both CTAs'
 //   loads count on the even CTA's barrier, its MMA commits to both CTAs'
 //   barriers, and both epilogues release the accumulator on the even CTA's
 //   barrier.  A pair tile covers 256 rows of one expert; an expert with an odd
@@ -61,7 +61,7 @@ struct Cfg {
   static constexpr int B_CHUNKS = 4 / CG;                   // 64-column chunks of B per CTA
   static constexpr int B_BYTES = B_CHUNKS * B_CHUNK;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;     // per CTA
-  static constexpr int STAGES = CG == 1 ? 4 : 6;
+  static constexpr int STAGES = CG == 1 ? 4 : 7;
   static constexpr int TILE_M = BM * CG;                    // accumulator rows of one (pair) tile
   static constexpr uint32_t IDESC = idesc_bf16_f32(TILE_M, MMA_N, /*b_mn_major=*/1);
 };
@@ -89,8 +89,6 @@ struct TcTail {
   uint32_t tmem_base;
   uint32_t abort;
   int32_t tile_start[kMaxGroups + 1];
-  int32_t row0[kMaxGroups];
-  int32_t count[kMaxGroups];
 };
 
 template <int CG>
@@ -102,8 +100,24 @@ struct Tile {
   int g, m0, n0;
 };
 
+// The rows [row0, row0 + count) of group g in the A / output buffers, read
+// from the segment table (L2-resident, a few loads per tile); a group outside
+// the buffers counts as empty (the prologue raises the bad-index flag for it).
+__device__ __forceinline__ int2 group_rows(const TcParams& p, int g) {
+  int r0 = 0, c = p.dense_rows;
+  if (p.seg_off != nullptr) {
+    r0 = __ldg(p.seg_off + g);
+    c = __ldg(p.seg_count + g);
+  }
+  if (r0 < 0 || c < 0 || static_cast<int64_t>(r0) + c > p.max_rows) {
+    r0 = 0;
+    c = 0;
+  }
+  return make_int2(r0, c);
+}
+
 // tile t -> (group, first row of the (pair) tile, first output column)
-__device__ __forceinline__ Tile decode_tile(const TcTail& s, int G, int bn, int tile_m, int t) {
+__device__ __forceinline__ Tile decode_tile(const TcTail& s, const TcParams& p, int G, int bn, int tile_m, int t) {
   int lo = 0, hi = G;  // largest g with tile_start[g] <= t
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
@@ -113,7 +127,7 @@ __device__ __forceinline__ Tile decode_tile(const TcTail& s, int G, int bn, int 
       hi = mid;
   }
   const int local = t - s.tile_start[lo];
-  const int mt = (s.count[lo] + tile_m - 1) / tile_m;
+  const int mt = (group_rows(p, lo).y + tile_m - 1) / tile_m;
   Tile r;
   r.g = lo;
   r.n0 = (local / mt) * bn;
@@ -208,19 +222,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int g_lo = min(G, lane * per), g_hi = min(G, g_lo + per);
     int local = 0;
     for (int g = g_lo; g < g_hi; ++g) {
-      int r0 = 0, c = p.dense_rows;
       if (p.seg_off != nullptr) {
-        r0 = p.seg_off[g];
-        c = p.seg_count[g];
+        const int r0 = p.seg_off[g], c = p.seg_count[g];
+        if (r0 < 0 || c < 0 || static_cast<int64_t>(r0) + c > p.max_rows) atomicOr(p.flags, kFlagBadIndex);
       }
-      if (r0 < 0 || c < 0 || static_cast<int64_t>(r0) + c > p.max_rows) {
-        atomicOr(p.flags, kFlagBadIndex);
-        r0 = 0;
-        c = 0;
-      }
-      tl.row0[g] = r0;
-      tl.count[g] = c;
-      local += (c + C::TILE_M - 1) / C::TILE_M * n_tiles;
+      local += (group_rows(p, g).y + C::TILE_M - 1) / C::TILE_M * n_tiles;
     }
     int incl = local;
 #pragma unroll
@@ -231,7 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int run = incl - local;
     for (int g = g_lo; g < g_hi; ++g) {
       tl.tile_start[g] = run;
-      run += (tl.count[g] + C::TILE_M - 1) / C::TILE_M * n_tiles;
+      run += (group_rows(p, g).y + C::TILE_M - 1) / C::TILE_M * n_tiles;
     }
     if (lane == 31) tl.tile_start[G] = incl;
   }
@@ -251,8 +257,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t stage = 0, phase = 0, issued = 0, last_par = 0;
       bool ok = true;
       for (int t = unit; ok && t < total; t += n_units) {
-        const Tile tile = decode_tile(tl, G, BN, C::TILE_M, t);
-        const int a_row = tl.row0[tile.g] + tile.m0 + static_cast<int>(rank) * BM;
+        const Tile tile = decode_tile(tl, p, G, BN, C::TILE_M, t);
+        const int a_row = group_rows(p, tile.g).x + tile.m0 + static_cast<int>(rank) * BM;
         const int b_row = tile.g * p.K;
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(smem_addr(&tl.empty[stage]), phase ^ 1u, abort, p.flags, kFlagTimeout)) {
@@ -368,13 +374,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r_in_tile = static_cast<int>(rank) * BM + quad * 32 + lane;
     uint32_t acc = 0, acc_phase = 0;
     for (int t = unit; t < total; t += n_units) {
-      const Tile tile = decode_tile(tl, G, BN, C::TILE_M, t);
+      const Tile tile = decode_tile(tl, p, G, BN, C::TILE_M, t);
+      const int2 gr = group_rows(p, tile.g);
       if (!mbar_wait(smem_addr(&tl.tfull[acc]), acc_phase, abort, p.flags, kFlagTimeout)) break;
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * MMA_N;
       const int row = tile.m0 + r_in_tile;
-      const bool valid = row < tl.count[tile.g];
-      uint16_t* orow = p.out + (static_cast<int64_t>(tl.row0[tile.g]) + row) * p.n_out;
+      const bool valid = row < gr.y;
+      uint16_t* orow = p.out + (static_cast<int64_t>(gr.x) + row) * p.n_out;
       if (MODE == MODE_SWIGLU) {
 #pragma unroll 1
         for (int c = 0; c < BN; c += 32) {
@@ -392,7 +399,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             store_row32(orow, tile.n0 + c, p.n_out, pk);
             if (p.save_g != nullptr) {
-              const int64_t off = (static_cast<int64_t>(tl.row0[tile.g]) + row) * p.n_out;
+              const int64_t off = (static_cast<int64_t>(gr.x) + row) * p.n_out;
 #pragma unroll
               for (int i = 0; i < 16; ++i)
                 pk[i] = pack_bf16x2(__uint_as_float(gv[2 * i]), __uint_as_float(gv[2 * i + 1]));
