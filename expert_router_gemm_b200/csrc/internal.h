@@ -48,7 +48,7 @@ struct RouteArgs {
 };
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t s);
 // The route kernel's blocks hold at least this many tokens (sizes zl_part).
-constexpr int kRouteMinBlockTokens = 32;
+constexpr int kRouteMinBlockTokens = 16;
 
 // b[i] += gamma * sign(T*k - N*counts[i]) for i < N (one block).
 cudaError_t launch_bias_update(float* b, const int32_t* counts, int64_t Tk, int N, float gamma, cudaStream_t s);

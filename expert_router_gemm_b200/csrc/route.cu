@@ -57,8 +57,9 @@ __device__ __forceinline__ float key_value(uint32_t k) {
 }
 
 // Tokens per block in logits mode (no GEMM tile to fill): small blocks keep
-// every SM busy even when T is small or N has few experts.
-constexpr int kLogitsTokens = 32;
+// every SM busy even when T is small or N has few experts, and give each SM
+// enough warps to hide the latency of the per-token reductions.
+constexpr int kLogitsTokens = 16;
 
 template <int NP, bool FROM_LOGITS>
 __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a) {
@@ -67,7 +68,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
   static_assert(FROM_LOGITS || BT == route_bt(NP), "route block size mismatch");
   static_assert(BT <= S::BT, "the logits tile holds at most S::BT tokens");
   static_assert(NP / TX == 8, "each thread owns 8 experts");
-  static_assert(BT >= kRouteMinBlockTokens, "z-loss partials are sized for 32-token blocks");
+  static_assert(BT >= kRouteMinBlockTokens, "z-loss partials are sized for 16-token blocks");
   __shared__ __align__(16) S sm;
 
   const int tid = threadIdx.x;
@@ -224,8 +225,9 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
   // The TPW tokens of a warp are processed in lock step so that their shuffle
   // reductions overlap.
   constexpr int NPL = NP >= 32 ? NP / 32 : 1;  // logits held per lane
-  constexpr int TPW = 4;
   constexpr int NW = kRouteThreads / 32;
+  constexpr int TPW = BT / NW < 4 ? BT / NW : 4;
+  static_assert(TPW >= 1 && BT % (NW * TPW) == 0, "whole token groups per warp");
   const int warp = tid >> 5, lane = tid & 31;
   float zacc[NPL];
 #pragma unroll
@@ -256,17 +258,17 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
     }
     if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(a.flags, kFlagNonfinite);
 
+    // max of the token's logits: one 32-bit reduction of the order-preserving
+    // keys of the lanes' maxima (NaN is out of contract and counts as -inf)
     float m[TPW], sum[TPW];
 #pragma unroll
     for (int q = 0; q < TPW; ++q) {
-      m[q] = -INFINITY;
+      float lm = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < NPL; ++c) m[q] = fmaxf(m[q], v[q][c]);
+      for (int c = 0; c < NPL; ++c) lm = fmaxf(lm, v[q][c]);
+      if (isnan(lm)) lm = -INFINITY;
+      m[q] = key_value(__reduce_max_sync(0xffffffffu, order_key(lm)));
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-      for (int q = 0; q < TPW; ++q) m[q] = fmaxf(m[q], __shfl_xor_sync(0xffffffffu, m[q], o));
 #pragma unroll
     for (int q = 0; q < TPW; ++q) {
       sum[q] = 0.f;
@@ -281,92 +283,92 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
 #pragma unroll
       for (int q = 0; q < TPW; ++q) sum[q] += __shfl_xor_sync(0xffffffffu, sum[q], o);
 #pragma unroll
-    for (int q = 0; q < TPW; ++q)
+    for (int q = 0; q < TPW; ++q) {
       if (valid[q]) {
         const float lse = m[q] + logf(sum[q]);  // log-partition of the unbiased logits
         zl += static_cast<double>(lse) * lse;
+        const float inv = 1.f / sum[q];
+#pragma unroll
+        for (int c = 0; c < NPL; ++c) zacc[c] += s[q][c] * inv;
       }
 #pragma unroll
-    for (int q = 0; q < TPW; ++q)
-#pragma unroll
-      for (int c = 0; c < NPL; ++c) {
-        if (valid[q]) {
-          s[q][c] = s[q][c] / sum[q];
-          zacc[c] += s[q][c];
-        }
+      for (int c = 0; c < NPL; ++c)
         if (isnan(v[q][c])) v[q][c] = -INFINITY;  // out of contract; keeps the selection defined
-      }
+    }
 
     // top-k on the logits (plus the selection bias, in fp32, when there is
-    // one).  Each (score, expert) becomes one 64-bit key whose unsigned order
-    // is "larger score first, then lower expert index" (-0.0 is taken as +0.0
-    // so equal scores tie).  A lane sorts its few keys; each round is one
-    // warp-wide max over the lanes' leading keys, and the winning lane drops
-    // its leading key.  The winner's weight is recomputed from its unbiased
-    // logit with the softmax's own expression.
-    uint64_t key[TPW][NPL];
+    // one): larger score first, ties to the lower expert index.  A lane holds
+    // the order-preserving 32-bit keys of its experts' scores (-0.0 taken as
+    // +0.0, so equal scores tie; 0 for padding experts, below every score),
+    // sorted, with the slot numbers c (expert lane + 32 c) packed 3 bits each.
+    // A round's winner is the warp max of the leading keys, then among the
+    // lanes holding it the lowest expert index: two 32-bit reductions.  The
+    // winning lane drops its head; lane j keeps the winner of round j.
+    uint32_t hk[TPW][NPL], cpk[TPW];
 #pragma unroll
     for (int q = 0; q < TPW; ++q) {
+      int cs[NPL];
 #pragma unroll
       for (int c = 0; c < NPL; ++c) {
         const int e = lane + 32 * c;
-        const float sel = biased ? v[q][c] + sb[c] : v[q][c];
-        key[q][c] = e < N ? (static_cast<uint64_t>(order_key(sel)) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(e))
-                          : 0ull;
+        hk[q][c] = e < N ? order_key(biased ? v[q][c] + sb[c] : v[q][c]) : 0u;
+        cs[c] = c;
       }
 #pragma unroll
       for (int i = 1; i < NPL; ++i)
 #pragma unroll
         for (int j2 = i; j2 > 0; --j2)
-          if (key[q][j2] > key[q][j2 - 1]) {
-            const uint64_t tmp = key[q][j2];
-            key[q][j2] = key[q][j2 - 1];
-            key[q][j2 - 1] = tmp;
+          if (hk[q][j2] > hk[q][j2 - 1]) {  // strict: equal keys keep the lower c first
+            const uint32_t th = hk[q][j2];
+            hk[q][j2] = hk[q][j2 - 1];
+            hk[q][j2 - 1] = th;
+            const int tc = cs[j2];
+            cs[j2] = cs[j2 - 1];
+            cs[j2 - 1] = tc;
           }
-    }
-    int my_idx[TPW];
-    float my_s[TPW], ssum[TPW];
+      cpk[q] = 0u;
 #pragma unroll
-    for (int q = 0; q < TPW; ++q) {
-      my_idx[q] = 0;
-      my_s[q] = 0.f;
-      ssum[q] = 0.f;
+      for (int c = 0; c < NPL; ++c) cpk[q] |= static_cast<uint32_t>(cs[c]) << (3 * c);
     }
+    uint32_t won_h[TPW], won_e[TPW];
+#pragma unroll
+    for (int q = 0; q < TPW; ++q) won_h[q] = won_e[q] = 0u;
     for (int j = 0; j < k; ++j) {
-      uint64_t best[TPW];
-#pragma unroll
-      for (int q = 0; q < TPW; ++q) best[q] = key[q][0];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-        for (int q = 0; q < TPW; ++q) {
-          const uint64_t other = __shfl_xor_sync(0xffffffffu, best[q], o);
-          best[q] = other > best[q] ? other : best[q];
-        }
 #pragma unroll
       for (int q = 0; q < TPW; ++q) {
-        if (key[q][0] == best[q]) {  // keys are unique: exactly one lane drops its head
+        const uint32_t h = hk[q][0];
+        const uint32_t hmax = __reduce_max_sync(0xffffffffu, h);
+        const uint32_t inv_e = 0xFFFFFFFFu - static_cast<uint32_t>(lane + 32 * (cpk[q] & 7u));
+        const uint32_t emax = __reduce_max_sync(0xffffffffu, h == hmax ? inv_e : 0u);
+        if (h == hmax && inv_e == emax) {  // keys are unique: exactly one lane drops its head
 #pragma unroll
-          for (int c = 0; c + 1 < NPL; ++c) key[q][c] = key[q][c + 1];
-          key[q][NPL - 1] = 0ull;
+          for (int c = 0; c + 1 < NPL; ++c) hk[q][c] = hk[q][c + 1];
+          hk[q][NPL - 1] = 0u;
+          cpk[q] >>= 3;
         }
-        const int e = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(best[q]));
-        const float ve = biased ? sm.u.lg[tl0 + q][e] : key_value(static_cast<uint32_t>(best[q] >> 32));
-        const float sv = expf(ve - m[q]) / sum[q];
-        ssum[q] += sv;
         if (lane == j) {
-          my_idx[q] = e;
-          my_s[q] = sv;
+          won_h[q] = hmax;
+          won_e[q] = 0xFFFFFFFFu - emax;
         }
       }
     }
+    // Lane j < k: the weight of slot j, s_e / sum of the k chosen s (summed in
+    // slot order), from the unbiased logit with the softmax's own expression.
 #pragma unroll
     for (int q = 0; q < TPW; ++q) {
+      const int e = static_cast<int>(won_e[q]);
+      float sv = 0.f;
+      if (lane < k) {
+        const float ve = biased ? sm.u.lg[tl0 + q][e] : key_value(won_h[q]);
+        sv = expf(ve - m[q]) / sum[q];
+      }
+      float ssum = __shfl_sync(0xffffffffu, sv, 0);
+      for (int j = 1; j < k; ++j) ssum += __shfl_sync(0xffffffffu, sv, j);
       if (valid[q] && lane < k) {
         const int64_t t = t0 + tl0 + q;
-        a.topk_idx[t * k + lane] = my_idx[q];
-        a.topk_w[t * k + lane] = my_s[q] / ssum[q];
-        if (a.want_stats) atomicAdd(&sm.hist[my_idx[q]], 1);
+        a.topk_idx[t * k + lane] = e;
+        a.topk_w[t * k + lane] = sv / ssum;
+        if (a.want_stats) atomicAdd(&sm.hist[e], 1);
       }
     }
   }
@@ -458,7 +460,13 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
   } else if (warp == 1 && a.stats.z_loss != nullptr) {
     // z-loss: the blocks' partials in block order (a fixed reduction tree)
     double t = 0.0;
-    for (unsigned b = lane; b < gridDim.x; b += 32) t += __ldcg(a.zl_part + b);
+    for (unsigned b0 = lane; b0 < gridDim.x; b0 += 32 * 8) {  // 8 loads in flight, then the adds in block order
+      double v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = b0 + 32 * u < gridDim.x ? __ldcg(a.zl_part + b0 + 32 * u) : 0.0;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) t += v[u];
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
     if (lane == 0) a.stats.z_loss[0] = static_cast<float>(t / static_cast<double>(T));

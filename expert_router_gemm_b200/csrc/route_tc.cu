@@ -73,23 +73,35 @@ struct RtParams {
   uint32_t* flags;
 };
 
-// W_r fp32 [d, N] -> three bf16 slabs [3][d][NP] (columns N..NP-1 zero)
-__global__ void split_router_kernel(const float* __restrict__ w, uint16_t* __restrict__ out, int d, int N,
-                                    int NP) {
-  const int64_t total = static_cast<int64_t>(d) * NP;
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t r = i / NP;
-    const int c = static_cast<int>(i % NP);
-    const float v = c < N ? w[r * N + c] : 0.f;
-    const __nv_bfloat16 hi = __float2bfloat16_rn(v);
-    const float r1 = v - __bfloat162float(hi);
-    const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
-    const float r2 = r1 - __bfloat162float(mid);
-    const __nv_bfloat16 lo = __float2bfloat16_rn(r2);
-    out[i] = *reinterpret_cast<const uint16_t*>(&hi);
-    out[total + i] = *reinterpret_cast<const uint16_t*>(&mid);
-    out[2 * total + i] = *reinterpret_cast<const uint16_t*>(&lo);
+// W_r fp32 [d, N] -> three bf16 slabs [3][d][NP] (columns N..NP-1 zero).
+// Block (32, 8): threadIdx.y picks one of 8 rows, a thread splits 4 adjacent
+// columns and stores each slab's 4 values as one 8-byte word.
+__device__ __forceinline__ void split3(float v, uint16_t& hi, uint16_t& mid, uint16_t& lo) {
+  const __nv_bfloat16 h = __float2bfloat16_rn(v);
+  const float r1 = v - __bfloat162float(h);
+  const __nv_bfloat16 m = __float2bfloat16_rn(r1);
+  const float r2 = r1 - __bfloat162float(m);
+  const __nv_bfloat16 l = __float2bfloat16_rn(r2);
+  hi = *reinterpret_cast<const uint16_t*>(&h);
+  mid = *reinterpret_cast<const uint16_t*>(&m);
+  lo = *reinterpret_cast<const uint16_t*>(&l);
+}
+
+__global__ void __launch_bounds__(256) split_router_kernel(const float* __restrict__ w, uint16_t* __restrict__ out,
+                                                           int d, int N, int NP) {
+  const int r = blockIdx.x * blockDim.y + threadIdx.y;
+  if (r >= d) return;
+  const int64_t plane = static_cast<int64_t>(d) * NP;
+  const float* wr = w + static_cast<int64_t>(r) * N;
+  for (int c = threadIdx.x * 4; c < NP; c += blockDim.x * 4) {
+    uint16_t p[3][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) split3(c + i < N ? wr[c + i] : 0.f, p[0][i], p[1][i], p[2][i]);
+    const int64_t o = static_cast<int64_t>(r) * NP + c;
+#pragma unroll
+    for (int s = 0; s < 3; ++s)
+      *reinterpret_cast<uint2*>(out + s * plane + o) =
+          make_uint2(p[s][0] | (static_cast<uint32_t>(p[s][1]) << 16), p[s][2] | (static_cast<uint32_t>(p[s][3]) << 16));
   }
 }
 
@@ -232,8 +244,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
+    // Epilogue: a warp owns 32 accumulator rows (tokens).  Each 32-column
+    // chunk goes through shared memory (the stage buffers, idle once every MMA
+    // has completed) so that the global stores are whole 128-byte row pieces.
     const int quad = warp & 3;
-    const int64_t t = static_cast<int64_t>(m0) + quad * 32 + lane;
+    float* stg = reinterpret_cast<float*>(base) + quad * 32 * 33;  // 32 x 33 words: conflict-free both ways
     if (KB > 0 && mbar_wait(smem_addr(&tl.tfull), 0u, abort, p.flags, kFlagTimeout)) {
       tc_fence_after();
 #pragma unroll 1
@@ -241,14 +256,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t v[32];
         tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + c, v);
         tmem_ld_wait();
-        if (t < p.T) {
-          float* dst = logits + t * p.N + n0 + c;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int e = n0 + c + i;
-            if (e < p.N) dst[i] = __uint_as_float(v[i]);
-          }
+        for (int i = 0; i < 32; ++i) stg[lane * 33 + i] = __uint_as_float(v[i]);
+        __syncwarp();
+        const int e = n0 + c + lane;
+#pragma unroll 4
+        for (int r = 0; r < 32; ++r) {
+          const int64_t t = static_cast<int64_t>(m0) + quad * 32 + r;
+          if (t < p.T && e < p.N) logits[t * p.N + e] = stg[r * 33 + lane];
         }
+        __syncwarp();
       }
     }
   }
@@ -311,10 +328,7 @@ size_t router_split_bytes(int d, int N) { return 3ull * d * split_width(N) * siz
 cudaError_t launch_router_tc(const RouteArgs& a, void* split, float* partials, int* n_partials, cudaStream_t s) {
   const bool pairs = a.N > 64;
   const int NP = split_width(a.N);
-  const int64_t total = static_cast<int64_t>(a.d) * NP;
-  const int threads = 256;
-  const int blocks = static_cast<int>(std::min<int64_t>((total + threads - 1) / threads, 4 * device_sm_count()));
-  split_router_kernel<<<blocks, threads, 0, s>>>(a.w_router, static_cast<uint16_t*>(split), a.d, a.N, NP);
+  split_router_kernel<<<(a.d + 7) / 8, dim3(32, 8), 0, s>>>(a.w_router, static_cast<uint16_t*>(split), a.d, a.N, NP);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   CUtensorMap mx, mw;
