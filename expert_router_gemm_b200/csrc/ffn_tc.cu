@@ -77,6 +77,7 @@ struct TcParams {
   uint16_t* out;             // [max_rows, n_out] bf16
   uint16_t* save_g;          // SwiGLU, optional: gate and up pre-activations [max_rows, n_out]
   uint16_t* save_u;          //   (bf16), kept for the backward pass
+  int v8;                    // output rows start on 32-byte boundaries: 32-byte stores
   uint32_t* flags;
 };
 
@@ -140,8 +141,17 @@ __device__ __forceinline__ Tile decode_tile(const TcTail& s, const TcParams& p, 
 // negative u, e^-u overflows to inf and the quotient is -0.
 __device__ __forceinline__ float silu_f32(float u) { return __fdividef(u, 1.0f + __expf(-u)); }
 
-__device__ __forceinline__ void store_row32(uint16_t* orow, int col, int n_out, const uint32_t (&pk)[16]) {
-  if (col + 32 <= n_out) {
+__device__ __forceinline__ void store_row32(uint16_t* orow, int col, int n_out, const uint32_t (&pk)[16],
+                                            bool v8) {
+  if (v8 && col + 32 <= n_out) {  // two 32-byte stores: each sector is written whole, once
+    uint32_t* dst = reinterpret_cast<uint32_t*>(orow + col);
+    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "r"(pk[0]), "r"(pk[1]),
+                 "r"(pk[2]), "r"(pk[3]), "r"(pk[4]), "r"(pk[5]), "r"(pk[6]), "r"(pk[7])
+                 : "memory");
+    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst + 8), "r"(pk[8]), "r"(pk[9]),
+                 "r"(pk[10]), "r"(pk[11]), "r"(pk[12]), "r"(pk[13]), "r"(pk[14]), "r"(pk[15])
+                 : "memory");
+  } else if (col + 32 <= n_out) {
     uint4* dst = reinterpret_cast<uint4*>(orow + col);
 #pragma unroll
     for (int q = 0; q < 4; ++q) dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
@@ -397,17 +407,17 @@ __global__ void __launch_bounds__(kThreads, 1)
               const float h1 = silu_f32(__uint_as_float(gv[2 * i + 1])) * __uint_as_float(uv[2 * i + 1]);
               pk[i] = pack_bf16x2(h0, h1);
             }
-            store_row32(orow, tile.n0 + c, p.n_out, pk);
+            store_row32(orow, tile.n0 + c, p.n_out, pk, p.v8);
             if (p.save_g != nullptr) {
               const int64_t off = (static_cast<int64_t>(gr.x) + row) * p.n_out;
 #pragma unroll
               for (int i = 0; i < 16; ++i)
                 pk[i] = pack_bf16x2(__uint_as_float(gv[2 * i]), __uint_as_float(gv[2 * i + 1]));
-              store_row32(p.save_g + off, tile.n0 + c, p.n_out, pk);
+              store_row32(p.save_g + off, tile.n0 + c, p.n_out, pk, p.v8);
 #pragma unroll
               for (int i = 0; i < 16; ++i)
                 pk[i] = pack_bf16x2(__uint_as_float(uv[2 * i]), __uint_as_float(uv[2 * i + 1]));
-              store_row32(p.save_u + off, tile.n0 + c, p.n_out, pk);
+              store_row32(p.save_u + off, tile.n0 + c, p.n_out, pk, p.v8);
             }
           }
         }
@@ -421,7 +431,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t pk[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-            store_row32(orow, tile.n0 + c, p.n_out, pk);
+            store_row32(orow, tile.n0 + c, p.n_out, pk, p.v8);
           }
         }
       }
@@ -502,6 +512,11 @@ cudaError_t launch_gemm(const CUtensorMap& A, const CUtensorMap& B0, const CUten
 // CTA pairs pay off when experts have many rows; with few rows per expert the
 // 256-row pair tiles waste more of the MMA work on rows past the segment end.
 // MOE_FFN_CTA_GROUP=1|2 forces one variant (tests run both).
+// every row of a bf16 [rows, n] buffer starts on a 32-byte boundary (null: no buffer)
+bool rows_32b_aligned(const uint16_t* p, int n) {
+  return (reinterpret_cast<uintptr_t>(p) & 31u) == 0 && n % 16 == 0;
+}
+
 int choose_cta_group(const FfnArgs& a) {
   static int forced = [] {
     const char* v = std::getenv("MOE_FFN_CTA_GROUP");
@@ -523,12 +538,15 @@ cudaError_t launch_pair(const FfnArgs& a, const CUtensorMap& mA1, const CUtensor
   p.out = static_cast<uint16_t*>(a.h);
   p.save_g = static_cast<uint16_t*>(a.save_g);
   p.save_u = static_cast<uint16_t*>(a.save_u);
+  p.v8 = rows_32b_aligned(p.out, p.n_out) && rows_32b_aligned(p.save_g, p.n_out) &&
+         rows_32b_aligned(p.save_u, p.n_out);
   cudaError_t e = launch_gemm<MODE_SWIGLU, CG>(mA1, mW1, mW3, p, m_bound * ((a.f + 127) / 128), s);
   if (e != cudaSuccess) return e;
   p.save_g = p.save_u = nullptr;
   p.K = a.f;
   p.n_out = a.d;
   p.out = static_cast<uint16_t*>(a.out);
+  p.v8 = rows_32b_aligned(p.out, p.n_out);
   return launch_gemm<MODE_PLAIN, CG>(mA2, mW2, mW2, p, m_bound * ((a.d + 255) / 256), s);
 }
 
