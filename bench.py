@@ -223,6 +223,66 @@ def run_reference(args, w, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def calibrate(cfg, w, dl, weights, stream, local, seconds=3.0):
+    """Per-clock efficiency of the grouped GEMM pair (moe_expert_ffn) looped
+    alone, next to a dense bf16 8192^3 GEMM of the vendor library (torch.matmul,
+    a reference measurement only) on the same GPU.  Each runs ~`seconds` so that
+    the power limiter settles; efficiency = TFLOP/s / (dense bf16 flops per SM
+    clock x 148 SMs x median SM clock)."""
+    import torch
+    from expert_router_gemm_b200 import moe
+    T, N, k, d, f = w.T, w.N, w.k, w.d, w.f
+    _, ob, max_rows = moe.moe_workspace_size(cfg)
+    ws = torch.empty(ob, dtype=torch.uint8, device="cuda")
+    i32 = dict(dtype=torch.int32, device="cuda")
+    idx, row_map = torch.empty((T, k), **i32), torch.empty((T, k), **i32)
+    wt = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    seg_off, seg_count = torch.empty(N + 1, **i32), torch.empty(N, **i32)
+    xp = torch.empty((max_rows, d), dtype=dl.x.dtype, device="cuda")
+    h = torch.empty((max_rows, f), dtype=dl.x.dtype, device="cuda")
+    o = torch.empty((max_rows, d), dtype=dl.x.dtype, device="cuda")
+    st = moe.make_stats()
+    moe.moe_route(cfg, dl.x, dl.w_router, dl.bias, None, None, idx, wt, st, ws, stream)
+    moe.moe_dispatch(cfg, dl.x, idx, row_map, seg_off, seg_count, xp, st, ws, stream)
+    torch.cuda.synchronize()
+    kept = int(seg_count.sum().item())
+    per_mhz = 8192 * 148 * 1e6 / 1e12   # dense bf16 TFLOP/s per MHz of SM clock (148 SMs)
+
+    def loop(fn, flops):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        t0, n = time.time(), 0
+        while time.time() - t0 < 0.3:
+            fn()
+            n += 1
+        torch.cuda.synchronize()
+        reps = max(5, int(seconds * n / (time.time() - t0)))
+        smp = ClockSampler(local, period_s=0.01)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with smp:
+            e0.record(stream)
+            for _ in range(reps):
+                fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / reps
+        c = smp.summary()
+        tf = flops / ms / 1e9
+        return {"ms": round(ms, 4), "TFLOP/s": round(tf, 1), "sm_mhz": c.get("sm_mhz"),
+                "reasons": c.get("reasons"), "power_w_max": c.get("power_w_max"),
+                "per_clock": round(tf / (per_mhz * c["sm_mhz"]), 4) if c.get("sm_mhz") else None}
+
+    out = {"grouped_gemm_pair": loop(
+        lambda: moe.moe_expert_ffn(cfg, xp, seg_off, seg_count, weights, h, o, ws, stream), 6.0 * d * f * kept)}
+    a = torch.randn(8192, 8192, dtype=torch.bfloat16, device="cuda")
+    b = torch.randn(8192, 8192, dtype=torch.bfloat16, device="cuda")
+    c = torch.empty(8192, 8192, dtype=torch.bfloat16, device="cuda")
+    out["reference_dense_bf16_gemm_8192^3"] = dict(
+        loop(lambda: torch.matmul(a, b, out=c), 2.0 * 8192 ** 3), library="cuBLAS via torch.matmul (reference only)")
+    return out
+
+
 def workload_config(w):
     return {"workload": w.name, "T": w.T, "d": w.d, "N": w.N, "k": w.k, "f": w.f,
             "f_shared": w.f_shared, "capacity_factor": w.capacity_factor,
@@ -249,6 +309,9 @@ def main():
     ap.add_argument("--gemm", default="act", choices=["act", "mxfp8"],
                     help="number format of the routed experts' GEMMs: the activation dtype, or "
                          "block-scaled FP8 (weights quantized once before the timed region)")
+    ap.add_argument("--calibrate", action="store_true",
+                    help="also loop the grouped GEMM pair alone and a dense bf16 library GEMM "
+                         "(cuBLAS, reference only) for ~3 s each and report their per-clock efficiency")
     ap.add_argument("--shape", default="",
                     help="override workload fields for small profiling cases, e.g. T=2048,N=32")
     args = ap.parse_args()
@@ -613,6 +676,9 @@ def main():
             "gemm_flops_per_step": gemm_fl, "gemm_TFLOP/s": round(gemm_fl / (bms / 1e3) / 1e12, 1),
             "frac_of_sustained_bf16_peak": round(gemm_fl / (bms / 1e3) / 1e12 / peaks["bf16_tflops_sustained"], 4),
             "peak_source": peak_src, "device_flags": bflags, "clocks": bsampler.summary()}
+
+    if args.calibrate and world == 1 and not mx and w.dtype == "bf16":
+        line["calibration"] = calibrate(cfg, w, dl, weights, stream, local)
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.quick:
         steps, t_route = oracle_expert_steps(w, inp, budget_s=args.cpu_budget, mx=mx)
