@@ -7,9 +7,12 @@
 // point 4 (router kept in fp32 against softmax 0/0), and for the statistics
 // "负载均衡策略：MoE训练稳定性保障", section "辅助损失函数" (y_i, z_i).
 //
-// One kernel per token block: the GEMM tile is accumulated in registers
-// (CUDA-core FFMA over smem tiles), written to a shared logits tile, then one
-// warp per token does the softmax and the top-k by warp-shuffle reductions.
+// One kernel per token block.  The logits tile comes either from a CUDA-core
+// FFMA GEMM over shared-memory tiles (fp32 layers) or from the tensor-core
+// router's split-K partial sums (bf16 layers: added in split order, then the
+// bias); a warp then takes its tokens two to four at a time through the
+// softmax (shuffle-tree sum, 32-bit reduction for the max) and the top-k (two
+// 32-bit warp reductions per slot).
 #include <math.h>
 
 #include "device_utils.cuh"

@@ -17,8 +17,8 @@
 //
 // 192 threads per CTA: warp 0 lane 0 issues the TMA loads (x slab 128 x 64 and
 // the three weight slabs of this CTA's experts per stage), warp 1 allocates TMEM
-// and lane 0 issues the MMAs, warps 2-5 move the accumulator to registers and
-// store the fp32 partial sums.  The operand stream is latency-bound (each
+// and lane 0 issues the MMAs, warps 2-5 move the accumulator through registers
+// and shared memory to the fp32 partial sums (whole 128-byte row pieces).  The operand stream is latency-bound (each
 // CTA streams its own tokens), so the work per staged byte decides the speed:
 //   CG = 1: one CTA per 128 tokens x 64 experts (M=128, N=64 MMA), N <= 64;
 //   CG = 2: a CTA pair per 256 tokens x 128 experts (cta_group::2, M=256,
