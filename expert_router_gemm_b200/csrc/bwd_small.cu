@@ -224,6 +224,115 @@ __global__ void router_wgrad_reduce_kernel(int n_chunks, int d, int N, const flo
   }
 }
 
+// The same two products for wide routers (N > 64) with 128 x 128 output tiles:
+// 256 threads, each an 8 x 8 register tile (rows {4ty + a, 64 + 4ty + a} and
+// columns {4tx + b, 64 + 4tx + b}, a, b < 4), so that every 64 FMAs read four
+// 16-byte words of shared memory.  Reduction slabs of 16.
+constexpr int WT = 128;
+constexpr int WK = 16;
+constexpr int WP = WT + 4;   // padded smem row (floats): 16-byte aligned rows
+
+__device__ __forceinline__ void tile_fma_8x8(const float (*as)[WP], const float (*bs)[WP], int tx, int ty,
+                                             float (&acc)[8][8]) {
+#pragma unroll 4
+  for (int r = 0; r < WK; ++r) {
+    const float4 a0 = *reinterpret_cast<const float4*>(&as[r][ty * 4]);
+    const float4 a1 = *reinterpret_cast<const float4*>(&as[r][64 + ty * 4]);
+    const float4 b0 = *reinterpret_cast<const float4*>(&bs[r][tx * 4]);
+    const float4 b1 = *reinterpret_cast<const float4*>(&bs[r][64 + tx * 4]);
+    const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+    const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+    for (int a = 0; a < 8; ++a)
+#pragma unroll
+      for (int b = 0; b < 8; ++b) acc[a][b] = fmaf(av[a], bv[b], acc[a][b]);
+  }
+}
+
+__device__ __forceinline__ int tile_row(int ty, int a) { return a < 4 ? ty * 4 + a : 64 + ty * 4 + (a - 4); }
+
+// partial[z][c][i] = sum_{t in chunk z} x[t][c] dg[t][i] for c <= d (row d: x = 1,
+// the bias gradient)
+__global__ void __launch_bounds__(256) router_wgrad_wide_kernel(int64_t T, int d, int N, const uint16_t* __restrict__ x,
+                                                               const float* __restrict__ dg,
+                                                               float* __restrict__ part) {
+  __shared__ __align__(16) float xs[WK][WP];
+  __shared__ __align__(16) float gs[WK][WP];
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  const int c0 = blockIdx.x * WT, i0 = blockIdx.y * WT;
+  const int64_t t_begin = static_cast<int64_t>(blockIdx.z) * kChunkRows;
+  const int64_t t_end = t_begin + kChunkRows < T ? t_begin + kChunkRows : T;
+  float acc[8][8] = {};
+  for (int64_t tb = t_begin; tb < t_end; tb += WK) {
+#pragma unroll
+    for (int u = 0; u < WK * WT / 256; ++u) {   // one row of 128 per 128 threads: coalesced
+      const int v = threadIdx.x + 256 * u;
+      const int r = v / WT, c = v % WT;
+      const int64_t t = tb + r;
+      float xv = 0.f, gv = 0.f;
+      if (t < t_end) {
+        if (c0 + c < d)
+          xv = __uint_as_float(static_cast<uint32_t>(x[t * d + c0 + c]) << 16);
+        else if (c0 + c == d)
+          xv = 1.f;
+        if (i0 + c < N) gv = dg[t * N + i0 + c];
+      }
+      xs[r][c] = xv;
+      gs[r][c] = gv;
+    }
+    __syncthreads();
+    tile_fma_8x8(xs, gs, tx, ty, acc);
+    __syncthreads();
+  }
+  float* pz = part + static_cast<int64_t>(blockIdx.z) * (d + 1) * N;
+#pragma unroll
+  for (int a = 0; a < 8; ++a) {
+    const int c = c0 + tile_row(ty, a);
+    if (c > d) continue;
+#pragma unroll
+    for (int b = 0; b < 8; ++b) {
+      const int i = i0 + tile_row(tx, b);
+      if (i < N) pz[static_cast<int64_t>(c) * N + i] = acc[a][b];
+    }
+  }
+}
+
+// dxr[t][c] = sum_i dg[t][i] W_r[c][i]
+__global__ void __launch_bounds__(256) router_dgrad_wide_kernel(int64_t T, int d, int N, const float* __restrict__ dg,
+                                                               const float* __restrict__ wr,
+                                                               float* __restrict__ dxr) {
+  __shared__ __align__(16) float gs[WK][WP];   // [i][t]
+  __shared__ __align__(16) float ws[WK][WP];   // [i][c]
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * WT;
+  const int c0 = blockIdx.y * WT;
+  float acc[8][8] = {};
+  for (int ib = 0; ib < N; ib += WK) {
+#pragma unroll
+    for (int u = 0; u < WK * WT / 256; ++u) {   // i fastest: 64-byte pieces of the rows of dg and W_r
+      const int v = threadIdx.x + 256 * u;
+      const int r = v / WK, i = v % WK;
+      const int64_t t = t0 + r;
+      const int c = c0 + r;
+      gs[i][r] = (t < T && ib + i < N) ? dg[t * N + ib + i] : 0.f;
+      ws[i][r] = (c < d && ib + i < N) ? wr[static_cast<int64_t>(c) * N + ib + i] : 0.f;
+    }
+    __syncthreads();
+    tile_fma_8x8(gs, ws, tx, ty, acc);
+    __syncthreads();
+  }
+#pragma unroll
+  for (int a = 0; a < 8; ++a) {
+    const int64_t t = t0 + tile_row(ty, a);
+    if (t >= T) continue;
+#pragma unroll
+    for (int b = 0; b < 8; ++b) {
+      const int c = c0 + tile_row(tx, b);
+      if (c < d) dxr[t * d + c] = acc[a][b];
+    }
+  }
+}
+
 // dxr[t][c] = sum_i dg[t][i] W_r[c][i]
 __global__ void __launch_bounds__(256) router_dgrad_kernel(int64_t T, int d, int N, const float* __restrict__ dg,
                                                           const float* __restrict__ wr, float* __restrict__ dxr) {
@@ -354,6 +463,13 @@ cudaError_t launch_router_wgrad(int64_t T, int d, int N, const uint16_t* x, cons
                                 float* dbias, float* scratch, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
   const int chunks = static_cast<int>((T + kChunkRows - 1) / kChunkRows);
+  if (N > 64) {
+    router_wgrad_wide_kernel<<<dim3(static_cast<unsigned>(d / WT + 1), static_cast<unsigned>((N + WT - 1) / WT),
+                                    static_cast<unsigned>(chunks)),
+                               256, 0, s>>>(T, d, N, x, dg, scratch);
+    router_wgrad_reduce_kernel<<<256, 256, 0, s>>>(chunks, d, N, scratch, dw_router, dbias);
+    return cudaGetLastError();
+  }
   router_wgrad_kernel<<<dim3(static_cast<unsigned>(d / RT + 1), static_cast<unsigned>((N + RT - 1) / RT),
                              static_cast<unsigned>(chunks)),
                         256, 0, s>>>(T, d, N, x, dg, scratch);
@@ -364,6 +480,11 @@ cudaError_t launch_router_wgrad(int64_t T, int d, int N, const uint16_t* x, cons
 cudaError_t launch_router_dgrad(int64_t T, int d, int N, const float* dg, const float* w_router, float* dxr,
                                 cudaStream_t s) {
   if (T == 0) return cudaSuccess;
+  if (N > 64) {
+    router_dgrad_wide_kernel<<<dim3(static_cast<unsigned>((T + WT - 1) / WT), static_cast<unsigned>((d + WT - 1) / WT)),
+                               256, 0, s>>>(T, d, N, dg, w_router, dxr);
+    return cudaGetLastError();
+  }
   router_dgrad_kernel<<<dim3(static_cast<unsigned>((T + RT - 1) / RT), static_cast<unsigned>((d + RT - 1) / RT)), 256,
                         0, s>>>(T, d, N, dg, w_router, dxr);
   return cudaGetLastError();

@@ -33,6 +33,10 @@ CASES = [
               bias_pattern=_BIAS16, bias_beta_gamma=(0.25, -0.125)), 0.3, 0.2),
     (Workload("bwd-ragged", T=300, d=320, N=8, k=2, f=192, capacity_factor=1.1), 0.05, 0.0),
     (Workload("bwd-finegrained", T=768, d=256, N=128, k=8, f=128, capacity_factor=1.0, seed=1), 0.01, 1e-3),
+    # wide routers (N > 64: the 128 x 128-tile router gradient kernels) with ragged T, d not a
+    # multiple of 128 and N not a multiple of 4; and two 128-expert column tiles
+    (Workload("bwd-wide-ragged", T=300, d=320, N=100, k=4, f=128, capacity_factor=1.1), 0.05, 1e-3),
+    (Workload("bwd-n256", T=256, d=256, N=256, k=8, f=128, capacity_factor=1.25), 0.01, 1e-3),
 ]
 
 
