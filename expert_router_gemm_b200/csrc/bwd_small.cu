@@ -18,6 +18,8 @@
 // All reductions run in a fixed order: results are deterministic.
 #include <math.h>
 
+#include <algorithm>
+
 #include "device_utils.cuh"
 #include "internal.h"
 
@@ -224,115 +226,6 @@ __global__ void router_wgrad_reduce_kernel(int n_chunks, int d, int N, const flo
   }
 }
 
-// The same two products for wide routers (N > 64) with 128 x 128 output tiles:
-// 256 threads, each an 8 x 8 register tile (rows {4ty + a, 64 + 4ty + a} and
-// columns {4tx + b, 64 + 4tx + b}, a, b < 4), so that every 64 FMAs read four
-// 16-byte words of shared memory.  Reduction slabs of 16.
-constexpr int WT = 128;
-constexpr int WK = 16;
-constexpr int WP = WT + 4;   // padded smem row (floats): 16-byte aligned rows
-
-__device__ __forceinline__ void tile_fma_8x8(const float (*as)[WP], const float (*bs)[WP], int tx, int ty,
-                                             float (&acc)[8][8]) {
-#pragma unroll 4
-  for (int r = 0; r < WK; ++r) {
-    const float4 a0 = *reinterpret_cast<const float4*>(&as[r][ty * 4]);
-    const float4 a1 = *reinterpret_cast<const float4*>(&as[r][64 + ty * 4]);
-    const float4 b0 = *reinterpret_cast<const float4*>(&bs[r][tx * 4]);
-    const float4 b1 = *reinterpret_cast<const float4*>(&bs[r][64 + tx * 4]);
-    const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-    const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-#pragma unroll
-    for (int a = 0; a < 8; ++a)
-#pragma unroll
-      for (int b = 0; b < 8; ++b) acc[a][b] = fmaf(av[a], bv[b], acc[a][b]);
-  }
-}
-
-__device__ __forceinline__ int tile_row(int ty, int a) { return a < 4 ? ty * 4 + a : 64 + ty * 4 + (a - 4); }
-
-// partial[z][c][i] = sum_{t in chunk z} x[t][c] dg[t][i] for c <= d (row d: x = 1,
-// the bias gradient)
-__global__ void __launch_bounds__(256) router_wgrad_wide_kernel(int64_t T, int d, int N, const uint16_t* __restrict__ x,
-                                                               const float* __restrict__ dg,
-                                                               float* __restrict__ part) {
-  __shared__ __align__(16) float xs[WK][WP];
-  __shared__ __align__(16) float gs[WK][WP];
-  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-  const int c0 = blockIdx.x * WT, i0 = blockIdx.y * WT;
-  const int64_t t_begin = static_cast<int64_t>(blockIdx.z) * kChunkRows;
-  const int64_t t_end = t_begin + kChunkRows < T ? t_begin + kChunkRows : T;
-  float acc[8][8] = {};
-  for (int64_t tb = t_begin; tb < t_end; tb += WK) {
-#pragma unroll
-    for (int u = 0; u < WK * WT / 256; ++u) {   // one row of 128 per 128 threads: coalesced
-      const int v = threadIdx.x + 256 * u;
-      const int r = v / WT, c = v % WT;
-      const int64_t t = tb + r;
-      float xv = 0.f, gv = 0.f;
-      if (t < t_end) {
-        if (c0 + c < d)
-          xv = __uint_as_float(static_cast<uint32_t>(x[t * d + c0 + c]) << 16);
-        else if (c0 + c == d)
-          xv = 1.f;
-        if (i0 + c < N) gv = dg[t * N + i0 + c];
-      }
-      xs[r][c] = xv;
-      gs[r][c] = gv;
-    }
-    __syncthreads();
-    tile_fma_8x8(xs, gs, tx, ty, acc);
-    __syncthreads();
-  }
-  float* pz = part + static_cast<int64_t>(blockIdx.z) * (d + 1) * N;
-#pragma unroll
-  for (int a = 0; a < 8; ++a) {
-    const int c = c0 + tile_row(ty, a);
-    if (c > d) continue;
-#pragma unroll
-    for (int b = 0; b < 8; ++b) {
-      const int i = i0 + tile_row(tx, b);
-      if (i < N) pz[static_cast<int64_t>(c) * N + i] = acc[a][b];
-    }
-  }
-}
-
-// dxr[t][c] = sum_i dg[t][i] W_r[c][i]
-__global__ void __launch_bounds__(256) router_dgrad_wide_kernel(int64_t T, int d, int N, const float* __restrict__ dg,
-                                                               const float* __restrict__ wr,
-                                                               float* __restrict__ dxr) {
-  __shared__ __align__(16) float gs[WK][WP];   // [i][t]
-  __shared__ __align__(16) float ws[WK][WP];   // [i][c]
-  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * WT;
-  const int c0 = blockIdx.y * WT;
-  float acc[8][8] = {};
-  for (int ib = 0; ib < N; ib += WK) {
-#pragma unroll
-    for (int u = 0; u < WK * WT / 256; ++u) {   // i fastest: 64-byte pieces of the rows of dg and W_r
-      const int v = threadIdx.x + 256 * u;
-      const int r = v / WK, i = v % WK;
-      const int64_t t = t0 + r;
-      const int c = c0 + r;
-      gs[i][r] = (t < T && ib + i < N) ? dg[t * N + ib + i] : 0.f;
-      ws[i][r] = (c < d && ib + i < N) ? wr[static_cast<int64_t>(c) * N + ib + i] : 0.f;
-    }
-    __syncthreads();
-    tile_fma_8x8(gs, ws, tx, ty, acc);
-    __syncthreads();
-  }
-#pragma unroll
-  for (int a = 0; a < 8; ++a) {
-    const int64_t t = t0 + tile_row(ty, a);
-    if (t >= T) continue;
-#pragma unroll
-    for (int b = 0; b < 8; ++b) {
-      const int c = c0 + tile_row(tx, b);
-      if (c < d) dxr[t * d + c] = acc[a][b];
-    }
-  }
-}
-
 // dxr[t][c] = sum_i dg[t][i] W_r[c][i]
 __global__ void __launch_bounds__(256) router_dgrad_kernel(int64_t T, int d, int N, const float* __restrict__ dg,
                                                           const float* __restrict__ wr, float* __restrict__ dxr) {
@@ -454,40 +347,211 @@ cudaError_t launch_zero_pad_rows(int N, const int32_t* seg_off, const int32_t* s
   return cudaGetLastError();
 }
 
-size_t router_wgrad_scratch_floats(int64_t T, int d, int N) {
-  const int64_t chunks = (T + kChunkRows - 1) / kChunkRows;
-  return static_cast<size_t>(chunks) * (d + 1) * N;
-}
+// ---------------------------------------------------------------- router gradients
+namespace {
 
-cudaError_t launch_router_wgrad(int64_t T, int d, int N, const uint16_t* x, const float* dg, float* dw_router,
-                                float* dbias, float* scratch, cudaStream_t s) {
-  if (T == 0) return cudaSuccess;
-  const int chunks = static_cast<int>((T + kChunkRows - 1) / kChunkRows);
-  if (N > 64) {
-    router_wgrad_wide_kernel<<<dim3(static_cast<unsigned>(d / WT + 1), static_cast<unsigned>((N + WT - 1) / WT),
-                                    static_cast<unsigned>(chunks)),
-                               256, 0, s>>>(T, d, N, x, dg, scratch);
-    router_wgrad_reduce_kernel<<<256, 256, 0, s>>>(chunks, d, N, scratch, dw_router, dbias);
-    return cudaGetLastError();
+constexpr int kColsumRows = 32;   // rows per block of the bias column sums
+
+// Tensor-core path: sizes of the operand and partial buffers.
+struct RgPlan {
+  bool tc;
+  int64_t T, Tp;        // Tp = T rounded up to 8 (16-byte rows of the transposed operand)
+  int d, N, Np, Nk;     // Np = N rounded up to 8, Nk = N rounded up to 64
+  int chunk, G;         // weight gradient: G row chunks of `chunk` rows (the last one ragged)
+  int bias_blocks;      // column sums of dg: blocks of kColsumRows rows
+  size_t parts, wpart, table, at, bt, bias, end;   // scratch offsets (bytes)
+  int64_t cc_chunks;    // CUDA-core path: rows chunks of kChunkRows
+};
+
+size_t up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+RgPlan rg_plan(int64_t T, int d, int N) {
+  RgPlan P{};
+  P.T = T;
+  P.d = d;
+  P.N = N;
+  P.tc = N >= 64 && T >= 64;
+  P.Tp = (T + 7) / 8 * 8;
+  P.Np = (N + 7) / 8 * 8;
+  P.Nk = (N + 63) / 64 * 64;
+  P.chunk = static_cast<int>(std::max<int64_t>(1024, (T + 255) / 256 + 63) / 64 * 64);
+  P.G = static_cast<int>((T + P.chunk - 1) / P.chunk);
+  P.bias_blocks = static_cast<int>((T + kColsumRows - 1) / kColsumRows);
+  P.cc_chunks = (T + kChunkRows - 1) / kChunkRows;
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at_ = o;
+    o = up(o + bytes, 256);
+    return at_;
+  };
+  if (P.tc) {
+    P.parts = take(2ull * T * P.Np * 2);                        // dg hi / lo, bf16 [2][T][Np]
+    P.wpart = take(2ull * P.G * d * P.Np * 4);                  // fp32 [2][G][d][Np]
+    P.table = take(4ull * (P.G + 1));                           // chunk row offsets
+    P.at = take(3ull * P.Nk * P.Tp * 2);                        // [dg_hi^T; dg_hi^T; dg_lo^T] bf16
+    P.bt = take(3ull * P.Nk * d * 2);                           // [W_hi^T; W_lo^T; W_hi^T] bf16
+    P.bias = take(4ull * P.bias_blocks * N);                    // column sums of dg per kColsumRows rows
+  } else {
+    P.wpart = take(4ull * P.cc_chunks * (d + 1) * N);
   }
-  router_wgrad_kernel<<<dim3(static_cast<unsigned>(d / RT + 1), static_cast<unsigned>((N + RT - 1) / RT),
-                             static_cast<unsigned>(chunks)),
-                        256, 0, s>>>(T, d, N, x, dg, scratch);
-  router_wgrad_reduce_kernel<<<256, 256, 0, s>>>(chunks, d, N, scratch, dw_router, dbias);
-  return cudaGetLastError();
+  P.end = o;
+  return P;
 }
 
-cudaError_t launch_router_dgrad(int64_t T, int d, int N, const float* dg, const float* w_router, float* dxr,
+__device__ __forceinline__ void split2(float v, uint16_t& hi, uint16_t& lo) {
+  const __nv_bfloat16 h = __float2bfloat16_rn(v);
+  const __nv_bfloat16 l = __float2bfloat16_rn(v - __bfloat162float(h));
+  hi = *reinterpret_cast<const uint16_t*>(&h);
+  lo = *reinterpret_cast<const uint16_t*>(&l);
+}
+
+// parts[0][t][i] = hi(dg[t][i]), parts[1][t][i] = lo(dg[t][i]); zero for N <= i < Np
+__global__ void dg_split_kernel(int64_t T, int N, int Np, const float* __restrict__ dg, uint16_t* __restrict__ parts) {
+  const int64_t total = T * Np;
+  for (int64_t v = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; v < total;
+       v += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t t = v / Np;
+    const int i = static_cast<int>(v - t * Np);
+    uint16_t hi = 0, lo = 0;
+    if (i < N) split2(dg[t * N + i], hi, lo);
+    parts[v] = hi;
+    parts[total + v] = lo;
+  }
+}
+
+// Transposed split of a fp32 [R, N] matrix into three stacked bf16 blocks of
+// [Nk][Rp] (rows i >= N and columns r >= R zero): block b holds part
+// (sel >> b) & 1 of src^T (0 = hi, 1 = lo).  32 x 32 tiles through shared memory.
+__global__ void split_transpose_kernel(int64_t R, int64_t Rp, int N, int Nk, const float* __restrict__ src,
+                                       uint16_t* __restrict__ out, int sel) {
+  __shared__ float tile[32][33];
+  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * 32;
+  const int i0 = blockIdx.y * 32;
+  for (int y = threadIdx.y; y < 32; y += blockDim.y) {
+    const int64_t r = r0 + y;
+    const int i = i0 + threadIdx.x;
+    tile[y][threadIdx.x] = (r < R && i < N) ? src[r * N + i] : 0.f;
+  }
+  __syncthreads();
+  for (int y = threadIdx.y; y < 32; y += blockDim.y) {
+    const int i = i0 + y;
+    const int64_t r = r0 + threadIdx.x;
+    if (r >= Rp) continue;
+    uint16_t hi, lo;
+    split2(tile[threadIdx.x][y], hi, lo);
+#pragma unroll
+    for (int b = 0; b < 3; ++b) out[(static_cast<int64_t>(b) * Nk + i) * Rp + r] = ((sel >> b) & 1) ? lo : hi;
+  }
+}
+
+__global__ void chunk_table_kernel(int G, int chunk, int64_t T, int32_t* __restrict__ table) {
+  for (int g = threadIdx.x; g <= G; g += blockDim.x)
+    table[g] = static_cast<int32_t>(static_cast<int64_t>(g) * chunk < T ? static_cast<int64_t>(g) * chunk : T);
+}
+
+// part[b][i] = sum of dg[t][i] over the kColsumRows rows of block b, in row order
+__global__ void __launch_bounds__(256) dg_colsum_kernel(int64_t T, int N, const float* __restrict__ dg,
+                                                        float* __restrict__ part) {
+  const int i = threadIdx.x;
+  if (i >= N) return;
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kColsumRows;
+  const int64_t t1 = t0 + kColsumRows < T ? t0 + kColsumRows : T;
+  float s = 0.f;
+  for (int64_t t = t0; t < t1; t += 8) {
+    float v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] = t + u < t1 ? dg[(t + u) * N + i] : 0.f;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) s += v[u];
+  }
+  part[static_cast<int64_t>(blockIdx.x) * N + i] = s;
+}
+
+// dw[c][i] = sum over (part, chunk) of wpart[part][chunk][c][i] (parts outer, chunks
+// inner); dbias[i] = sum over blocks of colsum[b][i]
+__global__ void router_grad_reduce_kernel(int G, int d, int N, int Np, int bias_blocks, const float* __restrict__ wpart,
+                                          const float* __restrict__ colsum, float* __restrict__ dw,
+                                          float* __restrict__ dbias) {
+  const int64_t total = static_cast<int64_t>(d) * N;
+  const int64_t plane = static_cast<int64_t>(d) * Np;
+  for (int64_t v = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; v < total + N;
+       v += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    if (v < total) {
+      const int64_t c = v / N;
+      const int i = static_cast<int>(v - c * N);
+      float s = 0.f;
+      for (int q = 0; q < 2 * G; ++q) s += wpart[q * plane + c * Np + i];
+      dw[v] = s;
+    } else if (dbias != nullptr) {
+      const int i = static_cast<int>(v - total);
+      float s = 0.f;
+      for (int b = 0; b < bias_blocks; ++b) s += colsum[static_cast<int64_t>(b) * N + i];
+      dbias[i] = s;
+    }
+  }
+}
+
+}  // namespace
+
+size_t router_grad_scratch_bytes(int64_t T, int d, int N) { return rg_plan(T, d, N).end; }
+
+int64_t router_dxr_rows(int64_t T) { return (T + 7) / 8 * 8; }
+
+cudaError_t launch_router_grads(int64_t T, int d, int N, const uint16_t* x, const float* dg, const float* w_router,
+                                float* dw_router, float* dbias, float* dxr, void* scratch, uint32_t* flags,
                                 cudaStream_t s) {
   if (T == 0) return cudaSuccess;
-  if (N > 64) {
-    router_dgrad_wide_kernel<<<dim3(static_cast<unsigned>((T + WT - 1) / WT), static_cast<unsigned>((d + WT - 1) / WT)),
-                               256, 0, s>>>(T, d, N, dg, w_router, dxr);
+  const RgPlan P = rg_plan(T, d, N);
+  uint8_t* sc = static_cast<uint8_t*>(scratch);
+  if (!P.tc) {
+    const int chunks = static_cast<int>(P.cc_chunks);
+    float* part = reinterpret_cast<float*>(sc + P.wpart);
+    router_wgrad_kernel<<<dim3(static_cast<unsigned>(d / RT + 1), static_cast<unsigned>((N + RT - 1) / RT),
+                               static_cast<unsigned>(chunks)),
+                          256, 0, s>>>(T, d, N, x, dg, part);
+    router_wgrad_reduce_kernel<<<256, 256, 0, s>>>(chunks, d, N, part, dw_router, dbias);
+    router_dgrad_kernel<<<dim3(static_cast<unsigned>((T + RT - 1) / RT), static_cast<unsigned>((d + RT - 1) / RT)),
+                          256, 0, s>>>(T, d, N, dg, w_router, dxr);
     return cudaGetLastError();
   }
-  router_dgrad_kernel<<<dim3(static_cast<unsigned>((T + RT - 1) / RT), static_cast<unsigned>((d + RT - 1) / RT)), 256,
-                        0, s>>>(T, d, N, dg, w_router, dxr);
-  return cudaGetLastError();
+  uint16_t* parts = reinterpret_cast<uint16_t*>(sc + P.parts);
+  float* wpart = reinterpret_cast<float*>(sc + P.wpart);
+  int32_t* table = reinterpret_cast<int32_t*>(sc + P.table);
+  uint16_t* at_ = reinterpret_cast<uint16_t*>(sc + P.at);
+  uint16_t* bt = reinterpret_cast<uint16_t*>(sc + P.bt);
+  float* colsum = reinterpret_cast<float*>(sc + P.bias);
+  const int sms = device_sm_count();
+
+  // dW_r = x^T dg_hi + x^T dg_lo, per chunk of rows (fills the GPU), then the fixed-order sum
+  dg_split_kernel<<<4 * sms, 256, 0, s>>>(T, N, P.Np, dg, parts);
+  chunk_table_kernel<<<1, 256, 0, s>>>(P.G, P.chunk, T, table);
+  dg_colsum_kernel<<<P.bias_blocks, 256, 0, s>>>(T, N, dg, colsum);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  BwdGroups chunks{};
+  chunks.G = P.G;
+  chunks.max_rows = T;
+  chunks.seg_off = table;
+  chunks.flags = flags;
+  for (int q = 0; q < 2 && e == cudaSuccess; ++q)
+    e = launch_wgrad(chunks, d, P.Np, x, parts + static_cast<int64_t>(q) * T * P.Np,
+                     wpart + static_cast<int64_t>(q) * P.G * d * P.Np, s);
+  if (e != cudaSuccess) return e;
+  router_grad_reduce_kernel<<<2 * sms, 256, 0, s>>>(P.G, d, N, P.Np, P.bias_blocks, wpart, colsum, dw_router, dbias);
+
+  // dxr = dg W_r^T = [dg_hi | dg_hi | dg_lo] [W_hi | W_lo | W_hi]^T: one GEMM over 3 Nk stacked rows
+  split_transpose_kernel<<<dim3(static_cast<unsigned>((P.Tp + 31) / 32), static_cast<unsigned>(P.Nk / 32)),
+                           dim3(32, 8), 0, s>>>(T, P.Tp, N, P.Nk, dg, at_, 0b100);   // hi, hi, lo
+  split_transpose_kernel<<<dim3(static_cast<unsigned>((d + 31) / 32), static_cast<unsigned>(P.Nk / 32)),
+                           dim3(32, 8), 0, s>>>(d, d, N, P.Nk, w_router, bt, 0b010);   // hi, lo, hi
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  BwdGroups stacked{};
+  stacked.G = 1;
+  stacked.dense_rows = 3 * P.Nk;
+  stacked.max_rows = 3 * P.Nk;
+  stacked.flags = flags;
+  return launch_wgrad(stacked, static_cast<int>(P.Tp), d, at_, bt, dxr, s);
 }
 
 cudaError_t launch_dx_gather(int64_t T, int d, int k, const int32_t* row_map, const uint16_t* dXp, const float* dxr,

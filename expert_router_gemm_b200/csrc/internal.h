@@ -236,13 +236,17 @@ struct PadBufs {
 };
 cudaError_t launch_zero_pad_rows(int N, const int32_t* seg_off, const int32_t* seg_count, const PadBufs& b,
                                  cudaStream_t s);
-// dW_r = x^T dg (fp32 [d, N]) and dbias = sum_t dg[t] (may be null), with
-// per-chunk partials summed in a fixed order (scratch: n_chunks * (d + 1) * N floats).
-size_t router_wgrad_scratch_floats(int64_t T, int d, int N);
-cudaError_t launch_router_wgrad(int64_t T, int d, int N, const uint16_t* x, const float* dg, float* dw_router,
-                                float* dbias, float* scratch, cudaStream_t s);
-// dxr = dg W_r^T (fp32 [T, d]).
-cudaError_t launch_router_dgrad(int64_t T, int d, int N, const float* dg, const float* w_router, float* dxr,
+// The router's two gradient products (x bf16 [T, d], dg fp32 [T, N], W_r fp32
+// [d, N]): dW_r = x^T dg (fp32 [d, N]), dbias = sum_t dg[t] (may be null) and
+// dxr = dg W_r^T (fp32, router_dxr_rows(T) rows of d; rows >= T are scratch).
+// Wide routers (N >= 64, T >= 64) run on the tensor cores through the weight-
+// gradient GEMM: the fp32 operands split into bf16 parts (dg = hi + lo,
+// W_r = hi + lo; x is bf16 already), the part products summed in fp32.  Small
+// routers run on CUDA cores.  Partial sums are added in a fixed order.
+size_t router_grad_scratch_bytes(int64_t T, int d, int N);
+int64_t router_dxr_rows(int64_t T);
+cudaError_t launch_router_grads(int64_t T, int d, int N, const uint16_t* x, const float* dg, const float* w_router,
+                                float* dw_router, float* dbias, float* dxr, void* scratch, uint32_t* flags,
                                 cudaStream_t s);
 // dx[t] = sum over kept slots of dXp[row] + dxr[t] (+ dxs[t]), one rounding to bf16.
 cudaError_t launch_dx_gather(int64_t T, int d, int k, const int32_t* row_map, const uint16_t* dXp, const float* dxr,

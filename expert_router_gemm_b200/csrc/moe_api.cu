@@ -195,8 +195,8 @@ BwdLayout bwd_layout(const Dims& D) {
   B.counts = take(4 * D.N);
   B.dw = take(4 * T * D.k);
   B.dg = take(4 * T * D.N);
-  B.dxr = take(4 * T * D.d);
-  B.rws = take(4 * router_wgrad_scratch_floats(D.T, D.d, D.N));
+  B.dxr = take(4 * static_cast<size_t>(router_dxr_rows(D.T)) * D.d);
+  B.rws = take(router_grad_scratch_bytes(D.T, D.d, D.N));
   B.xp = take(2 * R * D.d);
   B.g = take(2 * R * D.f);
   B.u = take(2 * R * D.f);
@@ -804,11 +804,10 @@ moe_status_t moe_layer_bwd(const moe_config_t* cfg, const moe_weights_t* weights
   if (e == cudaSuccess) e = launch_wgrad(grp, d, f, xp, u, grads->dw3, st);
   if (e == cudaSuccess) e = launch_wgrad(grp, f, d, h, o, grads->dw2, st);
   if (e == cudaSuccess) e = launch_dgrad_plain2(grp, d, f, g, u, weights->w1, weights->w3, xp, st);   // dXp over xp
-  if (e == cudaSuccess)
-    e = launch_router_wgrad(T, d, N, static_cast<const uint16_t*>(x), a.dg, grads->dw_router, dbias,
-                            at<float*>(ws, B.rws), st);
   float* dxr = at<float*>(ws, B.dxr);
-  if (e == cudaSuccess) e = launch_router_dgrad(T, d, N, a.dg, weights->w_router, dxr, st);
+  if (e == cudaSuccess)
+    e = launch_router_grads(T, d, N, static_cast<const uint16_t*>(x), a.dg, weights->w_router, grads->dw_router,
+                            dbias, dxr, at<void*>(ws, B.rws), flags, st);
   if (e != cudaSuccess) return cuda_status(e);
 
   void* dxs = nullptr;
