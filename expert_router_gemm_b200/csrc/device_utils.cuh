@@ -216,6 +216,16 @@ __device__ __forceinline__ void tc_mma_f16_pair(uint32_t d_tmem, uint64_t adesc,
 }
 // Arrive once on `bar` (a shared::cluster address, this CTA's or the peer's)
 // when every pair MMA issued so far by this thread has completed.
+// One commit whose arrival lands on the mbarrier at this shared-memory offset
+// in both CTAs of the pair (cta mask 0b11).  This is the MMA-completion commit,
+// not a memory load: two separate commits per K slab cost the pair GEMM about
+// 7 % of its tensor-pipe cycles.
+__device__ __forceinline__ void tc_commit_pair_both(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+      "h"(static_cast<uint16_t>(3))
+      : "memory");
+}
 __device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
                : "memory");

@@ -343,9 +343,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               tc_mma_mxf8(d_tmem, adesc, bdesc, idesc, sfa_col | sel, sfb_col | sel, (kb | kk) != 0 ? 1u : 0u);
           }
           if (CG == 2) {
-            const uint32_t e = smem_addr(&tl.empty[stage]);
-            tc_commit_pair(e);
-            tc_commit_pair(mapa_shared(e, 1));
+            tc_commit_pair_both(smem_addr(&tl.empty[stage]));
           } else {
             tc_commit(smem_addr(&tl.empty[stage]));
           }
@@ -356,9 +354,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!ok) break;
         if (CG == 2) {
-          const uint32_t f = smem_addr(&tl.tfull[acc]);
-          tc_commit_pair(f);
-          tc_commit_pair(mapa_shared(f, 1));
+          tc_commit_pair_both(smem_addr(&tl.tfull[acc]));
         } else {
           tc_commit(smem_addr(&tl.tfull[acc]));
         }

@@ -221,8 +221,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         any = true;
         const uint32_t e = smem_addr(&tl.empty[stage]);
         if (CG == 2) {
-          tc_commit_pair(e);
-          tc_commit_pair(mapa_shared(e, 1));
+          tc_commit_pair_both(e);
         } else {
           tc_commit(e);
         }
@@ -235,8 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (any) {  // hand the accumulator to the epilogues; every MMA has drained before TMEM is freed
         const uint32_t f = smem_addr(&tl.tfull);
         if (CG == 2) {
-          tc_commit_pair(f);
-          tc_commit_pair(mapa_shared(f, 1));
+          tc_commit_pair_both(f);
         } else {
           tc_commit(f);
         }
