@@ -62,8 +62,20 @@ def _gpu_backward(dl, dy, aux, z):
 
 @pytest.mark.parametrize("w,aux,z", CASES, ids=[c[0].name for c in CASES])
 def test_layer_backward_vs_oracle(w, aux, z):
+    _check_backward(w, aux, z)
+
+
+def test_layer_backward_segments_aligned_to_64():
+    """Segments padded to 64 rows: a 128- or 256-row GEMM tile of one expert
+    reaches into the next expert's rows, which its epilogue must leave alone
+    (about 37 kept rows per expert here)."""
+    w = Workload("bwd-align64", T=300, d=256, N=16, k=2, f=128, capacity_factor=1.25)
+    _check_backward(w, 0.05, 1e-3, seg_align=64)
+
+
+def _check_backward(w, aux, z, seg_align=0):
     inp = synth.make_inputs(w)
-    cfg = moe.config_from_workload(w)
+    cfg = moe.config_from_workload(w, seg_align=seg_align)
     dl = moe.to_device(inp, cfg)
     dy = synth.f32_to_bf16_bits(synth.normal_f32(11, 77, (w.T, w.d)))
     # the routing of the GPU equals the oracle's (no near ties in these cases)
@@ -150,3 +162,20 @@ def test_layer_backward_edge_cases(w, aux, z, sel):
             continue
         rel = orc.rel_frobenius(np.asarray(a, np.float64), b)
         assert rel <= TOL, (w.name, name, rel)
+
+
+@pytest.mark.parametrize("cta_group", ["1", "2"])
+def test_layer_backward_cta_group_variants(cta_group):
+    """Both tile shapes of the backward GEMMs (single CTAs with 128-row tiles,
+    CTA pairs with 256-row tiles) on every small case, each shape in its own
+    process (the choice is made once per process)."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, MOE_BWD_CTA_GROUP=cta_group)
+    sel = [__file__ + "::test_layer_backward_vs_oracle", __file__ + "::test_layer_backward_edge_cases",
+           __file__ + "::test_layer_backward_segments_aligned_to_64"]
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider", *sel], env=env,
+                       cwd=root, capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
