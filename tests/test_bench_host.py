@@ -1,0 +1,85 @@
+"""Host logic of bench.py on the CPU: the DRAM-traffic records keyed to kernel
+sources, the peak table and its fallback, the CPU-rate arithmetic, and the JSON
+line of the reference arm (the fp64 oracle, which needs no GPU)."""
+import hashlib
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+
+def _fake_root(tmp_path, kernel_src: bytes, records: str):
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "expert_router_gemm_b200" / "csrc").mkdir(parents=True)
+    (tmp_path / "expert_router_gemm_b200" / "csrc" / "k.cu").write_bytes(kernel_src)
+    (tmp_path / "profiles" / "dram_traffic.txt").write_text(records)
+    return hashlib.sha256(kernel_src).hexdigest()[:16]
+
+
+def test_traffic_record_applies_only_to_the_captured_source(tmp_path, monkeypatch):
+    sha = _fake_root(tmp_path, b"kernel v1", "")
+    (tmp_path / "profiles" / "dram_traffic.txt").write_text(
+        "# comment line " + sha + " 1 2\n"
+        f"expert_ffn_per_step {sha} 100.5e6 20e6\n"
+        "expert_ffn_per_step 0123456789abcdef 7e6 8e6\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.traffic_record("k.cu") == {"expert_ffn_per_step": pytest.approx(120.5e6)}
+    # the source changes: the counters no longer describe it
+    (tmp_path / "expert_router_gemm_b200" / "csrc" / "k.cu").write_bytes(b"kernel v2")
+    assert bench.traffic_record("k.cu") is None
+    assert bench.traffic_record("missing.cu") is None
+
+
+def test_committed_traffic_records_are_well_formed():
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    lines = [ln.split() for ln in open(path) if ln.strip() and not ln.startswith("#")]
+    assert lines
+    for unit, sha, rd, wr in lines:
+        assert unit == "expert_ffn_per_step"
+        assert len(sha) == 16 and int(sha, 16) >= 0
+        assert float(rd) > 0 and float(wr) > 0
+
+
+def test_peaks_fall_back_when_the_measured_file_is_absent(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    peaks, src = bench.load_peaks()
+    assert src == "fallback" and peaks == bench.FALLBACK_PEAKS
+    (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({"hbm_gbs": 1.0, "bf16_tflops": 2.0,
+                                                             "bf16_tflops_sustained": 3.0}))
+    peaks, src = bench.load_peaks()
+    assert src == "measured" and peaks["bf16_tflops_sustained"] == 3.0
+
+
+def test_cpu_rate_amortises_the_routing_per_token():
+    # two steps of 100 and 300 token-equivalents in 1 s and 3 s, routing of
+    # T = 1000 tokens in 2 s: 400 tokens cost 4 s + 2 * 400 / 1000 s
+    rate, tok, sec = bench.cpu_rate([(100, 1.0), (300, 3.0)], 2.0, 1000)
+    assert tok == 400 and sec == pytest.approx(4.8)
+    assert rate == pytest.approx(400 / 4.8)
+    assert bench.cpu_rate([], 0.0, 10)[0] == 0.0
+
+
+def test_reference_arm_json_line():
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--config", "tiny", "--steps", "2",
+                        "--warmup", "3"], cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stdout[-2000:] + r.stderr[-2000:]
+    lines = [json.loads(x) for x in r.stdout.splitlines() if x.startswith("{")]
+    assert len(lines) == 1
+    line = lines[0]
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC
+    assert line["n_gpus"] == 1 and line["steps"] == 2 and line["warmup"] == 3
+    assert line["value"] > 0 and line["unit"] == "tokens/s" and line["higher_is_better"] is True
+    assert line["config"]["workload"] == "tiny-fp32"
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["cpu_baseline"]["value"] == line["value"]
+    assert line["e2e"] == {"value": line["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
