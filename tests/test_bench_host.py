@@ -83,3 +83,28 @@ def test_reference_arm_json_line():
     assert line["cpu_baseline"]["value"] == line["value"]
     assert line["e2e"] == {"value": line["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
+
+
+def test_clock_summary_decodes_reasons_and_takes_the_median():
+    s = bench.ClockSampler.__new__(bench.ClockSampler)
+    s.ok, s.max_mhz = True, 1965
+    # (SM MHz, watts, clocks-event-reason bits): idle is not reported, the others are
+    s.samples = [(1200, 700.0, 0x1), (1100, 990.0, 0x4), (1300, 650.0, 0x4 | 0x40)]
+    c = s.summary()
+    assert c["sm_mhz"] == 1200 and c["sm_max_mhz"] == 1965 and c["samples"] == 3
+    assert c["power_w_max"] == 990.0
+    assert c["reasons"] == ["sw_power_cap", "hw_thermal_slowdown"]
+    s.samples = []
+    assert s.summary()["samples"] == 0
+    s.ok = False
+    assert s.summary()["sm_mhz"] is None
+
+
+def test_workload_config_names_the_workload_and_its_sizes():
+    from expert_router_gemm_b200 import configs
+    w = configs.get("qwen3")
+    c = bench.workload_config(w)
+    assert c["workload"] == "qwen3-moe-shaped"
+    assert (c["T"], c["d"], c["N"], c["k"], c["f"]) == (8192, 4096, 128, 8, 1536)
+    assert c["capacity"] == 512 and c["act_dtype"] == "bf16" and c["router_dtype"] == "f32"
+    assert "model" not in c
