@@ -6,6 +6,7 @@ CPU) and confirm that at least one pin catches it.
 """
 import itertools
 import math
+import struct
 
 import numpy as np
 import pytest
@@ -500,8 +501,88 @@ def check_bf16_decode(o=orc):
     np.testing.assert_array_equal(o.bf16_bits_to_f64(bits), want)
 
 
+def _py_bf16_rne(v: float) -> float:
+    """Round a Python float to the nearest bf16 value, ties to even, by integer
+    arithmetic on its IEEE-754 double bit pattern (sign, 11-bit exponent, 52-bit
+    fraction): bf16 keeps 7 fraction bits, so 45 fraction bits are dropped.
+    Normal, finite values only (the cases below stay far from the extremes)."""
+    bits = struct.unpack("<Q", struct.pack("<d", v))[0]
+    drop = 45
+    keep = bits >> drop
+    rest = bits & ((1 << drop) - 1)
+    half = 1 << (drop - 1)
+    if rest > half or (rest == half and (keep & 1)):
+        keep += 1                       # a carry into the exponent is the right result
+    return struct.unpack("<d", struct.pack("<Q", keep << drop))[0]
+
+
+def check_layer_bf16_h_rounding(o=orc):
+    # bf16 compute with fp32 accumulation, read as: h = silu(x W1) * (x W3) is
+    # formed exactly, rounded once to bf16 (nearest, ties to even), and only then
+    # multiplied by W2 ("MoE 训练加速实战" §2.2 for the layer; reading (iii) for
+    # where the one bf16 rounding sits).  Tokens are one-hot rows of a 4 x 4
+    # identity, so token t's hidden unit j sees g = W1[t, j], u = W3[t, j]; for
+    # g >= 64, e^-g < 2^-92 and silu(g) = g exactly in fp64, so h = g * u is an
+    # exact dyadic number placed on or next to a bf16 rounding boundary.
+    d = f = 4
+    w1 = np.full((1, d, f), 64.0)
+    w3 = np.zeros((1, d, f))
+    cases = {  # (token, unit): (g, u, bf16(h) worked out by hand)
+        (0, 0): (64.0, (1 + 2.0**-8) / 64, 1.0),                         # tie -> even (down)
+        (0, 1): (64.0, (1 + 3 * 2.0**-8) / 64, 1 + 2.0**-6),             # tie -> even (up)
+        (0, 2): (96.0, 2.0**-6 * (1 + 2.0**-8 + 2.0**-9), 1.5078125),    # h = 1.5087890625
+        (0, 3): (64.0, -(1 + 2.0**-8 + 2.0**-30) / 64, -(1 + 2.0**-7)),  # just past a tie
+        (1, 0): (64.0, 2.0**-6 * (1 + 2.0**-9), 1.0),                    # below half a step
+        (1, 1): (128.0, 3 * 2.0**-7 * (1 + 2.0**-9), 3.0),
+        (1, 2): (64.0, 2.0**-6 * 257 / 256 * 3, 3.015625),                # 3 (1 + 2^-8): 3/4 step, up
+        (1, 3): (64.0, 2.0**-6 * (1 - 2.0**-10), 1.0),                   # rounds up to 1
+    }
+    for (t, j), (g, u, _) in cases.items():
+        w1[0, t, j], w3[0, t, j] = g, u
+    w2 = np.zeros((1, f, d))
+    for j in range(f):
+        w2[0, j, j] = 3.0                 # o_j = 3 bf16(h_j): rounding o instead of h shows
+    x = np.eye(4, dtype=np.float32)
+    wr = np.zeros((d, 1), dtype=np.float32)
+    res = o.layer_forward(x, wr, None, w1, w3, w2, k=1, cap=4, bf16=True, align=1)
+    for (t, j), (g, u, want_h) in cases.items():
+        assert res.y[t, j] == 3.0 * want_h, ((t, j), res.y[t, j], 3.0 * want_h)
+        assert _py_bf16_rne(g * u) == want_h, ((t, j), g * u)   # the hand values themselves
+    # the same layer without the rounding keeps h exact
+    res32 = o.layer_forward(x, wr, None, w1, w3, w2, k=1, cap=4, bf16=False, align=1)
+    for (t, j), (g, u, _) in cases.items():
+        assert res32.y[t, j] == 3.0 * g * u, ((t, j), res32.y[t, j])
+
+    # random small layer: every output against a plain-Python loop that rounds h
+    # with the integer rounding above and nothing else
+    rng = np.random.default_rng(31)
+    T, d, f, N = 5, 8, 6, 3
+    x = rng.normal(size=(T, d)).astype(np.float32)
+    wr = rng.normal(size=(d, N)).astype(np.float32)
+    w1, w3, w2 = _tiny_weights(rng, N, d, f)
+    res = o.layer_forward(x, wr, None, w1, w3, w2, k=N, cap=T, bf16=True, align=1)
+    for t in range(T):
+        xr = [float(v) for v in x[t]]
+        gl = [sum(xr[c] * float(wr[c, i]) for c in range(d)) for i in range(N)]
+        m = max(gl)
+        ex = [math.exp(v - m) for v in gl]
+        s = [v / sum(ex) for v in ex]
+        want = [0.0] * d
+        for i in range(N):
+            gg = _py_matvec(xr, w1[i].tolist())
+            uu = _py_matvec(xr, w3[i].tolist())
+            h = [_py_bf16_rne(a / (1.0 + math.exp(-a)) * b) for a, b in zip(gg, uu)]
+            oi = _py_matvec(h, w2[i].tolist())
+            want = [acc + s[i] * b for acc, b in zip(want, oi)]
+        np.testing.assert_allclose(res.y[t], want, rtol=1e-12, atol=1e-12)
+
+
 def test_bf16_rounding():
     check_bf16_rounding()
+
+
+def test_layer_bf16_h_rounding():
+    check_layer_bf16_h_rounding()
 
 
 def test_bf16_decode():
@@ -518,7 +599,7 @@ ALL_CHECKS = [check_capacity_worked_example, check_capacity_closed_forms, check_
               check_dropped_slots_contribute_zero, check_shared_expert_added, check_aux_hand,
               check_aux_uniform, check_bf16_rounding, check_bf16_decode, check_selection_bias_hand,
               check_selection_bias_bruteforce, check_bias_update_hand, check_z_loss,
-              check_load_metrics_hand, check_aux_loss_free_balances]
+              check_load_metrics_hand, check_aux_loss_free_balances, check_layer_bf16_h_rounding]
 
 
 def _mut_topk_high_index_ties(g, k, selection_bias=None):
@@ -655,6 +736,34 @@ def _mut_load_avg_counts(counts, kept, T, k):
     return m
 
 
+def _mut_swiglu_no_h_rounding(x64, w1, w3, w2, round_h_bf16):
+    # the bf16 flag is ignored: h reaches W2 unrounded
+    return _ORIG["swiglu_ffn"](x64, w1, w3, w2, False)
+
+
+def _mut_swiglu_rounds_output(x64, w1, w3, w2, round_h_bf16):
+    # the rounding is applied to the expert output instead of h
+    o = _ORIG["swiglu_ffn"](x64, w1, w3, w2, False)
+    return orc.round_to_bf16(o) if round_h_bf16 else o
+
+
+def _mut_swiglu_rounds_gate_up(x64, w1, w3, w2, round_h_bf16):
+    # g and u are rounded before silu and the product, h itself is not
+    g = x64 @ orc.as_f64(w1)
+    u = x64 @ orc.as_f64(w3)
+    if round_h_bf16:
+        g, u = orc.round_to_bf16(g), orc.round_to_bf16(u)
+    return (orc.silu(g) * u) @ orc.as_f64(w2)
+
+
+def _mut_swiglu_truncates_h(x64, w1, w3, w2, round_h_bf16):
+    # h is cut to bf16 by dropping the low half of its fp32 pattern (no rounding)
+    h = orc.silu(x64 @ orc.as_f64(w1)) * (x64 @ orc.as_f64(w3))
+    if round_h_bf16:
+        h = (h.astype(np.float32).view(np.uint32) & np.uint32(0xFFFF0000)).view(np.float32).astype(np.float64)
+    return h @ orc.as_f64(w2)
+
+
 _ORIG = {n: getattr(orc, n) for n in ("dispatch", "swiglu_ffn", "aux_stats", "topk", "load_metrics")}
 
 MUTANTS = [
@@ -680,6 +789,10 @@ MUTANTS = [
     ("load_metrics", _mut_load_std_sample),
     ("load_metrics", _mut_load_top1),
     ("load_metrics", _mut_load_avg_counts),
+    ("swiglu_ffn", _mut_swiglu_no_h_rounding),
+    ("swiglu_ffn", _mut_swiglu_rounds_output),
+    ("swiglu_ffn", _mut_swiglu_rounds_gate_up),
+    ("swiglu_ffn", _mut_swiglu_truncates_h),
 ]
 
 
