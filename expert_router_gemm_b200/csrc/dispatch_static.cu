@@ -4,10 +4,11 @@
 // file-scope device array of fixed size that the library holds on every GPU
 // that loads it.  The host never touches the array through its name: the name
 // is only a host-side stand-in, so the device address is looked up with
-// cudaGetSymbolAddress (once per device, with that device current) and passed
-// to the kernels as plain pointers.
-#include <mutex>
-
+// cudaGetSymbolAddress, with the caller's device current, on every call and
+// passed to the kernels as plain pointers.  Looking it up each time (a host-side
+// table lookup once the device code is loaded) keeps the address right even
+// after cudaDeviceReset or a new primary context, which load the module again
+// and may place the array elsewhere.
 #include "internal.h"
 
 namespace {
@@ -23,23 +24,14 @@ static_assert(kFlagOff + 256 <= kScratchBytes, "static dispatch scratch layout")
 
 static __device__ __align__(256) uint8_t g_dispatch_scratch[kScratchBytes];
 
-std::mutex g_mu;
-void* g_scratch_addr[64] = {};
-
-// Device address of g_dispatch_scratch on the current device.
+// Device address of g_dispatch_scratch in the current device's context.  The
+// first lookup on a device loads the library's device code there.
 cudaError_t scratch_address(uint8_t** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_dispatch_scratch);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lock(g_mu);
-  if (g_scratch_addr[dev] == nullptr) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_dispatch_scratch);
-    if (e != cudaSuccess) return e;
-    g_scratch_addr[dev] = p;
-  }
-  *out = static_cast<uint8_t*>(g_scratch_addr[dev]);
+  if (p == nullptr) return cudaErrorInvalidSymbol;
+  *out = static_cast<uint8_t*>(p);
   return cudaSuccess;
 }
 

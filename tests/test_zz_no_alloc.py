@@ -5,11 +5,13 @@ device memory belongs to another allocator, or they allocate only at start-up
 and may not call cudaMalloc (which can fail and synchronises the device) while
 serving.  moe_dispatch_static serves them with a fixed scratch array inside the
 library instead of a caller workspace.  This test calls it through the C ABI
-twice in a row (the second call finds the first call's leftovers in the shared
-array) and requires the same bytes as moe_dispatch, the entry point with a
-workspace: dispatch results are integers and copied rows, so the tolerance of
-the dispatch tests applies, which is exact equality.  The file sorts last so
-that a run stopping at the first failure has run every other test before it.
+twice in a row on each case (the second call finds the first call's leftovers
+in the shared array, and the second case the first case's) and requires the
+same bytes as moe_dispatch, the entry point with a workspace, and the oracle's
+dispatch itself: dispatch results are integers and copied rows, so the
+tolerance of the dispatch tests applies, which is exact equality.  The file
+sorts last so that a run stopping at the first failure has run every other test
+before it.
 """
 import numpy as np
 import pytest
@@ -55,13 +57,25 @@ def test_static_dispatch_matches_workspace_dispatch_twice():
             x = synth.f32_to_bf16_bits(x)
         cfg = moe.make_config(T=T, d=d, N=N, k=k, f=64, capacity=cap, dtype=dtype)
         xt, it = gu.cuda_tensor(x), gu.cuda_tensor(idx)
-        got = _static_dispatch(cfg, xt, it)
         want = gu.dispatch(cfg, xt, it)
-        assert got["flags"] == 0 and want["flags"] == 0
-        for key in ("row_map", "seg_off", "seg_count", "xp"):
-            np.testing.assert_array_equal(got[key], want[key], err_msg=key)
-        for key in ("counts", "kept", "num_dropped"):
-            np.testing.assert_array_equal(got["stats"][key], want["stats"][key], err_msg=key)
+        ref = orc.dispatch(idx, N, cap, 128)
+        for call in range(2):
+            got = _static_dispatch(cfg, xt, it)
+            assert got["flags"] == 0 and want["flags"] == 0, call
+            for key in ("row_map", "seg_off", "seg_count", "xp"):
+                np.testing.assert_array_equal(got[key], want[key], err_msg=f"{key}, call {call}")
+            for key in ("counts", "kept", "num_dropped"):
+                np.testing.assert_array_equal(got["stats"][key], want["stats"][key],
+                                              err_msg=f"{key}, call {call}")
+            # the oracle's capacity clip and permutation, compared directly
+            np.testing.assert_array_equal(got["row_map"], ref.row_map, err_msg=f"oracle row_map, call {call}")
+            np.testing.assert_array_equal(got["seg_off"], ref.seg_off, err_msg=f"oracle seg_off, call {call}")
+            np.testing.assert_array_equal(got["seg_count"], ref.kept, err_msg=f"oracle kept, call {call}")
+            np.testing.assert_array_equal(got["stats"]["counts"], ref.counts)
+            assert int(got["stats"]["num_dropped"][0]) == ref.num_dropped
+            t_of, j_of = np.nonzero(ref.row_map >= 0)
+            np.testing.assert_array_equal(got["xp"][ref.row_map[t_of, j_of]], x[t_of],
+                                          err_msg=f"permuted rows, call {call}")
 
 
 def test_static_dispatch_rejects_batches_beyond_its_scratch():
