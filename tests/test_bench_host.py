@@ -80,6 +80,7 @@ def test_reference_arm_json_line():
     assert line["value"] > 0 and line["unit"] == "tokens/s" and line["higher_is_better"] is True
     assert line["config"]["workload"] == "tiny-fp32"
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["cpu_baseline"]["cpu_model"]
     assert line["cpu_baseline"]["value"] == line["value"]
     assert line["e2e"] == {"value": line["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
@@ -108,3 +109,27 @@ def test_workload_config_names_the_workload_and_its_sizes():
     assert (c["T"], c["d"], c["N"], c["k"], c["f"]) == (8192, 4096, 128, 8, 1536)
     assert c["capacity"] == 512 and c["act_dtype"] == "bf16" and c["router_dtype"] == "f32"
     assert "model" not in c
+
+
+def test_tensor_peak_follows_the_length_of_the_timed_region():
+    peaks = {"hbm_gbs": 6538.0, "bf16_tflops": 1674.7, "bf16_tflops_sustained": 1364.1}
+    p, key, why = bench.choose_tensor_peak(peaks, 0.042)     # 20 layer steps: a burst
+    assert (p, key) == (1674.7, "bf16_tflops") and "burst" in why
+    p, key, why = bench.choose_tensor_peak(peaks, bench.SUSTAINED_REGION_S)
+    assert (p, key) == (1364.1, "bf16_tflops_sustained") and "sustained" in why
+    p, key, _ = bench.choose_tensor_peak(peaks, 12.0)
+    assert key == "bf16_tflops_sustained"
+
+
+def test_cpu_model_is_named():
+    m = bench.cpu_model()
+    assert isinstance(m, str) and m and m != "unknown"
+
+
+def test_cpu_baseline_covers_the_whole_small_layer():
+    from expert_router_gemm_b200 import configs, synth
+    w = configs.get("tiny")
+    e = bench.cpu_baseline_entry(w, synth.make_inputs(w))
+    assert e["kind"] == "oracle" and e["extrapolated"] is False and e["value"] > 0
+    assert e["cores"] >= 1 and e["cpu_model"] and "whole layer" in e["sample"]
+    assert "tiny-fp32" in bench.FULL_LAYER_WORKLOADS and "qwen3-moe-shaped" in bench.FULL_LAYER_WORKLOADS
