@@ -25,7 +25,7 @@ from expert_router_gemm_b200 import moe  # noqa: E402
 from tests import gpu_util as gu  # noqa: E402
 from tests.layer_check import compare_layer, oracle_routing  # noqa: E402
 
-SAMPLE = 256
+SAMPLE = 1024   # tokens of each full-size layer whose outputs the oracle recomputes
 
 
 @pytest.mark.parametrize("name", ["tiny-fp32", "mixtral-8x7b-shaped", "qwen3-moe-shaped",
