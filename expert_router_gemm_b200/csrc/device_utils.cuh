@@ -76,18 +76,38 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// The same with acquire at cluster scope: for a barrier that the other CTA of a
+// pair arrives on after writing its own shared memory.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait until the phase with parity `parity` of `bar` has completed.  Gives up
-// (returns false) when *abort becomes non-zero or after kWaitLimitNs; a timeout
+// (returns false) when *abort becomes non-zero or after limit_ns; a timeout
 // raises `timeout_bit` in *gflags and sets *abort so the other roles stop too.
+// CLUSTER: acquire at cluster scope.
+template <bool CLUSTER = false>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile uint32_t* abort,
-                                          uint32_t* gflags, uint32_t timeout_bit) {
-  if (mbar_try_wait(bar, parity)) return true;
+                                          uint32_t* gflags, uint32_t timeout_bit,
+                                          uint64_t limit_ns = kWaitLimitNs) {
+  auto try_once = [&] { return CLUSTER ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
+  if (try_once()) return true;
   const uint64_t t0 = global_timer_ns();
+  // the clock is read every 32nd poll under the default bound, every poll under a shorter one
+  const uint32_t cadence = limit_ns < kWaitLimitNs ? 0u : 31u;
   for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 31u) == 0) {
+    if (try_once()) return true;
+    if ((i & cadence) == 0) {
       if (abort != nullptr && *abort != 0u) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
+      if (global_timer_ns() - t0 > limit_ns) {
         atomicOr(gflags, timeout_bit);
         if (abort != nullptr) *abort = 1u;
         return false;
@@ -95,6 +115,22 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     }
   }
 }
+
+// ------------------------------------------------------------------ cp.async
+// 16-byte copy global -> shared through L2 only.  The shared-memory write is a
+// generic-proxy write of this thread: before the tensor cores (async proxy)
+// read it, wait for it (cp_async_wait), fence.proxy.async, then synchronise.
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+// One arrival on `bar` (this CTA's shared memory), made when every cp.async this
+// thread has issued so far has completed; the barrier's expected count includes
+// it (noinc).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+// wait until every cp.async this thread has issued has completed
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 // ------------------------------------------------------------------ TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
@@ -193,6 +229,27 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap
       "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+      : "memory");
+}
+// Row-gather tile load: four rows r0..r3 of a 2-D tensor (columns x .. x+box-1,
+// the tensor map's box being one row high) land as four consecutive rows at
+// dst, swizzled like rows of a tiled box at the same shared-memory address.
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map, uint32_t bar, int32_t x, int32_t r0,
+                                            int32_t r1, int32_t r2, int32_t r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+      : "memory");
+}
+// The same with completion counted on `bar`, which may be the barrier of either
+// CTA of the pair.
+__device__ __forceinline__ void tma_gather4_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar, int32_t x,
+                                                 int32_t r0, int32_t r1, int32_t r2, int32_t r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
       : "memory");
 }
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {

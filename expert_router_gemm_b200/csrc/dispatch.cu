@@ -16,7 +16,9 @@
 //               kept = min(count, C) and the aligned segment offsets;
 //   3. scatter: rank of (t, e) = base[block][e] + popcount of the mask bits below
 //               t, kept iff rank < C; row = seg_off[e] + rank; one warp per token
-//               copies x[t] with 16-byte vectors to each of its kept rows.
+//               copies x[t] with 16-byte vectors to each of its kept rows.  In the
+//               layer pass the rows are not copied: an index kernel records the
+//               token of every kept row and the grouped GEMM gathers from x.
 #include <cuda_fp8.h>
 
 #include "device_utils.cuh"
@@ -195,6 +197,39 @@ __global__ void __launch_bounds__(kScatterThreads) dispatch_scatter_kernel(const
   }
 }
 
+// The permutation as an index only: each kept slot's row gets its token number
+// (row_token[row] = t) and nothing is copied; the grouped GEMM then gathers the
+// token rows of x itself.  One block per 32-token mask block, one thread per
+// (token, slot).
+__global__ void __launch_bounds__(kMaskThreads) dispatch_index_kernel(const DispatchArgs a) {
+  __shared__ uint32_t m[256];
+  __shared__ int base_s[256];
+  __shared__ int off_s[256];
+  const int N = a.N, k = a.k;
+  const int64_t blk = blockIdx.x;
+  for (int e = threadIdx.x; e < N; e += kMaskThreads) {
+    m[e] = a.mask[blk * N + e];
+    base_s[e] = a.base[blk * N + e];
+    off_s[e] = a.seg_off[e];
+  }
+  __syncthreads();
+  const int64_t t0 = blk * kDispatchTokens;
+  for (int s = threadIdx.x; s < kDispatchTokens * k; s += kMaskThreads) {
+    const int pos = s / k, j = s % k;
+    const int64_t t = t0 + pos;
+    if (t >= a.T) break;
+    const int32_t* row = a.topk_idx + t * k;
+    const int e = row[j];
+    int r = -1;
+    if (slot_valid(row, j, e, N)) {
+      const int rank = base_s[e] + __popc(m[e] & ((1u << pos) - 1u));
+      if (rank < a.capacity) r = off_s[e] + rank;
+    }
+    a.row_map[t * k + j] = r;
+    if (r >= 0) a.row_token[r] = static_cast<int32_t>(t);
+  }
+}
+
 // The same permutation with the rows quantized on the way: block-scaled FP8
 // (E4M3 codes, one E8M0 scale per 32 values of d, the smallest power of two
 // that keeps the block within 448).  A warp reads its bf16 token row once;
@@ -282,7 +317,9 @@ cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t s) {
   dispatch_mask_kernel<<<blocks, kMaskThreads, 0, s>>>(a);
   dispatch_scan_kernel<<<(a.N + 31) / 32, 1024, 0, s>>>(a, blocks);
   const unsigned sblocks = static_cast<unsigned>((a.T + kScatterTokens - 1) / kScatterTokens);
-  if (a.xp_sf != nullptr)
+  if (a.row_token != nullptr)
+    dispatch_index_kernel<<<blocks, kMaskThreads, 0, s>>>(a);
+  else if (a.xp_sf != nullptr)
     dispatch_scatter_mx_kernel<<<sblocks, kScatterThreads, 0, s>>>(a);
   else
     dispatch_scatter_kernel<<<sblocks, kScatterThreads, 0, s>>>(a);

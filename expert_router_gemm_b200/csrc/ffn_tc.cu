@@ -7,9 +7,14 @@
 //   GEMM2 (PLAIN):  out[r] = h[r] W2_e                       -> bf16
 //
 // Per CTA (one per SM, 192 threads):
-//   warp 0 lane 0   TMA producer: A slab 128 x 64 (K-major rows of the permuted
+//   warp 0          TMA producer: A slab 128 x 64 (K-major rows of the permuted
 //                   activations) and B slab 64 x (256/CG) (rows of the row-major
 //                   weight, i.e. MN-major), 128-byte swizzle, multi-stage ring.
+//                   Lane 0 loads a permuted-row A slab as one tile.  Given a
+//                   row -> token table instead (a layer pass whose dispatch
+//                   copies no rows, MOE_GATHER=lsu|tma), the 32 lanes gather the
+//                   slab's 128 token rows straight from x, as 16-byte cp.async
+//                   copies or four rows per tile::gather4 load.
 //   warp 1          allocates 512 TMEM columns (two accumulators, so the
 //                   epilogue of tile i overlaps the main loop of tile i+1);
 //                   lane 0 issues tcgen05.mma kind::f16, K=16, fp32 accumulator.
@@ -35,6 +40,7 @@
 // MOE_FLAG_WAIT_TIMEOUT, waits (bounded) for its own copies and MMAs in flight,
 // frees its TMEM and returns.
 #include <algorithm>
+#include <atomic>
 #include <cstdlib>
 #include <mutex>
 
@@ -55,6 +61,7 @@ constexpr int kTmemCols = 2 * MMA_N;
 constexpr int kMaxGroups = 256;
 
 enum { MODE_SWIGLU = 0, MODE_PLAIN = 1 };
+enum { A_TILE = 0, A_GATHER_TMA = 1, A_GATHER_LSU = 2 };
 
 template <int CG>
 struct Cfg {
@@ -74,16 +81,24 @@ struct TcParams {
   int64_t max_rows;          // rows of the A and output buffers
   int K;                     // reduction length (multiple of 64)
   int n_out;                 // output columns
+  const int32_t* a_token;    // non-null: A row r (absolute) is row a_token[r] of a_src [a_token_rows, K]
+                             // (rows past a group's count read row 0; indices outside a_src too)
+  const void* a_src;         //   the gathered tensor (bf16), also under tmA (one-row boxes)
+  int a_token_rows;
+  int a_gather;              //   A_GATHER_TMA or A_GATHER_LSU
   uint16_t* out;             // [max_rows, n_out] bf16
   uint16_t* save_g;          // SwiGLU, optional: gate and up pre-activations [max_rows, n_out]
   uint16_t* save_u;          //   (bf16), kept for the backward pass
   int v8;                    // output rows start on 32-byte boundaries: 32-byte stores
+  uint64_t wait_ns;          // bound of the pipeline waits (those that also watch the abort flag);
+                             // the waits that drain copies and MMAs in flight keep kWaitLimitNs
   uint32_t* flags;
 };
 
 struct TcTail {
   uint64_t full[8];
   uint64_t empty[8];
+  uint64_t afull[8];   // odd CTA of a pair: its cp.async A slab of the stage has landed
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t drain;
@@ -202,9 +217,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int KB = p.K / BK;
 
   if (warp == 0 && lane == 0) {
+    // full: the expect-tx arrival; with a cp.async slab also one arrival per
+    // producer lane, and on a pair one relayed arrival for the odd CTA's slab
+    // (counted on afull, 32 lanes, in the odd CTA)
+    const bool lsu = p.a_token != nullptr && p.a_gather == A_GATHER_LSU;
+    const uint32_t full_count = lsu ? (CG == 2 ? 34u : 33u) : 1u;
     for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(smem_addr(&tl.full[s]), 1);
+      mbar_init(smem_addr(&tl.full[s]), full_count);
       mbar_init(smem_addr(&tl.empty[s]), 1);
+      mbar_init(smem_addr(&tl.afull[s]), 32);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(smem_addr(&tl.tfull[a]), 1);
@@ -262,16 +283,43 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile uint32_t* abort = &tl.abort;
 
   if (warp == 0) {
-    if (lane == 0) {
-      // ---------------------------------------------------------------- producer
+    // ------------------------------------------------------------------ producer
+    // A arrives one of three ways: a slab of permuted rows as one TMA tile
+    // (lane 0); or, with a row -> token table, the slab's 128 token rows of x
+    // gathered by the whole warp, either as tile::gather4 TMA loads (lane i:
+    // rows 4i..4i+3) or as 16-byte cp.async copies into the swizzled slab (lane
+    // i: chunk i % 8 of rows i / 8, i / 8 + 4, ...), each lane arriving on the
+    // stage's barrier when its copies have landed.  Lane 0 waits for free
+    // stages, posts the expected TMA bytes and loads B.
+    const int amode = p.a_token == nullptr ? A_TILE : p.a_gather;
+    if (amode != A_TILE || lane == 0) {
       uint32_t stage = 0, phase = 0, issued = 0, last_par = 0;
       bool ok = true;
       for (int t = unit; ok && t < total; t += n_units) {
         const Tile tile = decode_tile(tl, p, G, BN, C::TILE_M, t);
-        const int a_row = group_rows(p, tile.g).x + tile.m0 + static_cast<int>(rank) * BM;
+        const int2 gr = group_rows(p, tile.g);
+        const int a_row = gr.x + tile.m0 + static_cast<int>(rank) * BM;
         const int b_row = tile.g * p.K;
+        const int r_base = tile.m0 + static_cast<int>(rank) * BM;   // this CTA's first row in the group
+        // token of row r of this CTA's slab (rows past the group's count read row 0)
+        auto token_of = [&](int r) {
+          const int v = r_base + r < gr.y ? __ldg(p.a_token + gr.x + r_base + r) : 0;
+          return static_cast<unsigned>(v) < static_cast<unsigned>(p.a_token_rows) ? v : 0;
+        };
+        int tok4[4] = {0, 0, 0, 0};
+        int tok32[32];
+        if (amode == A_GATHER_TMA) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) tok4[i] = token_of(4 * lane + i);
+        } else if (amode == A_GATHER_LSU) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) tok32[i] = token_of(4 * i + (lane >> 3));
+        }
         for (int kb = 0; kb < KB; ++kb) {
-          if (!mbar_wait(smem_addr(&tl.empty[stage]), phase ^ 1u, abort, p.flags, kFlagTimeout)) {
+          bool free_stage = true;
+          if (lane == 0) free_stage = mbar_wait(smem_addr(&tl.empty[stage]), phase ^ 1u, abort, p.flags, kFlagTimeout, p.wait_ns);
+          if (amode != A_TILE) free_stage = __shfl_sync(0xffffffffu, free_stage ? 1 : 0, 0) != 0;
+          if (!free_stage) {
             ok = false;
             break;
           }
@@ -279,22 +327,45 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t a_dst = smem_addr(sA + stage * A_BYTES);
           const uint32_t b_dst = smem_addr(sB + stage * C::B_BYTES);
           const int ky = b_row + kb * BK;
-          if (CG == 1) {
-            mbar_arrive_expect_tx(fb_local, C::STAGE_BYTES);
-            tma_load_2d(a_dst, &tmA, fb_local, kb * BK, a_row);
-#pragma unroll
-            for (int i = 0; i < Cfg<CG>::B_CHUNKS; ++i)
-              tma_load_2d(b_dst + i * B_CHUNK, b_box_map<MODE, CG>(&tmB0, &tmB1, rank, i), fb_local,
-                          b_box_col<MODE, CG>(tile.n0, rank, i), ky);
+          // both CTAs' TMA bytes of a pair complete on the even CTA's barrier
+          const uint32_t fb = (CG == 1 || rank == 0) ? fb_local : mapa_shared(fb_local, 0);
+          const uint32_t tx = static_cast<uint32_t>((amode == A_GATHER_LSU ? 0 : A_BYTES) + C::B_BYTES);
+          if (lane == 0 && (CG == 1 || rank == 0)) mbar_arrive_expect_tx(fb_local, CG * tx);
+          if (amode == A_TILE) {
+            if (CG == 1)
+              tma_load_2d(a_dst, &tmA, fb, kb * BK, a_row);
+            else
+              tma_load_2d_pair(a_dst, &tmA, fb, kb * BK, a_row);
+          } else if (amode == A_GATHER_TMA) {
+            __syncwarp();
+            if (CG == 1)
+              tma_gather4(a_dst + lane * 4 * 128, &tmA, fb, kb * BK, tok4[0], tok4[1], tok4[2], tok4[3]);
+            else
+              tma_gather4_pair(a_dst + lane * 4 * 128, &tmA, fb, kb * BK, tok4[0], tok4[1], tok4[2], tok4[3]);
           } else {
-            // both CTAs' bytes complete on the even CTA's barrier
-            const uint32_t fb = rank == 0 ? fb_local : mapa_shared(fb_local, 0);
-            if (rank == 0) mbar_arrive_expect_tx(fb_local, 2 * C::STAGE_BYTES);
-            tma_load_2d_pair(a_dst, &tmA, fb, kb * BK, a_row);
+            // chunk c of row r lands at 16 * (c ^ (r % 8)) in the row's 128 bytes:
+            // the 128-byte swizzle of a 1024-byte aligned slab
+            const int c = lane & 7;
+            const uint16_t* xs = static_cast<const uint16_t*>(p.a_src) + kb * BK + c * 8;
 #pragma unroll
-            for (int i = 0; i < Cfg<CG>::B_CHUNKS; ++i)
-              tma_load_2d_pair(b_dst + i * B_CHUNK, b_box_map<MODE, CG>(&tmB0, &tmB1, rank, i), fb,
-                               b_box_col<MODE, CG>(tile.n0, rank, i), ky);
+            for (int i = 0; i < 32; ++i) {
+              const int r = 4 * i + (lane >> 3);
+              cp_async_16(a_dst + r * 128 + ((c ^ (r & 7)) << 4), xs + static_cast<int64_t>(tok32[i]) * p.K);
+            }
+            // the odd CTA of a pair counts its slab on its own barrier; its MMA
+            // warp relays the completion to the even CTA
+            cp_async_arrive_noinc(CG == 2 && rank != 0 ? smem_addr(&tl.afull[stage]) : fb_local);
+          }
+          if (lane == 0) {
+#pragma unroll
+            for (int i = 0; i < Cfg<CG>::B_CHUNKS; ++i) {
+              if (CG == 1)
+                tma_load_2d(b_dst + i * B_CHUNK, b_box_map<MODE, CG>(&tmB0, &tmB1, rank, i), fb,
+                            b_box_col<MODE, CG>(tile.n0, rank, i), ky);
+              else
+                tma_load_2d_pair(b_dst + i * B_CHUNK, b_box_map<MODE, CG>(&tmB0, &tmB1, rank, i), fb,
+                                 b_box_col<MODE, CG>(tile.n0, rank, i), ky);
+            }
           }
           issued |= 1u << stage;
           last_par = (last_par & ~(1u << stage)) | (phase << stage);
@@ -304,32 +375,62 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      // Every load issued by this thread has landed before the CTA may exit:
-      // the even CTA sees its barrier complete; the odd CTA sees the MMA that
+      // every copy into shared memory lands before the CTA may exit
+      if (amode == A_GATHER_LSU) cp_async_wait_all();
+      // Every TMA load issued by this warp has landed before the CTA may exit
+      // (all lanes' loads of a stage complete on the stage's one barrier): the
+      // even CTA sees its barrier complete; the odd CTA sees the MMA that
       // consumed the load release the stage.
-      for (int s = 0; s < C::STAGES; ++s)
-        if ((issued >> s) & 1u) {
-          if (rank == 0)
-            mbar_wait(smem_addr(&tl.full[s]), (last_par >> s) & 1u, nullptr, p.flags, kFlagTimeout);
-          else
-            mbar_wait(smem_addr(&tl.empty[s]), (last_par >> s) & 1u, nullptr, p.flags, kFlagTimeout);
-        }
+      if (lane == 0) {
+        for (int s = 0; s < C::STAGES; ++s)
+          if ((issued >> s) & 1u) {
+            if (rank == 0)
+              mbar_wait(smem_addr(&tl.full[s]), (last_par >> s) & 1u, nullptr, p.flags, kFlagTimeout);
+            else
+              mbar_wait(smem_addr(&tl.empty[s]), (last_par >> s) & 1u, nullptr, p.flags, kFlagTimeout);
+          }
+      }
     }
   } else if (warp == 1) {
-    if (lane == 0 && rank == 0) {
+    const bool lsu_a = p.a_token != nullptr && p.a_gather == A_GATHER_LSU;
+    if (CG == 2 && lane == 0 && rank != 0 && lsu_a) {
+      // ------------------------------------------------------ relay (odd CTA)
+      // The odd CTA's producer lanes count each stage's cp.async slab on afull;
+      // this thread forwards it, in the producer's stage order, as one arrival
+      // on the even CTA's full barrier (cp.async completion can only signal a
+      // barrier of the issuing CTA).
+      uint32_t stage = 0, phase = 0;
+      bool ok = true;
+      for (int t = unit; ok && t < total; t += n_units) {
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(smem_addr(&tl.afull[stage]), phase, abort, p.flags, kFlagTimeout, p.wait_ns)) {
+            ok = false;
+            break;
+          }
+          fence_proxy_async_smem();
+          mbar_arrive_cluster(mapa_shared(smem_addr(&tl.full[stage]), 0));
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    } else if (lane == 0 && rank == 0) {
       // ---------------------------------------------------------------- MMA issuer
       uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
       bool ok = true, issued_any = false;
       for (int t = unit; ok && t < total; t += n_units) {
-        if (!mbar_wait(smem_addr(&tl.tempty[acc]), acc_phase ^ 1u, abort, p.flags, kFlagTimeout)) break;
+        if (!mbar_wait(smem_addr(&tl.tempty[acc]), acc_phase ^ 1u, abort, p.flags, kFlagTimeout, p.wait_ns)) break;
         tc_fence_after();
         issued_any = true;
         const uint32_t d_tmem = tmem_base + acc * MMA_N;
         for (int kb = 0; kb < KB; ++kb) {
-          if (!mbar_wait(smem_addr(&tl.full[stage]), phase, abort, p.flags, kFlagTimeout)) {
+          // cluster scope: the odd CTA's cp.async slab is announced by its own arrival
+          if (!mbar_wait<CG == 2>(smem_addr(&tl.full[stage]), phase, abort, p.flags, kFlagTimeout, p.wait_ns)) {
             ok = false;
             break;
           }
+          if (lsu_a) fence_proxy_async_smem();   // cp.async (generic proxy) writes -> MMA operand reads
           tc_fence_after();
           const uint32_t a_addr = smem_addr(sA + stage * A_BYTES);
           const uint32_t b_addr = smem_addr(sB + stage * C::B_BYTES);
@@ -382,7 +483,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = unit; t < total; t += n_units) {
       const Tile tile = decode_tile(tl, p, G, BN, C::TILE_M, t);
       const int2 gr = group_rows(p, tile.g);
-      if (!mbar_wait(smem_addr(&tl.tfull[acc]), acc_phase, abort, p.flags, kFlagTimeout)) break;
+      if (!mbar_wait(smem_addr(&tl.tfull[acc]), acc_phase, abort, p.flags, kFlagTimeout, p.wait_ns)) break;
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * MMA_N;
       const int row = tile.m0 + r_in_tile;
@@ -513,6 +614,31 @@ bool rows_32b_aligned(const uint16_t* p, int n) {
   return (reinterpret_cast<uintptr_t>(p) & 31u) == 0 && n % 16 == 0;
 }
 
+// Whether the layer pass gathers GEMM1's token rows from x instead of reading
+// the permuted copy, and how: MOE_GATHER=tma (tile::gather4 TMA loads) or lsu
+// (cp.async copies).  Unset or anything else: no gather.  Both gathers measured
+// slower than the copy on the Qwen3-shaped layer (GEMM1 2.29 ms with cp.async,
+// about 3.5 ms with gather4, against 1.26 ms reading the permuted rows as TMA
+// tiles, under ncu), so the copy is the default.
+int gather_mode() {
+  static int mode = [] {
+    const char* v = std::getenv("MOE_GATHER");
+    if (v == nullptr) return static_cast<int>(A_TILE);
+    if (v[0] == 't') return static_cast<int>(A_GATHER_TMA);
+    if (v[0] == 'l') return static_cast<int>(A_GATHER_LSU);
+    return static_cast<int>(A_TILE);
+  }();
+  return mode;
+}
+
+// Bound of the grouped GEMM's pipeline waits (moe_set_wait_limit_ns); 0 = kWaitLimitNs.
+std::atomic<uint64_t> g_pipeline_wait_ns{0};
+
+uint64_t pipeline_wait_ns() {
+  const uint64_t v = g_pipeline_wait_ns.load(std::memory_order_relaxed);
+  return v == 0 ? kWaitLimitNs : v;
+}
+
 int choose_cta_group(const FfnArgs& a) {
   static int forced = [] {
     const char* v = std::getenv("MOE_FFN_CTA_GROUP");
@@ -536,8 +662,15 @@ cudaError_t launch_pair(const FfnArgs& a, const CUtensorMap& mA1, const CUtensor
   p.save_u = static_cast<uint16_t*>(a.save_u);
   p.v8 = rows_32b_aligned(p.out, p.n_out) && rows_32b_aligned(p.save_g, p.n_out) &&
          rows_32b_aligned(p.save_u, p.n_out);
+  p.a_token = a.a_token;
+  p.a_src = a.a;
+  p.a_token_rows = static_cast<int>(a.a_token_rows);
+  p.a_gather = gather_mode();
   cudaError_t e = launch_gemm<MODE_SWIGLU, CG>(mA1, mW1, mW3, p, m_bound * ((a.f + 127) / 128), s);
   if (e != cudaSuccess) return e;
+  p.a_token = nullptr;
+  p.a_src = nullptr;
+  p.a_token_rows = 0;
   p.save_g = p.save_u = nullptr;
   p.K = a.f;
   p.n_out = a.d;
@@ -548,17 +681,26 @@ cudaError_t launch_pair(const FfnArgs& a, const CUtensorMap& mA1, const CUtensor
 
 }  // namespace
 
+void set_pipeline_wait_ns(uint64_t ns) { g_pipeline_wait_ns.store(ns, std::memory_order_relaxed); }
+
+bool layer_gathers_rows() { return gather_mode() != A_TILE; }
+
 cudaError_t launch_ffn_bf16(const FfnArgs& a, cudaStream_t s) {
   if (a.max_rows <= 0 || a.G <= 0) return cudaSuccess;
   const bool dense = a.seg_off == nullptr;
   const uint64_t G = dense ? 1 : static_cast<uint64_t>(a.G);
   CUtensorMap mA1, mW1, mW3, mA2, mW2;
-  if (!make_tma_2d_bf16(&mA1, a.a, a.d, a.max_rows, BK, BM) ||
+  // GEMM1's A: the permuted rows as 128-row tiles, or x one row per box for the
+  // row gather (the gather load's box is one row high)
+  const bool gather = a.a_token != nullptr;
+  if (gather && (a.a_token_rows <= 0 || a.a_token_rows >= (int64_t(1) << 31))) return cudaErrorInvalidValue;
+  if (!make_tma_2d_bf16(&mA1, a.a, a.d, gather ? a.a_token_rows : a.max_rows, BK, gather ? 1 : BM) ||
       !make_tma_2d_bf16(&mW1, a.w1, a.f, G * a.d, 64, BK) || !make_tma_2d_bf16(&mW3, a.w3, a.f, G * a.d, 64, BK) ||
       !make_tma_2d_bf16(&mA2, a.h, a.f, a.max_rows, BK, BM) || !make_tma_2d_bf16(&mW2, a.w2, a.d, G * a.f, 64, BK))
     return cudaErrorInvalidValue;
 
   TcParams p{};
+  p.wait_ns = pipeline_wait_ns();
   p.seg_off = a.seg_off;
   p.seg_count = a.seg_count;
   p.G = static_cast<int>(G);

@@ -93,6 +93,8 @@ struct DispatchArgs {
   void* xp;
   uint8_t* xp_sf;           // non-null: xp receives block-scaled FP8 codes and these
                             // scale bytes (tile-interleaved, d/32 per row)
+  int32_t* row_token;       // non-null: no rows are copied; row_token[row_map[t][j]] = t instead
+                            // (the grouped GEMM then gathers its A rows from x)
   uint32_t* mask;           // [blocks, N] scratch
   int32_t* base;            // [blocks, N] scratch
   int32_t* counts;          // [N] scratch
@@ -127,7 +129,10 @@ struct FfnArgs {
   int d, f;
   const int32_t* seg_off;
   const int32_t* seg_count;
-  const void* a;            // [rows, d]
+  const void* a;            // [rows, d], or x [a_token_rows, d] when a_token is set
+  const int32_t* a_token;   // bf16 path, optional: row r of a group reads row a_token[r] of `a`
+                            // (GEMM1 gathers the token rows; entries past a group's count unused)
+  int64_t a_token_rows;     // rows of `a` when a_token is set
   const void* w1;           // [G][d][f]
   const void* w3;           // [G][d][f]
   const void* w2;           // [G][f][d]
@@ -138,6 +143,11 @@ struct FfnArgs {
   uint32_t* flags;
 };
 cudaError_t launch_ffn_bf16(const FfnArgs& a, cudaStream_t s);
+// Bound of the bf16 grouped GEMM's pipeline waits for later launches (0: the default).
+void set_pipeline_wait_ns(uint64_t ns);
+// The bf16 layer pass lets GEMM1 gather token rows from x (MOE_GATHER=lsu|tma)
+// instead of copying them into the permuted buffer first.
+bool layer_gathers_rows();
 cudaError_t launch_ffn_f32(const FfnArgs& a, cudaStream_t s);
 
 // Block-scaled FP8 (E4M3 codes, one E8M0 scale byte per 32 values along K,

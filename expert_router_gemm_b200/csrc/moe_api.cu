@@ -126,7 +126,7 @@ moe_status_t derive(const moe_config_t* cfg, Dims* D) {
 // of h, and x8 / x8sf / h8sf the FP8 rows and the two scale buffers.
 struct Layout {
   size_t flags, rticket, rcnt, rz, zero_end, rzl, rsplit, rlogits, dmask, dbase, dcounts, dticket, op_end;
-  size_t idx, w, row_map, seg_off, seg_count, xp, h, hs, sh, x8, x8sf, h8sf, layer_end;
+  size_t idx, w, row_map, seg_off, seg_count, rtok, xp, h, hs, sh, x8, x8sf, h8sf, layer_end;
 };
 
 Layout layout(const Dims& D) {
@@ -158,7 +158,8 @@ Layout layout(const Dims& D) {
   L.row_map = take(sizeof(int32_t) * D.T * D.k);
   L.seg_off = take(sizeof(int32_t) * (D.N + 1));
   L.seg_count = take(sizeof(int32_t) * D.N);
-  L.xp = take(static_cast<size_t>(D.elem) * D.max_rows * D.d);  // permuted rows, then expert outputs
+  L.rtok = take(sizeof(int32_t) * D.max_rows);                   // row -> token (bf16 layer: GEMM1 gathers)
+  L.xp = take(static_cast<size_t>(D.elem) * D.max_rows * D.d);  // permuted rows / expert outputs
   L.h = take(static_cast<size_t>(D.elem) * D.max_rows * D.f);
   L.hs = take(static_cast<size_t>(D.elem) * (D.fs ? D.T * D.fs : 0));
   L.sh = take(static_cast<size_t>(D.elem) * (D.fs ? D.T * D.d : 0));
@@ -287,7 +288,7 @@ moe_status_t do_route(const Dims& D, const void* x, const float* w_router, const
 
 moe_status_t do_dispatch(const Dims& D, const void* x, const int32_t* topk_idx, int32_t* row_map,
                          int32_t* seg_off, int32_t* seg_count, void* xp, uint8_t* xp_sf,
-                         const moe_stats_t* stats, void* ws, cudaStream_t st) {
+                         const moe_stats_t* stats, void* ws, cudaStream_t st, int32_t* row_token = nullptr) {
   const Layout L = layout(D);
   if (D.T == 0) {
     cudaError_t e = cudaMemsetAsync(seg_off, 0, sizeof(int32_t) * (D.N + 1), st);
@@ -314,6 +315,7 @@ moe_status_t do_dispatch(const Dims& D, const void* x, const int32_t* topk_idx, 
   a.seg_count = seg_count;
   a.xp = xp;
   a.xp_sf = xp_sf;
+  a.row_token = row_token;
   a.mask = at<uint32_t*>(ws, L.dmask);
   a.base = at<int32_t*>(ws, L.dbase);
   a.counts = at<int32_t*>(ws, L.dcounts);
@@ -325,7 +327,8 @@ moe_status_t do_dispatch(const Dims& D, const void* x, const int32_t* topk_idx, 
 
 moe_status_t do_ffn(const Dims& D, const void* a_rows, const int32_t* seg_off, const int32_t* seg_count,
                     const void* w1, const void* w3, const void* w2, int f, bool dense, void* h, void* out,
-                    void* ws, cudaStream_t st, void* save_g = nullptr, void* save_u = nullptr) {
+                    void* ws, cudaStream_t st, void* save_g = nullptr, void* save_u = nullptr,
+                    const int32_t* a_token = nullptr) {
   const Layout L = layout(D);
   FfnArgs a{};
   a.G = dense ? 1 : D.N;
@@ -338,6 +341,8 @@ moe_status_t do_ffn(const Dims& D, const void* a_rows, const int32_t* seg_off, c
   a.seg_off = dense ? nullptr : seg_off;
   a.seg_count = dense ? nullptr : seg_count;
   a.a = a_rows;
+  a.a_token = a_token;
+  a.a_token_rows = a_token != nullptr ? D.T : 0;
   a.w1 = w1;
   a.w3 = w3;
   a.w2 = w2;
@@ -615,7 +620,7 @@ moe_status_t moe_layer_fwd(const moe_config_t* cfg, const moe_weights_t* weights
   int32_t* seg_count = at<int32_t*>(ws, L.seg_count);
   void* xp = at<void*>(ws, L.xp);
   void* h = at<void*>(ws, L.h);
-  void* out_rows = xp;  // the permuted rows are dead once GEMM1 has read them
+  void* out_rows = xp;  // expert outputs: the permuted rows are dead once GEMM1 has read them
   void* shared_out = D.fs ? at<void*>(ws, L.sh) : nullptr;
 
   if ((s = do_route(D, x, weights->w_router, weights->router_bias, weights->selection_bias, nullptr, nullptr, idx, w,
@@ -627,6 +632,15 @@ moe_status_t moe_layer_fwd(const moe_config_t* cfg, const moe_weights_t* weights
     if ((s = do_dispatch(D, x, idx, row_map, seg_off, seg_count, x8, x8sf, stats, ws, st)) != MOE_OK) return s;
     if ((s = do_ffn_mx(D, x8, x8sf, seg_off, seg_count, weights, h, at<void*>(ws, L.h8sf), out_rows, ws, st)) !=
         MOE_OK)
+      return s;
+  } else if (D.bf16 && layer_gathers_rows()) {
+    // no permuted copy of x: the dispatch records each kept row's token and the
+    // SwiGLU GEMM gathers those rows of x itself
+    int32_t* rtok = at<int32_t*>(ws, L.rtok);
+    if ((s = do_dispatch(D, x, idx, row_map, seg_off, seg_count, nullptr, nullptr, stats, ws, st, rtok)) != MOE_OK)
+      return s;
+    if ((s = do_ffn(D, x, seg_off, seg_count, weights->w1, weights->w3, weights->w2, D.f, false, h, out_rows, ws, st,
+                    nullptr, nullptr, rtok)) != MOE_OK)
       return s;
   } else {
     if ((s = do_dispatch(D, x, idx, row_map, seg_off, seg_count, xp, nullptr, stats, ws, st)) != MOE_OK) return s;
@@ -833,6 +847,12 @@ moe_status_t moe_layer_bwd(const moe_config_t* cfg, const moe_weights_t* weights
   }
   return cuda_status(launch_dx_gather(T, d, k, row_map, static_cast<const uint16_t*>(xp), dxr,
                                       static_cast<const uint16_t*>(dxs), static_cast<uint16_t*>(grads->dx), st));
+}
+
+moe_status_t moe_set_wait_limit_ns(uint64_t ns) {
+  if (ns > 2000000000ull) return MOE_ERR_INVALID_ARG;
+  set_pipeline_wait_ns(ns);
+  return MOE_OK;
 }
 
 moe_status_t moe_read_flags(const void* ws, size_t ws_bytes, uint32_t* flags, moe_stream_t stream) {

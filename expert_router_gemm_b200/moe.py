@@ -88,6 +88,7 @@ _PROTOS = {
     "moe_layer_fwd": (ctypes.c_int, [ctypes.POINTER(moe_config_t), ctypes.POINTER(moe_weights_t),
                                      _P, _P, ctypes.POINTER(moe_stats_t), _P, _SZ, _P]),
     "moe_read_flags": (ctypes.c_int, [_P, _SZ, ctypes.POINTER(ctypes.c_uint32), _P]),
+    "moe_set_wait_limit_ns": (ctypes.c_int, [ctypes.c_uint64]),
     "moe_backward_workspace_size": (ctypes.c_int, [ctypes.POINTER(moe_config_t), ctypes.POINTER(_SZ)]),
     "moe_layer_bwd": (ctypes.c_int, [ctypes.POINTER(moe_config_t), ctypes.POINTER(moe_weights_t), _P, _P,
                                      ctypes.c_float, ctypes.c_float, ctypes.POINTER(moe_grads_t), _P, _SZ,
@@ -318,6 +319,11 @@ def moe_read_flags(ws, stream=None) -> int:
     if st not in (MOE_OK, MOE_ERR_NONFINITE, MOE_ERR_DEVICE):
         _check(st, "moe_read_flags")
     return v.value
+
+
+def moe_set_wait_limit_ns(ns: int) -> None:
+    """Bound of the bf16 grouped GEMM's pipeline waits for later launches (0: the 2 s default)."""
+    _check(_lib.moe_set_wait_limit_ns(int(ns)), "moe_set_wait_limit_ns")
 
 
 def raw_call(name: str, *args) -> int:

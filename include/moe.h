@@ -258,9 +258,10 @@ moe_status_t moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t*
  *  - all calls share the one array and it keeps the last call's contents (each
  *    call rewrites every part it reads).  Calls whose work overlaps on the GPU
  *    (different streams, or several host threads) race on it: order them.
- *  - the first call on a device looks up the array's device address (once per
- *    device, with that device current); make that first call before any stream
- *    capture.
+ *  - every call looks up the array's device address on the current device
+ *    (cudaGetSymbolAddress), so the address stays right after cudaDeviceReset;
+ *    the first call on a device also loads the library's device code there:
+ *    make that first call before any stream capture.
  */
 #define MOE_DISPATCH_STATIC_MAX_CELLS 131072
 #define MOE_DISPATCH_STATIC_SCRATCH_BYTES (2u * 4u * MOE_DISPATCH_STATIC_MAX_CELLS + 2048u)
@@ -403,6 +404,19 @@ moe_status_t moe_backward_workspace_size(const moe_config_t* cfg, size_t* bytes)
 moe_status_t moe_layer_bwd(const moe_config_t* cfg, const moe_weights_t* weights, const void* x,
                            const void* dy, float aux_weight, float z_weight, moe_grads_t* grads,
                            void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * moe_set_wait_limit_ns - failure handling (the pages define no such call):
+ * the time bound of the bf16 grouped GEMM's pipeline waits (a stage's operands,
+ * a free stage, an accumulator) for kernels launched after this call, process
+ * wide.  ns = 0 restores the default of 2 s, within which every legitimate wait
+ * ends; a shorter bound makes those waits run out on purpose, which is how the
+ * timeout path is tested: the kernel then raises MOE_FLAG_WAIT_TIMEOUT, still
+ * waits (with the default bound) for the copies and MMAs it has in flight,
+ * frees its tensor memory and returns, leaving the outputs undefined.
+ * Errors: MOE_ERR_INVALID_ARG for ns above 2 s.
+ */
+moe_status_t moe_set_wait_limit_ns(uint64_t ns);
 
 /*
  * moe_read_flags - wait for `stream`, then copy the workspace's device flags

@@ -229,3 +229,10 @@ def test_mx_entry_validation():
     layer = lambda wt: moe.raw_call("moe_layer_fwd", ctypes.byref(mx), ctypes.byref(wt), 0x1000,  # noqa: E731
                                     0x2000, None, 0x3000, ctypes.c_size_t(1 << 40), None)
     assert layer(w) == INVALID
+
+
+def test_wait_limit_validation():
+    # host only: a bound above the 2 s default is refused, 0 restores the default
+    st = moe.raw_call("moe_set_wait_limit_ns", ctypes.c_uint64(2_000_000_001))
+    assert st == INVALID
+    assert moe.raw_call("moe_set_wait_limit_ns", ctypes.c_uint64(0)) == OK

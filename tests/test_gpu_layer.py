@@ -91,20 +91,27 @@ dl = moe.to_device(inp, moe.config_from_workload(w))
 st = gu.staged_layer(dl)
 assert st["flags"] == 0
 rel, n, flips = compare_layer(inp, w, st["y"], st["idx"], st["row_map"], st["logits"], tol=2e-2)
+y, _, flags = gu.layer_fwd(dl)        # GEMM1 gathers the token rows of x itself
+assert flags == 0
+import numpy as np
+np.testing.assert_array_equal(y, st["y"])
 print("REL", rel)
 """
 
 
-@pytest.mark.parametrize("cta_group", ["1", "2"])
-def test_grouped_gemm_cta_group_variants(cta_group):
+@pytest.mark.parametrize("cta_group,gather", [("1", "lsu"), ("2", "lsu"), ("1", "tma"), ("2", "tma")])
+def test_grouped_gemm_cta_group_variants(cta_group, gather):
     """Both tile shapes of the grouped GEMM (one CTA per 128x256 tile, or CTA
-    pairs per 256x256 tile) on a ragged layer with a shared expert.  The choice
-    is made once per process, so each variant runs in its own process."""
+    pairs per 256x256 tile), each with both ways the layer pass gathers token
+    rows (cp.async copies or tile::gather4 TMA loads), on a ragged layer with a
+    shared expert: the staged path against the oracle, the one-call layer bit
+    for bit against the staged path.  The choices are made once per process, so
+    each variant runs in its own process."""
     import os
     import subprocess
     import sys
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-    env = dict(os.environ, MOE_FFN_CTA_GROUP=cta_group)
+    env = dict(os.environ, MOE_FFN_CTA_GROUP=cta_group, MOE_GATHER=gather)
     r = subprocess.run([sys.executable, "-c", _VARIANT_SCRIPT.format(root=root)], env=env,
                        capture_output=True, text=True, timeout=600)
     assert r.returncode == 0, r.stdout + r.stderr

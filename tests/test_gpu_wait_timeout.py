@@ -1,0 +1,56 @@
+"""The grouped GEMM's wait-timeout path, made to run out without a fault.
+
+Every mbarrier wait in the tcgen05 kernels is bounded.  moe_set_wait_limit_ns
+shortens the bound of the bf16 grouped GEMM's pipeline waits (a stage's
+operands, a free stage, an accumulator) to a few hundred nanoseconds, which
+ordinary loads and MMAs outlast, so those waits give up on a normal small
+layer.  The kernel must then raise MOE_FLAG_WAIT_TIMEOUT (moe_read_flags reports
+MOE_ERR_DEVICE), wait with the full bound for its own copies and MMAs in flight,
+free its tensor memory and return; the CUDA context stays usable, and the next
+call with the default bound is correct.  No wait is left without a bound and
+nothing traps: the failure is a status the host reads."""
+import numpy as np
+import pytest
+import torch
+
+from expert_router_gemm_b200 import synth
+from expert_router_gemm_b200.configs import Workload
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+from expert_router_gemm_b200 import moe  # noqa: E402
+from tests import gpu_util as gu  # noqa: E402
+from tests.layer_check import compare_layer  # noqa: E402
+
+SHORT_NS = 300
+
+
+@pytest.mark.parametrize("w", [
+    Workload("timeout-pairs", T=4096, d=1024, N=8, k=2, f=1024, capacity_factor=1.25),    # CTA pairs
+    Workload("timeout-single", T=2048, d=1024, N=64, k=4, f=512, capacity_factor=1.0),    # single CTAs
+], ids=lambda w: w.name)
+def test_pipeline_wait_timeout_is_reported_and_the_next_call_is_correct(w):
+    inp = synth.make_inputs(w)
+    dl = moe.to_device(inp, moe.config_from_workload(w))
+    cfg = dl.cfg
+    lb, _, _ = moe.moe_workspace_size(cfg)
+    ws = torch.empty(lb, dtype=torch.uint8, device="cuda")
+    y = torch.zeros((w.T, w.d), dtype=moe.act_dtype(cfg), device="cuda")
+    moe.moe_set_wait_limit_ns(SHORT_NS)
+    try:
+        moe.moe_layer_fwd(cfg, dl.weights(), dl.x, y, None, ws)
+        flags = moe.moe_read_flags(ws)          # waits for the stream: the call has returned
+    finally:
+        moe.moe_set_wait_limit_ns(0)
+    assert flags & moe.MOE_FLAG_WAIT_TIMEOUT, f"flags {flags:#x}"
+    assert torch.cuda.synchronize() is None     # no sticky CUDA error
+
+    # default bound again: the same layer is correct and raises nothing
+    staged = gu.staged_layer(dl)
+    y2, _, flags2 = gu.layer_fwd(dl)
+    assert flags2 == 0 and staged["flags"] == 0
+    np.testing.assert_array_equal(y2, staged["y"])
+    compare_layer(inp, w, y2, staged["idx"], staged["row_map"], staged["logits"], tol=2e-2)
