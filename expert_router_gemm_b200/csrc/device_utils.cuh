@@ -283,6 +283,23 @@ __device__ __forceinline__ void tc_commit_pair_both(uint32_t bar) {
       "h"(static_cast<uint16_t>(3))
       : "memory");
 }
+// The same with the pair at cluster ranks (2j, 2j+1) of a larger cluster:
+// cta mask 0b11 << 2j.
+__device__ __forceinline__ void tc_commit_pair_mask(uint32_t bar, uint16_t mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+      "h"(mask)
+      : "memory");
+}
+// 16-byte store into the shared memory of a CTA of the cluster (address from mapa)
+__device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, float c, float d) {
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+// barrier among `count` threads (whole warps) of this CTA on hardware barrier `id`
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
 __device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
                : "memory");

@@ -53,16 +53,22 @@ constexpr int kRouteMinBlockTokens = 16;
 // b[i] += gamma * sign(T*k - N*counts[i]) for i < N (one block).
 cudaError_t launch_bias_update(float* b, const int32_t* counts, int64_t Tk, int N, float gamma, cudaStream_t s);
 
-// Router GEMM on the tensor cores (bf16 x): splits W_r into the three
-// bf16 slabs at `split` (router_split_bytes) and writes fp32 logits (+ bias) to
-// `logits` [T, N]; the softmax / top-k pass then runs in logits mode.
+// Router GEMM on the tensor cores (bf16 x) over the three bf16 parts of W_r
+// ([3][d][router_split_width(N)] bf16, made by launch_router_split): fp32
+// partial sums over up to kRouterMaxPartials K slices, slice z at
+// partials + z * T * N, without the bias; *n_partials receives the number of
+// slices.  `split` is a split made earlier, or (make_split) one is first
+// written to split_buf.  The softmax / top-k pass (launch_route) then runs in
+// logits mode on the partials.
 constexpr int kRouterTcMinExperts = 1;  // every bf16 layer
-// The router GEMM splits K into up to kRouterMaxPartials slices (more CTAs for
-// small T or N); slice z writes partial sums to partials + z * T * N, without
-// the bias.  *n_partials receives the number of slices used.
 constexpr int kRouterMaxPartials = 4;
+int router_split_width(int N);
 size_t router_split_bytes(int d, int N);
-cudaError_t launch_router_tc(const RouteArgs& a, void* split, float* partials, int* n_partials, cudaStream_t s);
+cudaError_t launch_router_split(const float* w_router, int d, int N, void* split, cudaStream_t s);
+cudaError_t launch_router_tc(const RouteArgs& a, const void* split, bool make_split, void* split_buf, float* partials,
+                             int* n_partials, cudaStream_t s);
+// z-loss partial slots (RouteArgs.zl_part) for T tokens
+size_t router_zl_slots(int64_t T);
 
 // 2-D bf16 TMA tensor map over a row-major [outer, inner] tensor, 128-byte
 // swizzle, zero fill outside the tensor.

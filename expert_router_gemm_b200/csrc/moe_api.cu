@@ -144,7 +144,7 @@ Layout layout(const Dims& D) {
   L.rcnt = take(sizeof(int32_t) * D.N);
   L.rz = take(sizeof(unsigned long long) * D.N);
   L.zero_end = o;
-  L.rzl = take(sizeof(double) * ((D.T + kRouteMinBlockTokens - 1) / kRouteMinBlockTokens));
+  L.rzl = take(sizeof(double) * router_zl_slots(D.T));
   const bool tc_router = D.bf16 && D.N >= kRouterTcMinExperts;
   L.rsplit = take(tc_router ? router_split_bytes(D.d, D.N) : 0);
   L.rlogits = take(tc_router ? sizeof(float) * kRouterMaxPartials * D.T * D.N : 0);
@@ -231,7 +231,8 @@ bool route_stats_requested(const moe_stats_t* s) {
 
 moe_status_t do_route(const Dims& D, const void* x, const float* w_router, const float* bias,
                       const float* sel_bias, const float* logits_in, float* logits_out, int32_t* topk_idx,
-                      float* topk_w, const moe_stats_t* stats, void* ws, cudaStream_t st) {
+                      float* topk_w, const moe_stats_t* stats, void* ws, cudaStream_t st,
+                      const void* w_split = nullptr) {
   const Layout L = layout(D);
   cudaError_t e = cudaMemsetAsync(ws, 0, L.zero_end, st);
   if (e != cudaSuccess) return cuda_status(e);
@@ -272,11 +273,13 @@ moe_status_t do_route(const Dims& D, const void* x, const float* w_router, const
   if (want_stats) a.stats = *stats;
   a.flags = at<uint32_t*>(ws, L.flags);
   a.n_partials = 1;
-  if (logits_in == nullptr && D.bf16 && D.N >= kRouterTcMinExperts && D.T > 0) {
-    // tensor-core router GEMM -> fp32 partial sums over K slices; the softmax /
+  if (logits_in == nullptr && D.bf16 && D.N >= kRouterTcMinExperts) {
+    // tensor-core router GEMM -> fp32 partial sums over K slices (the router
+    // weight's bf16 split made here unless the caller has one); the softmax /
     // top-k pass adds them (and the bias) in a fixed order and writes logits_out
     int parts = 1;
-    e = launch_router_tc(a, at<void*>(ws, L.rsplit), at<float*>(ws, L.rlogits), &parts, st);
+    e = launch_router_tc(a, w_split, w_split == nullptr, at<void*>(ws, L.rsplit), at<float*>(ws, L.rlogits), &parts,
+                         st);
     if (e != cudaSuccess) return cuda_status(e);
     a.logits_in = at<float*>(ws, L.rlogits);
     a.n_partials = parts;
@@ -609,6 +612,7 @@ moe_status_t moe_layer_fwd(const moe_config_t* cfg, const moe_weights_t* weights
     return MOE_ERR_MISALIGNED;
   if (D.fs > 0 && (!aligned16(weights->ws1) || !aligned16(weights->ws3) || !aligned16(weights->ws2)))
     return MOE_ERR_MISALIGNED;
+  if (!aligned16(weights->w_router_split)) return MOE_ERR_MISALIGNED;
   const Layout L = layout(D);
   if ((s = check_ws(ws, ws_bytes, L.layer_end)) != MOE_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -624,7 +628,7 @@ moe_status_t moe_layer_fwd(const moe_config_t* cfg, const moe_weights_t* weights
   void* shared_out = D.fs ? at<void*>(ws, L.sh) : nullptr;
 
   if ((s = do_route(D, x, weights->w_router, weights->router_bias, weights->selection_bias, nullptr, nullptr, idx, w,
-                    stats, ws, st)) != MOE_OK)
+                    stats, ws, st, D.bf16 ? weights->w_router_split : nullptr)) != MOE_OK)
     return s;
   if (D.mx) {
     void* x8 = at<void*>(ws, L.x8);
@@ -847,6 +851,22 @@ moe_status_t moe_layer_bwd(const moe_config_t* cfg, const moe_weights_t* weights
   }
   return cuda_status(launch_dx_gather(T, d, k, row_map, static_cast<const uint16_t*>(xp), dxr,
                                       static_cast<const uint16_t*>(dxs), static_cast<uint16_t*>(grads->dx), st));
+}
+
+moe_status_t moe_router_split_bytes(int32_t d, int32_t N, size_t* bytes) {
+  if (d < 1 || N < 1 || bytes == nullptr) return MOE_ERR_INVALID_ARG;
+  if (N > 256) return MOE_ERR_UNSUPPORTED;
+  *bytes = router_split_bytes(d, N);
+  return MOE_OK;
+}
+
+moe_status_t moe_router_split(const float* w_router, int32_t d, int32_t N, void* split, size_t bytes,
+                              moe_stream_t stream) {
+  if (d < 1 || N < 1 || w_router == nullptr || split == nullptr) return MOE_ERR_INVALID_ARG;
+  if (N > 256 || d % 64) return MOE_ERR_UNSUPPORTED;
+  if (bytes < router_split_bytes(d, N)) return MOE_ERR_WORKSPACE;
+  if (!aligned16(split)) return MOE_ERR_MISALIGNED;
+  return cuda_status(launch_router_split(w_router, d, N, split, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 moe_status_t moe_set_wait_limit_ns(uint64_t ns) {

@@ -14,6 +14,8 @@
 // is already bf16, so every product x*hi, x*mid, x*lo is exact and the three
 // MMAs of a K slab accumulate x*w in the fp32 tensor-memory accumulator.  The
 // result differs from a CUDA-core fp32 dot product only in summation order.
+// The split is made per call (split_router_kernel) unless the caller passes one
+// made once by moe_router_split.
 //
 // 192 threads per CTA: warp 0 lane 0 issues the TMA loads (x slab 128 x 64 and
 // the three weight slabs of this CTA's experts per stage), warp 1 allocates TMEM
@@ -321,14 +323,25 @@ int split_width(int N) { return N > 64 ? (N + 127) / 128 * 128 : (N + 63) / 64 *
 
 }  // namespace
 
+int router_split_width(int N) { return split_width(N); }
+
 size_t router_split_bytes(int d, int N) { return 3ull * d * split_width(N) * sizeof(uint16_t); }
 
-cudaError_t launch_router_tc(const RouteArgs& a, void* split, float* partials, int* n_partials, cudaStream_t s) {
+cudaError_t launch_router_split(const float* w_router, int d, int N, void* split, cudaStream_t s) {
+  split_router_kernel<<<(d + 7) / 8, dim3(32, 8), 0, s>>>(w_router, static_cast<uint16_t*>(split), d, N,
+                                                         split_width(N));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_router_tc(const RouteArgs& a, const void* split, bool make_split, void* split_buf, float* partials,
+                             int* n_partials, cudaStream_t s) {
   const bool pairs = a.N > 64;
   const int NP = split_width(a.N);
-  split_router_kernel<<<(a.d + 7) / 8, dim3(32, 8), 0, s>>>(a.w_router, static_cast<uint16_t*>(split), a.d, a.N, NP);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  if (make_split) {
+    cudaError_t e = launch_router_split(a.w_router, a.d, a.N, split_buf, s);
+    if (e != cudaSuccess) return e;
+    split = split_buf;
+  }
   CUtensorMap mx, mw;
   if (!make_tma_2d_bf16(&mx, a.x, a.d, a.T, BK, BM) || !make_tma_2d_bf16(&mw, split, NP, 3ull * a.d, 64, BK))
     return cudaErrorInvalidValue;

@@ -42,7 +42,8 @@ class moe_config_t(ctypes.Structure):
 class moe_weights_t(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("w_router", "router_bias", "w1", "w3", "w2", "ws1", "ws3", "ws2",
-                 "selection_bias", "w1_mx", "w1_sf", "w3_mx", "w3_sf", "w2_mx", "w2_sf")]
+                 "selection_bias", "w1_mx", "w1_sf", "w3_mx", "w3_sf", "w2_mx", "w2_sf",
+                 "w_router_split")]
 
 
 class moe_stats_t(ctypes.Structure):
@@ -89,6 +90,8 @@ _PROTOS = {
                                      _P, _P, ctypes.POINTER(moe_stats_t), _P, _SZ, _P]),
     "moe_read_flags": (ctypes.c_int, [_P, _SZ, ctypes.POINTER(ctypes.c_uint32), _P]),
     "moe_set_wait_limit_ns": (ctypes.c_int, [ctypes.c_uint64]),
+    "moe_router_split_bytes": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int32, ctypes.POINTER(_SZ)]),
+    "moe_router_split": (ctypes.c_int, [_P, ctypes.c_int32, ctypes.c_int32, _P, _SZ, _P]),
     "moe_backward_workspace_size": (ctypes.c_int, [ctypes.POINTER(moe_config_t), ctypes.POINTER(_SZ)]),
     "moe_layer_bwd": (ctypes.c_int, [ctypes.POINTER(moe_config_t), ctypes.POINTER(moe_weights_t), _P, _P,
                                      ctypes.c_float, ctypes.c_float, ctypes.POINTER(moe_grads_t), _P, _SZ,
@@ -157,10 +160,10 @@ def config_from_workload(w, T: Optional[int] = None, **over) -> moe_config_t:
 
 def make_weights(w_router, router_bias=None, w1=None, w3=None, w2=None, ws1=None, ws3=None,
                  ws2=None, selection_bias=None, w1_mx=None, w1_sf=None, w3_mx=None, w3_sf=None,
-                 w2_mx=None, w2_sf=None) -> moe_weights_t:
+                 w2_mx=None, w2_sf=None, w_router_split=None) -> moe_weights_t:
     return moe_weights_t(*[_ptr(t) for t in (w_router, router_bias, w1, w3, w2, ws1, ws3, ws2,
                                             selection_bias, w1_mx, w1_sf, w3_mx, w3_sf, w2_mx,
-                                            w2_sf)])
+                                            w2_sf, w_router_split)])
 
 
 def make_stats(y_frac=None, z_mean=None, l_aux_p3=None, l_aux_switch=None, counts=None,
@@ -321,6 +324,17 @@ def moe_read_flags(ws, stream=None) -> int:
     return v.value
 
 
+def moe_router_split_bytes(d: int, N: int) -> int:
+    b = _SZ()
+    _check(_lib.moe_router_split_bytes(d, N, ctypes.byref(b)), "moe_router_split_bytes")
+    return b.value
+
+
+def moe_router_split(w_router, d: int, N: int, split, stream=None) -> None:
+    _check(_lib.moe_router_split(_ptr(w_router), d, N, _ptr(split), split.numel() * split.element_size(),
+                                 _stream(stream)), "moe_router_split")
+
+
 def moe_set_wait_limit_ns(ns: int) -> None:
     """Bound of the bf16 grouped GEMM's pipeline waits for later launches (0: the 2 s default)."""
     _check(_lib.moe_set_wait_limit_ns(int(ns)), "moe_set_wait_limit_ns")
@@ -347,13 +361,23 @@ class DeviceLayer:
     ws2: Optional[torch.Tensor] = None
     selection_bias: Optional[torch.Tensor] = None
     mx: Optional[dict] = None      # block-scaled FP8 weights (quantize_mx)
+    router_split: Optional[torch.Tensor] = None   # bf16 split of w_router (split_router)
 
     def weights(self) -> moe_weights_t:
         m = self.mx or {}
         return make_weights(self.w_router, self.bias, self.w1, self.w3, self.w2,
                             self.ws1, self.ws3, self.ws2, self.selection_bias,
                             m.get("w1_mx"), m.get("w1_sf"), m.get("w3_mx"), m.get("w3_sf"),
-                            m.get("w2_mx"), m.get("w2_sf"))
+                            m.get("w2_mx"), m.get("w2_sf"), self.router_split)
+
+    def split_router(self, stream=None) -> torch.Tensor:
+        """Make the bf16 split of the router weight once (moe_router_split) and
+        pass it to later layer calls through weights()."""
+        d, N = self.cfg.d, self.cfg.N
+        buf = torch.empty(moe_router_split_bytes(d, N), dtype=torch.uint8, device=self.w_router.device)
+        moe_router_split(self.w_router, d, N, buf, stream)
+        self.router_split = buf
+        return buf
 
     def quantize_mx(self, stream=None) -> dict:
         """Quantize the routed experts' bf16 weights to block-scaled FP8 on the

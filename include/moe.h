@@ -115,6 +115,9 @@ typedef struct {
   const void* w3_sf;
   const void* w2_mx;         /* [N][d][f] codes of W2 (K = f) */
   const void* w2_sf;         /* N * d * f / 32 bytes */
+  /* Optional bf16 split of w_router made by moe_router_split (bf16 layers); NULL =
+     moe_layer_fwd splits w_router itself on every call. */
+  const void* w_router_split;
 } moe_weights_t;
 
 /* Load-balance and capacity statistics.  Device pointers; each may be NULL. */
@@ -200,6 +203,24 @@ moe_status_t moe_route_from_logits(const moe_config_t* cfg, const float* logits,
                                    const float* selection_bias, int32_t* topk_idx,
                                    float* topk_w, moe_stats_t* stats, void* ws,
                                    size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * moe_router_split / moe_router_split_bytes - the bf16 form of the fp32 router
+ * weight that the tensor-core router multiplies ("MoE 训练加速实战" §2.2,
+ * g = x W_r, with the router kept in fp32, §1 pain point 4): every weight w of
+ * W_r [d, N] is split exactly into three bf16 values, w = hi + mid + lo (hi =
+ * bf16(w), mid = bf16(w - hi), lo = w - hi - mid), stored as [3][d][NP] with
+ * NP = 64, 128 or 256 (the smallest of those >= N; columns N..NP-1 zero).  x is
+ * bf16, so each product x*hi, x*mid, x*lo is exact and their fp32 sum is x*w
+ * up to the order of the additions.  moe_layer_fwd uses a split passed in
+ * moe_weights_t.w_router_split instead of making its own; the split stays
+ * valid while W_r is unchanged.  split: device, 16-byte aligned, >= the bytes
+ * that moe_router_split_bytes reports; d % 64 == 0, N <= 256 (else
+ * MOE_ERR_UNSUPPORTED).
+ */
+moe_status_t moe_router_split_bytes(int32_t d, int32_t N, size_t* bytes);
+moe_status_t moe_router_split(const float* w_router, int32_t d, int32_t N, void* split, size_t bytes,
+                              moe_stream_t stream);
 
 /*
  * moe_bias_update - one Aux-Loss-Free bias step ("MoE 训练加速实战" §5.4):

@@ -236,3 +236,17 @@ def test_wait_limit_validation():
     st = moe.raw_call("moe_set_wait_limit_ns", ctypes.c_uint64(2_000_000_001))
     assert st == INVALID
     assert moe.raw_call("moe_set_wait_limit_ns", ctypes.c_uint64(0)) == OK
+
+
+def test_router_split_validation():
+    # host only: sizes, unsupported shapes and a short buffer are refused before any launch
+    assert moe.moe_router_split_bytes(4096, 128) == 3 * 4096 * 128 * 2
+    assert moe.moe_router_split_bytes(4096, 8) == 3 * 4096 * 64 * 2
+    assert moe.moe_router_split_bytes(7168, 256) == 3 * 7168 * 256 * 2
+    n = ctypes.c_size_t()
+    assert moe.raw_call("moe_router_split_bytes", 64, 257, ctypes.byref(n)) == UNSUP
+    assert moe.raw_call("moe_router_split_bytes", 0, 8, ctypes.byref(n)) == INVALID
+    fake = ctypes.c_void_p(16)
+    assert moe.raw_call("moe_router_split", fake, 64, 8, fake, ctypes.c_size_t(10), None) == WS
+    assert moe.raw_call("moe_router_split", fake, 96, 8, fake, ctypes.c_size_t(1 << 20), None) == UNSUP
+    assert moe.raw_call("moe_router_split", None, 64, 8, fake, ctypes.c_size_t(1 << 20), None) == INVALID

@@ -220,3 +220,59 @@ def test_empty_batch():
                     torch.empty((0, 2), dtype=torch.int32, device="cuda"))
     assert np.all(r["seg_off"] == 0) and np.all(r["seg_count"] == 0)
     assert r["stats"]["avg_tokens_per_expert"][0] == 0
+
+
+@pytest.mark.parametrize("T,d,N,k,bias,sel", [
+    (300, 256, 8, 2, True, False),      # N <= 64: 64-expert tiles, K split four ways
+    (8192, 4096, 128, 8, False, False),  # the Qwen3-shaped router: CTA pairs, two K splits
+    (1000, 512, 100, 6, True, True),     # ragged N, selection bias
+    (640, 7168, 256, 8, True, False),    # N = 256
+    (33, 1024, 128, 8, False, True),     # fewer tokens than one tile
+])
+def test_router_decisions_match_routing_its_own_logits(T, d, N, k, bias, sel):
+    """moe_route on the tensor cores (the router GEMM's K-slice partial sums, then
+    the routing kernel) and the routing kernel fed
+    the router's own fp32 logits through moe_route_from_logits take the same
+    decisions bit for bit, and report the same statistics within the fp32
+    summation-order difference of the two."""
+    x = synth.f32_to_bf16_bits(synth.normal_f32(11, 1, (T, d)))
+    wr = synth.normal_f32(11, 2, (d, N)) * np.float32(1 / np.sqrt(d))
+    b = synth.normal_f32(11, 3, (N,)) if bias else None
+    sb = synth.make_selection_bias(11, N) if sel else None
+    cfg = moe.make_config(T=T, d=d, N=N, k=k, f=64, capacity_factor=1.0, dtype="bf16")
+    logits = torch.full((T, N), float("nan"), device="cuda")
+    idx = torch.full((T, k), -1, dtype=torch.int32, device="cuda")
+    wt = torch.full((T, k), float("nan"), device="cuda")
+    ws = gu.op_workspace(cfg)
+    bufs, st = gu.new_stats(N)
+    moe.moe_route(cfg, gu.cuda_tensor(x), gu.cuda_tensor(wr), None if b is None else gu.cuda_tensor(b),
+                  None if sb is None else gu.cuda_tensor(sb), logits, idx, wt, st, ws)
+    assert moe.moe_read_flags(ws) == 0
+    lg = gu.host(logits)
+    assert np.all(np.isfinite(lg))
+    idx2, w2, st2, flags2 = gu.route_from_logits(cfg, lg, sb)
+    assert flags2 == 0
+    np.testing.assert_array_equal(gu.host(idx), idx2)
+    np.testing.assert_array_equal(gu.host(wt), w2)
+    fused = gu.stats_host(bufs)
+    np.testing.assert_array_equal(fused["counts"], st2["counts"])
+    for key in ("y_frac", "top2_ratio", "load_std"):
+        np.testing.assert_array_equal(fused[key], st2[key], err_msg=key)
+    for key in ("z_mean", "l_aux_p3", "l_aux_switch", "z_loss"):
+        np.testing.assert_allclose(fused[key], st2[key], rtol=1e-5, atol=1e-9, err_msg=key)
+
+
+def test_layer_with_a_router_split_made_once_is_unchanged():
+    """moe_layer_fwd with the bf16 split of W_r passed in (moe_router_split, made
+    once) gives the same bytes as the layer that splits W_r itself."""
+    from expert_router_gemm_b200.configs import Workload
+    w = Workload("presplit", T=1024, d=512, N=128, k=8, f=256, capacity_factor=1.0)
+    inp = synth.make_inputs(w)
+    dl = moe.to_device(inp, moe.config_from_workload(w))
+    y0, st0, f0 = gu.layer_fwd(dl)
+    dl.split_router()
+    y1, st1, f1 = gu.layer_fwd(dl)
+    assert f0 == 0 and f1 == 0
+    np.testing.assert_array_equal(y0, y1)
+    for key in st0:
+        np.testing.assert_array_equal(st0[key], st1[key], err_msg=key)
