@@ -196,7 +196,7 @@ __device__ __forceinline__ int b_box_col(int n0, uint32_t rank, int i) {
   return MODE == MODE_SWIGLU ? n0 + 64 * i : n0 + 128 * static_cast<int>(rank) + 64 * i;
 }
 
-template <int MODE, int CG>
+template <int MODE, int CG, int AMODE>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_ffn_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                        const __grid_constant__ CUtensorMap tmB1, const TcParams p) {
@@ -220,8 +220,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // full: the expect-tx arrival; with a cp.async slab also one arrival per
     // producer lane, and on a pair one relayed arrival for the odd CTA's slab
     // (counted on afull, 32 lanes, in the odd CTA)
-    const bool lsu = p.a_token != nullptr && p.a_gather == A_GATHER_LSU;
-    const uint32_t full_count = lsu ? (CG == 2 ? 34u : 33u) : 1u;
+    const uint32_t full_count = AMODE == A_GATHER_LSU ? (CG == 2 ? 34u : 33u) : 1u;
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(smem_addr(&tl.full[s]), full_count);
       mbar_init(smem_addr(&tl.empty[s]), 1);
@@ -291,7 +290,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // i: chunk i % 8 of rows i / 8, i / 8 + 4, ...), each lane arriving on the
     // stage's barrier when its copies have landed.  Lane 0 waits for free
     // stages, posts the expected TMA bytes and loads B.
-    const int amode = p.a_token == nullptr ? A_TILE : p.a_gather;
+    constexpr int amode = AMODE;
     if (amode != A_TILE || lane == 0) {
       uint32_t stage = 0, phase = 0, issued = 0, last_par = 0;
       bool ok = true;
@@ -307,11 +306,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           return static_cast<unsigned>(v) < static_cast<unsigned>(p.a_token_rows) ? v : 0;
         };
         int tok4[4] = {0, 0, 0, 0};
-        int tok32[32];
-        if (amode == A_GATHER_TMA) {
+        int tok32[amode == A_GATHER_LSU ? 32 : 1];
+        if constexpr (amode == A_GATHER_TMA) {
 #pragma unroll
           for (int i = 0; i < 4; ++i) tok4[i] = token_of(4 * lane + i);
-        } else if (amode == A_GATHER_LSU) {
+        } else if constexpr (amode == A_GATHER_LSU) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) tok32[i] = token_of(4 * i + (lane >> 3));
         }
@@ -331,12 +330,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t fb = (CG == 1 || rank == 0) ? fb_local : mapa_shared(fb_local, 0);
           const uint32_t tx = static_cast<uint32_t>((amode == A_GATHER_LSU ? 0 : A_BYTES) + C::B_BYTES);
           if (lane == 0 && (CG == 1 || rank == 0)) mbar_arrive_expect_tx(fb_local, CG * tx);
-          if (amode == A_TILE) {
+          if constexpr (amode == A_TILE) {
             if (CG == 1)
               tma_load_2d(a_dst, &tmA, fb, kb * BK, a_row);
             else
               tma_load_2d_pair(a_dst, &tmA, fb, kb * BK, a_row);
-          } else if (amode == A_GATHER_TMA) {
+          } else if constexpr (amode == A_GATHER_TMA) {
             __syncwarp();
             if (CG == 1)
               tma_gather4(a_dst + lane * 4 * 128, &tmA, fb, kb * BK, tok4[0], tok4[1], tok4[2], tok4[3]);
@@ -392,7 +391,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == 1) {
-    const bool lsu_a = p.a_token != nullptr && p.a_gather == A_GATHER_LSU;
+    constexpr bool lsu_a = AMODE == A_GATHER_LSU;
     if (CG == 2 && lane == 0 && rank != 0 && lsu_a) {
       // ------------------------------------------------------ relay (odd CTA)
       // The odd CTA's producer lanes count each stage's cp.async slab on afull;
@@ -425,8 +424,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         issued_any = true;
         const uint32_t d_tmem = tmem_base + acc * MMA_N;
         for (int kb = 0; kb < KB; ++kb) {
-          // cluster scope: the odd CTA's cp.async slab is announced by its own arrival
-          if (!mbar_wait<CG == 2>(smem_addr(&tl.full[stage]), phase, abort, p.flags, kFlagTimeout, p.wait_ns)) {
+          // with a cp.async slab on a CTA pair, the odd CTA announces its half by an
+          // arrival of its own: acquire at cluster scope (only then: it costs)
+          if (!mbar_wait<CG == 2 && lsu_a>(smem_addr(&tl.full[stage]), phase, abort, p.flags, kFlagTimeout,
+                                            p.wait_ns)) {
             ok = false;
             break;
           }
@@ -561,7 +562,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------- host side
-template <int MODE, int CG>
+template <int MODE, int CG, int AMODE>
 cudaError_t set_smem_attr() {
   static std::once_flag once[64];
   int dev = 0;
@@ -569,16 +570,16 @@ cudaError_t set_smem_attr() {
   if (e != cudaSuccess) return e;
   cudaError_t r = cudaSuccess;
   std::call_once(once[dev & 63], [&] {
-    r = cudaFuncSetAttribute(tc_ffn_gemm_kernel<MODE, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    r = cudaFuncSetAttribute(tc_ffn_gemm_kernel<MODE, CG, AMODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem_bytes<CG>()));
   });
   return r;
 }
 
-template <int MODE, int CG>
+template <int MODE, int CG, int AMODE = A_TILE>
 cudaError_t launch_gemm(const CUtensorMap& A, const CUtensorMap& B0, const CUtensorMap& B1, const TcParams& p,
                         int64_t bound_units, cudaStream_t s) {
-  cudaError_t e = set_smem_attr<MODE, CG>();
+  cudaError_t e = set_smem_attr<MODE, CG, AMODE>();
   if (e != cudaSuccess) return e;
   int units = device_sm_count() / CG;
   units = static_cast<int>(std::min<int64_t>(units, std::max<int64_t>(bound_units, 1)));
@@ -597,11 +598,11 @@ cudaError_t launch_gemm(const CUtensorMap& A, const CUtensorMap& B0, const CUten
     cfg.numAttrs = 1;
     // persistent: no more pairs than can be resident at once
     int max_clusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&max_clusters, tc_ffn_gemm_kernel<MODE, CG>, &cfg) == cudaSuccess &&
+    if (cudaOccupancyMaxActiveClusters(&max_clusters, tc_ffn_gemm_kernel<MODE, CG, AMODE>, &cfg) == cudaSuccess &&
         max_clusters > 0 && max_clusters < units)
       cfg.gridDim.x = static_cast<unsigned>(max_clusters * 2);
   }
-  e = cudaLaunchKernelEx(&cfg, tc_ffn_gemm_kernel<MODE, CG>, A, B0, B1, p);
+  e = cudaLaunchKernelEx(&cfg, tc_ffn_gemm_kernel<MODE, CG, AMODE>, A, B0, B1, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -666,7 +667,10 @@ cudaError_t launch_pair(const FfnArgs& a, const CUtensorMap& mA1, const CUtensor
   p.a_src = a.a;
   p.a_token_rows = static_cast<int>(a.a_token_rows);
   p.a_gather = gather_mode();
-  cudaError_t e = launch_gemm<MODE_SWIGLU, CG>(mA1, mW1, mW3, p, m_bound * ((a.f + 127) / 128), s);
+  const int64_t units1 = m_bound * ((a.f + 127) / 128);
+  cudaError_t e = p.a_token == nullptr       ? launch_gemm<MODE_SWIGLU, CG>(mA1, mW1, mW3, p, units1, s)
+                  : p.a_gather == A_GATHER_TMA ? launch_gemm<MODE_SWIGLU, CG, A_GATHER_TMA>(mA1, mW1, mW3, p, units1, s)
+                                               : launch_gemm<MODE_SWIGLU, CG, A_GATHER_LSU>(mA1, mW1, mW3, p, units1, s);
   if (e != cudaSuccess) return e;
   p.a_token = nullptr;
   p.a_src = nullptr;
