@@ -668,6 +668,12 @@ def main():
             "kcycles_per_step": (round(stage_ms["expert_ffn"] * clocks_b["sm_mhz"], 1)
                                  if clocks_b.get("sm_mhz") else None),
             "algorithmic_flops_per_step": ffn_flops,
+            # the other roofline of the same kernel: its expert weights stream from HBM
+            # once per call (the bound on layers with few rows per expert)
+            "weight_stream": {"bytes_per_step": ffn_wbytes,
+                              "GB/s": round(gbs(ffn_wbytes, stage_ms["expert_ffn"]), 1),
+                              "frac_hbm": round(gbs(ffn_wbytes, stage_ms["expert_ffn"]) / hbm, 4),
+                              "hbm_peak_gbs": hbm},
             "traffic": (tr["expert_ffn_per_step"] * 1.0 if tr and "expert_ffn_per_step" in tr else None)}
 
         # -------------------------------------------- e2e: host buffers through the C ABI
