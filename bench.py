@@ -443,6 +443,10 @@ def main():
         torch.cuda.synchronize()
         dl.w1 = dl.w3 = dl.w2 = None   # the FP8 layer reads only the quantized experts
         torch.cuda.empty_cache()
+    # the router weight is constant across calls: its exact bf16 split (what the
+    # tensor-core router multiplies) is made once, like the FP8 weights above
+    if w.dtype == "bf16":
+        dl.split_router()
     aux_free = args.aux_free > 0
     if aux_free:
         dl.selection_bias = torch.zeros(w.N, dtype=torch.float32, device="cuda")
@@ -499,10 +503,11 @@ def main():
     value = replicas.job_throughput(w.T, world, ms / 1e3)
     clocks = sampler.summary()
 
-    # route: bf16 splits W_r, runs the tensor-core router GEMM and the softmax /
-    # top-k kernel (fp32: one fused kernel); dispatch: mask, scan, scatter; two
-    # grouped GEMMs (+ two for the shared expert); combine; the bias update
-    per_step_launches = ((3 if w.dtype == "bf16" else 1) + 3 + 2 + (2 if w.f_shared else 0) + 1
+    # route: bf16 runs the tensor-core router GEMM (on the split made once) and
+    # the softmax / top-k kernel (fp32: one fused kernel); dispatch: mask, scan,
+    # scatter; two grouped GEMMs (+ two for the shared expert); combine; the bias
+    # update
+    per_step_launches = ((2 if w.dtype == "bf16" else 1) + 3 + 2 + (2 if w.f_shared else 0) + 1
                          + (1 if aux_free else 0))
     router_stats = {key: round(float(sbuf[key].item()), 6) for key in
                     ("l_aux_p3", "l_aux_switch", "z_loss", "load_std", "top2_ratio",
@@ -513,6 +518,8 @@ def main():
             "dtype": "mxfp8 experts (e4m3, bf16 in/out)" if mx else w.dtype,
             "data": "synthetic",
             "config": dict(workload_config(w), expert_gemm=args.gemm, parallelism=f"replicas x{world}",
+                           router_split=("made once before the loop (moe_router_split)"
+                                         if w.dtype == "bf16" else None),
                            l2="inputs larger than L2: the expert weights read every step "
                               f"({(inp.w1.nbytes + inp.w3.nbytes + inp.w2.nbytes) / 1e9:.2f} GB) "
                               "exceed the 126 MB L2; no flush"),
