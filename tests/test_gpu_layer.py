@@ -34,6 +34,16 @@ SMALL = [
              bias_pattern=configs.SKEW.bias_pattern, bias_beta_gamma=configs.SKEW_BETA_GAMMA),
     Workload("topN-bf16", T=300, d=128, N=8, k=8, f=128, capacity_factor=1.0),
     Workload("manytiles-bf16", T=1536, d=1024, N=4, k=2, f=1024, capacity_factor=1.0),
+    # the largest top-k (32 slots per token) and an odd one (the combine's
+    # generic slot loop), the latter with a shared expert
+    Workload("top32-bf16", T=512, d=256, N=64, k=32, f=128, capacity_factor=1.25),
+    Workload("top3-shared-bf16", T=600, d=192, N=12, k=3, f=192, f_shared=64, capacity_factor=1.0),
+]
+
+F32 = [
+    configs.TINY,
+    # ragged everywhere: d and f off every tile edge, an odd top-k, a shared expert
+    Workload("odd-f32", T=300, d=100, N=6, k=3, f=72, f_shared=40, capacity_factor=1.25, dtype="f32"),
 ]
 
 
@@ -47,8 +57,8 @@ def _run(w: Workload, align=0):
     return inp, staged, y, st
 
 
-def test_tiny_fp32_layer():
-    w = configs.TINY
+@pytest.mark.parametrize("w", F32, ids=[w.name for w in F32])
+def test_fp32_layers(w):
     inp, staged, y, st = _run(w)
     np.testing.assert_array_equal(y, staged["y"])
     rel, n, flips = compare_layer(inp, w, y, staged["idx"], staged["row_map"], staged["logits"],
