@@ -37,6 +37,8 @@ CASES = [
     # multiple of 128 and N not a multiple of 4; and two 128-expert column tiles
     (Workload("bwd-wide-ragged", T=300, d=320, N=100, k=4, f=128, capacity_factor=1.1), 0.05, 1e-3),
     (Workload("bwd-n256", T=256, d=256, N=256, k=8, f=128, capacity_factor=1.25), 0.01, 1e-3),
+    # ~256 rows per expert (the DeepSeek-shaped layer's tile occupancy)
+    (Workload("bwd-256-rows", T=1024, d=256, N=8, k=2, f=256, capacity_factor=1.25), 0.01, 1e-3),
 ]
 
 
