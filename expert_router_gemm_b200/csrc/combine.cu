@@ -42,6 +42,8 @@ template <int KS>
 __global__ void __launch_bounds__(kCombineThreads) combine_bf16_kernel(const CombineArgs a) {
   __shared__ int rows[32];
   __shared__ float wts[32];
+  grid_dep_wait();
+  grid_dep_launch();
   const int64_t t = blockIdx.x;
   const int k = KS > 0 ? KS : a.k;
   if (threadIdx.x < k) {
@@ -83,6 +85,8 @@ __global__ void __launch_bounds__(kCombineThreads) combine_bf16_kernel(const Com
 __global__ void __launch_bounds__(kCombineThreads) combine_f32_kernel(const CombineArgs a) {
   __shared__ int rows[32];
   __shared__ float wts[32];
+  grid_dep_wait();
+  grid_dep_launch();
   const int64_t t = blockIdx.x;
   const int k = a.k;
   if (threadIdx.x < k) {
@@ -121,20 +125,17 @@ __global__ void __launch_bounds__(kCombineThreads) combine_f32_kernel(const Comb
 
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s) {
   if (a.T == 0) return cudaSuccess;
-  const unsigned blocks = static_cast<unsigned>(a.T);
-  if (!a.is_bf16) {
-    combine_f32_kernel<<<blocks, kCombineThreads, 0, s>>>(a);
-  } else {
-    switch (a.k) {
-      case 1: combine_bf16_kernel<1><<<blocks, kCombineThreads, 0, s>>>(a); break;
-      case 2: combine_bf16_kernel<2><<<blocks, kCombineThreads, 0, s>>>(a); break;
-      case 4: combine_bf16_kernel<4><<<blocks, kCombineThreads, 0, s>>>(a); break;
-      case 6: combine_bf16_kernel<6><<<blocks, kCombineThreads, 0, s>>>(a); break;
-      case 8: combine_bf16_kernel<8><<<blocks, kCombineThreads, 0, s>>>(a); break;
-      default: combine_bf16_kernel<0><<<blocks, kCombineThreads, 0, s>>>(a); break;
-    }
+  // may start while the expert GEMM before it finishes (it waits for its results first)
+  const dim3 grid(static_cast<unsigned>(a.T)), block(kCombineThreads);
+  if (!a.is_bf16) return launch_overlapped(combine_f32_kernel, grid, block, 0, s, a);
+  switch (a.k) {
+    case 1: return launch_overlapped(combine_bf16_kernel<1>, grid, block, 0, s, a);
+    case 2: return launch_overlapped(combine_bf16_kernel<2>, grid, block, 0, s, a);
+    case 4: return launch_overlapped(combine_bf16_kernel<4>, grid, block, 0, s, a);
+    case 6: return launch_overlapped(combine_bf16_kernel<6>, grid, block, 0, s, a);
+    case 8: return launch_overlapped(combine_bf16_kernel<8>, grid, block, 0, s, a);
+    default: return launch_overlapped(combine_bf16_kernel<0>, grid, block, 0, s, a);
   }
-  return cudaGetLastError();
 }
 
 }  // namespace moe

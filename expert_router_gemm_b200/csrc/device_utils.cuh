@@ -45,6 +45,16 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 // microseconds; 2 s means the pipeline is broken.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
+// ------------------------------------------------------------------ launch overlap
+// Programmatic dependent launch: a kernel launched with launch_overlapped() may
+// start while the previous kernel of the stream is still running.  It calls
+// grid_dep_wait() before anything else that may read that kernel's results:
+// the wait returns once the previous kernel has completed and its writes are
+// visible (at once for a normal launch).  grid_dep_launch() lets the next
+// kernel of the stream start launching; it carries no data.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------------------ smem
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

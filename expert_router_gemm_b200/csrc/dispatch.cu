@@ -42,6 +42,8 @@ __device__ __forceinline__ bool slot_valid(const int32_t* idx_row, int j, int e,
 
 __global__ void __launch_bounds__(kMaskThreads) dispatch_mask_kernel(const DispatchArgs a) {
   __shared__ uint32_t m[256];
+  grid_dep_wait();
+  grid_dep_launch();
   const int tid = threadIdx.x;
   const int N = a.N, k = a.k;
   for (int e = tid; e < N; e += kMaskThreads) m[e] = 0u;
@@ -71,6 +73,8 @@ __global__ void __launch_bounds__(1024) dispatch_scan_kernel(const DispatchArgs 
   __shared__ int is_last;
   __shared__ int kept_s[256];
   __shared__ int drop_s[256];
+  grid_dep_wait();
+  grid_dep_launch();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int N = a.N;
   const int e = blockIdx.x * 32 + lane;
@@ -150,6 +154,8 @@ __global__ void __launch_bounds__(kScatterThreads) dispatch_scatter_kernel(const
   __shared__ int base_s[256];
   __shared__ int off_s[256];
   __shared__ int rows_s[kScatterTokens][32];
+  grid_dep_wait();
+  grid_dep_launch();
   const int N = a.N, k = a.k;
   const int64_t t_first = static_cast<int64_t>(blockIdx.x) * kScatterTokens;
   const int64_t blk = t_first / kDispatchTokens;                      // mask block
@@ -205,6 +211,8 @@ __global__ void __launch_bounds__(kMaskThreads) dispatch_index_kernel(const Disp
   __shared__ uint32_t m[256];
   __shared__ int base_s[256];
   __shared__ int off_s[256];
+  grid_dep_wait();
+  grid_dep_launch();
   const int N = a.N, k = a.k;
   const int64_t blk = blockIdx.x;
   for (int e = threadIdx.x; e < N; e += kMaskThreads) {
@@ -247,6 +255,8 @@ __global__ void __launch_bounds__(kScatterThreads) dispatch_scatter_mx_kernel(co
   __shared__ int base_s[256];
   __shared__ int off_s[256];
   __shared__ int rows_s[kScatterTokens][32];
+  grid_dep_wait();
+  grid_dep_launch();
   const int N = a.N, k = a.k;
   const int64_t t_first = static_cast<int64_t>(blockIdx.x) * kScatterTokens;
   const int64_t blk = t_first / kDispatchTokens;
@@ -314,16 +324,18 @@ __global__ void __launch_bounds__(kScatterThreads) dispatch_scatter_mx_kernel(co
 
 cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t s) {
   const int blocks = static_cast<int>((a.T + kDispatchTokens - 1) / kDispatchTokens);
-  dispatch_mask_kernel<<<blocks, kMaskThreads, 0, s>>>(a);
-  dispatch_scan_kernel<<<(a.N + 31) / 32, 1024, 0, s>>>(a, blocks);
+  // each kernel may start while the one before it finishes (it waits for its
+  // results first)
+  cudaError_t e = launch_overlapped(dispatch_mask_kernel, dim3(blocks), dim3(kMaskThreads), 0, s, a);
+  if (e == cudaSuccess)
+    e = launch_overlapped(dispatch_scan_kernel, dim3((a.N + 31) / 32), dim3(1024), 0, s, a, blocks);
+  if (e != cudaSuccess) return e;
   const unsigned sblocks = static_cast<unsigned>((a.T + kScatterTokens - 1) / kScatterTokens);
   if (a.row_token != nullptr)
-    dispatch_index_kernel<<<blocks, kMaskThreads, 0, s>>>(a);
-  else if (a.xp_sf != nullptr)
-    dispatch_scatter_mx_kernel<<<sblocks, kScatterThreads, 0, s>>>(a);
-  else
-    dispatch_scatter_kernel<<<sblocks, kScatterThreads, 0, s>>>(a);
-  return cudaGetLastError();
+    return launch_overlapped(dispatch_index_kernel, dim3(blocks), dim3(kMaskThreads), 0, s, a);
+  if (a.xp_sf != nullptr)
+    return launch_overlapped(dispatch_scatter_mx_kernel, dim3(sblocks), dim3(kScatterThreads), 0, s, a);
+  return launch_overlapped(dispatch_scatter_kernel, dim3(sblocks), dim3(kScatterThreads), 0, s, a);
 }
 
 }  // namespace moe

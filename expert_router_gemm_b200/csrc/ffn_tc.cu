@@ -246,6 +246,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_relinquish();
     }
   }
+  // the kernel before this one (the dispatch, or GEMM1 for GEMM2) has finished
+  // and its rows and segment table are visible; the next kernel may launch
+  grid_dep_wait();
+  grid_dep_launch();
   if (warp == 2) {
     // segment table -> per-group row range (clamped to the buffer) and tile prefix
     const int per = (G + 31) / 32;
@@ -588,14 +592,22 @@ cudaError_t launch_gemm(const CUtensorMap& A, const CUtensorMap& B0, const CUten
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem_bytes<CG>();
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  // CTA pairs may start while the kernel before them finishes (the kernel waits
+  // for its results first).  Single-CTA tiles are launched plainly: overlapped,
+  // the DeepSeek-shaped layer ran ~10 % slower at the power cap (its clock
+  // settled ~120 MHz lower), while the pair launches gained 1-3 % on the
+  // Qwen3-shaped layer.
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = (CG == 2 && launch_overlap_enabled()) ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   if (CG == 2) {
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 2;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.numAttrs = 2;
     // persistent: no more pairs than can be resident at once
     int max_clusters = 0;
     if (cudaOccupancyMaxActiveClusters(&max_clusters, tc_ffn_gemm_kernel<MODE, CG, AMODE>, &cfg) == cudaSuccess &&

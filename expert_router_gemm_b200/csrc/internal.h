@@ -287,4 +287,28 @@ constexpr uint32_t kFlagTimeout = MOE_FLAG_WAIT_TIMEOUT;
 
 int device_sm_count();    // cached per device
 
+// Whether forward-path kernels are launched to overlap the end of the
+// previous kernel of their stream (programmatic dependent launch; MOE_PDL=0
+// turns it off).
+bool launch_overlap_enabled();
+
+// Launches `kernel` so that it may start while the previous kernel of the
+// stream finishes; the kernel must call grid_dep_wait() before it reads
+// anything that kernel wrote (and before any early return).
+template <typename... Params, typename... Args>
+cudaError_t launch_overlapped(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = launch_overlap_enabled() ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 }  // namespace moe

@@ -4,12 +4,21 @@
 // CUDA kernels of route.cu, dispatch.cu, ffn_tc.cu, ffn_f32.cu and combine.cu.
 #include <algorithm>
 #include <cmath>
+#include <cstdlib>
 #include <cstdio>
 #include <cstring>
 
 #include "internal.h"
 
 namespace moe {
+
+bool launch_overlap_enabled() {
+  static const bool on = [] {
+    const char* v = std::getenv("MOE_PDL");
+    return v == nullptr || v[0] != '0';
+  }();
+  return on;
+}
 
 int device_sm_count() {
   static int cache[64] = {0};

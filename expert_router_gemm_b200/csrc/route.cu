@@ -64,6 +64,8 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const RouteArgs a)
   static_assert(NP / TX == 8, "each thread owns 8 experts");
   static_assert(BT >= kRouteMinBlockTokens, "z-loss partials are sized for kRouteMinBlockTokens-token blocks");
   __shared__ __align__(16) S sm;
+  grid_dep_wait();   // the router GEMM's partial sums are complete
+  grid_dep_launch();
 
   const int tid = threadIdx.x;
   const int64_t t0 = static_cast<int64_t>(blockIdx.x) * BT;
@@ -242,11 +244,10 @@ template <int NP>
 cudaError_t launch_np(const RouteArgs& a, cudaStream_t s) {
   const int bt = a.logits_in != nullptr ? kLogitsTokens : route_bt(NP);
   const unsigned blocks = static_cast<unsigned>((a.T + bt - 1) / bt);
+  // may start while the router GEMM before it finishes (it waits for its results first)
   if (a.logits_in != nullptr)
-    route_kernel<NP, true><<<blocks, kRouteThreads, 0, s>>>(a);
-  else
-    route_kernel<NP, false><<<blocks, kRouteThreads, 0, s>>>(a);
-  return cudaGetLastError();
+    return launch_overlapped(route_kernel<NP, true>, dim3(blocks), dim3(kRouteThreads), 0, s, a);
+  return launch_overlapped(route_kernel<NP, false>, dim3(blocks), dim3(kRouteThreads), 0, s, a);
 }
 
 }  // namespace
