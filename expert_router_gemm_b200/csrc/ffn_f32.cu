@@ -39,6 +39,8 @@ __global__ void __launch_bounds__(256) ffn1_f32_kernel(const FfnArgs a) {
   __shared__ float As[TS][TS + 1];
   __shared__ float B1s[TS][TS + 1];
   __shared__ float B3s[TS][TS + 1];
+  grid_dep_wait();   // the dispatch's rows and segment table are complete
+  grid_dep_launch();
   const int g = blockIdx.z;
   int count = 0;
   const int64_t seg0 = group_rows(a, g, &count);
@@ -83,6 +85,8 @@ __global__ void __launch_bounds__(256) ffn1_f32_kernel(const FfnArgs a) {
 __global__ void __launch_bounds__(256) ffn2_f32_kernel(const FfnArgs a) {
   __shared__ float As[TS][TS + 1];
   __shared__ float Bs[TS][TS + 1];
+  grid_dep_wait();   // h is complete
+  grid_dep_launch();
   const int g = blockIdx.z;
   int count = 0;
   const int64_t seg0 = group_rows(a, g, &count);
@@ -123,9 +127,10 @@ cudaError_t launch_ffn_f32(const FfnArgs& a, cudaStream_t s) {
   if (a.max_count <= 0 || a.G <= 0) return cudaSuccess;
   const dim3 block(TS, 8);
   const unsigned mt = static_cast<unsigned>((a.max_count + TS - 1) / TS);
-  ffn1_f32_kernel<<<dim3(mt, (a.f + TS - 1) / TS, a.G), block, 0, s>>>(a);
-  ffn2_f32_kernel<<<dim3(mt, (a.d + TS - 1) / TS, a.G), block, 0, s>>>(a);
-  return cudaGetLastError();
+  // each may start while the kernel before it finishes (it waits for its results first)
+  cudaError_t e = launch_overlapped(ffn1_f32_kernel, dim3(mt, (a.f + TS - 1) / TS, a.G), block, 0, s, a);
+  if (e != cudaSuccess) return e;
+  return launch_overlapped(ffn2_f32_kernel, dim3(mt, (a.d + TS - 1) / TS, a.G), block, 0, s, a);
 }
 
 }  // namespace moe
