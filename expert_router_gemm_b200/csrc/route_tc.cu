@@ -11,21 +11,28 @@
 // fp32 accuracy from bf16 tensor-core inputs: every fp32 router weight w is
 // split exactly into three bf16 values, w = hi + mid + lo (hi = bf16(w),
 // mid = bf16(w - hi), lo = w - hi - mid, which fits in 8 significant bits).  x
-// is already bf16, so every product x*hi, x*mid, x*lo is exact and the three
-// MMAs of a K slab accumulate x*w in the fp32 tensor-memory accumulator.  The
-// result differs from a CUDA-core fp32 dot product only in summation order.
-// The split is made per call (split_router_kernel) unless the caller passes one
+// is already bf16, so every product x*hi, x*mid, x*lo is exact.  Per K step
+// one MMA runs over the hi and mid parts side by side (staged as adjacent
+// 64-column chunks: twice the columns, one pass over A) into fp32 tensor-memory
+// accumulators of x*hi and x*mid, and one over the lo part into a third; the
+// epilogue adds hi + (mid + lo).  Where a logit is a single product, mid + lo
+// is exact and the logit is the correctly rounded x*w; otherwise the result
+// differs from a CUDA-core fp32 dot product only in summation order.  The
+// split is made per call (split_router_kernel) unless the caller passes one
 // made once by moe_router_split.
 //
 // 192 threads per CTA: warp 0 lane 0 issues the TMA loads (x slab 128 x 64 and
 // the three weight slabs of this CTA's experts per stage), warp 1 allocates TMEM
-// and lane 0 issues the MMAs, warps 2-5 move the accumulator through registers
-// and shared memory to the fp32 partial sums (whole 128-byte row pieces).  The operand stream is latency-bound (each
-// CTA streams its own tokens), so the work per staged byte decides the speed:
-//   CG = 1: one CTA per 128 tokens x 64 experts (M=128, N=64 MMA), N <= 64;
-//   CG = 2: a CTA pair per 256 tokens x 128 experts (cta_group::2, M=256,
-//           N=128): each CTA stages its own 128 tokens and 64 of the experts'
-//           weight columns, so each staged byte feeds twice the MMA work.
+// and lane 0 issues the MMAs, warps 2-5 move the accumulators through registers
+// and shared memory to the fp32 partial sums (whole 128-byte row pieces).  The
+// operand stream is latency-bound (each CTA streams its own tokens), so the
+// work per staged byte decides the speed:
+//   CG = 1: one CTA per 128 tokens x 64 experts (M=128; N=128 for hi|mid, 64
+//           for lo), N <= 64;
+//   CG = 2: a CTA pair per 256 tokens x 128 experts (cta_group::2, M=256;
+//           N=256 for hi|mid, 128 for lo): each CTA stages its own 128 tokens
+//           and 64 of the experts' weight columns, so each staged byte feeds
+//           twice the MMA work.
 // Every mbarrier wait is bounded (MOE_FLAG_WAIT_TIMEOUT).
 #include <algorithm>
 #include <mutex>
@@ -49,9 +56,14 @@ struct RtCfg {
   static constexpr int PART_BYTES = CHUNKS * CHUNK;           // one of hi / mid / lo
   static constexpr int STAGE_BYTES = A_BYTES + 3 * PART_BYTES;
   static constexpr int STAGES = STAGE_BYTES <= 40 * 1024 ? 5 : 3;
-  static constexpr int TMEM_COLS = BN;                        // power of two >= 32
-  static constexpr uint32_t IDESC = idesc_bf16_f32(BM * CG, BN, 1);
-  static_assert(COLS % 64 == 0, "weight columns per CTA are whole 64-column chunks");
+  // accumulators: x*hi and x*mid side by side (one MMA over the adjacent hi and
+  // mid chunks, 2*BN columns), then x*lo (BN columns)
+  static constexpr int LO_COL = 2 * BN;
+  static constexpr int TMEM_COLS = 3 * BN <= 256 ? 256 : 512;  // power of two >= 3*BN
+  static constexpr uint32_t IDESC_HM = idesc_bf16_f32(BM * CG, 2 * BN, 1);
+  static constexpr uint32_t IDESC_LO = idesc_bf16_f32(BM * CG, BN, 1);
+  static_assert(COLS == 64, "one 64-column chunk per part per CTA: hi and mid adjacent");
+  static_assert(2 * BN <= 256, "the hi|mid MMA is at most 256 columns wide");
 };
 
 struct RtTail {
@@ -209,17 +221,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t sa = smem_addr(base + stage * C::STAGE_BYTES);
 #pragma unroll
-        for (int part = 0; part < 3; ++part)
-#pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t adesc = smem_desc_sw128(sa + kk * 32, 16, 1024);
-            const uint64_t bdesc = smem_desc_sw128(sa + A_BYTES + part * C::PART_BYTES + kk * 2048, CHUNK, 1024);
-            const uint32_t acc = (kb | part | kk) != 0 ? 1u : 0u;
-            if (CG == 2)
-              tc_mma_f16_pair(tmem, adesc, bdesc, C::IDESC, acc);
-            else
-              tc_mma_f16(tmem, adesc, bdesc, C::IDESC, acc);
+        for (int kk = 0; kk < BK / 16; ++kk) {
+          const uint64_t adesc = smem_desc_sw128(sa + kk * 32, 16, 1024);
+          // the hi and mid chunks are adjacent: one MMA over both (chunk stride CHUNK)
+          const uint64_t bdesc_hm = smem_desc_sw128(sa + A_BYTES + kk * 2048, CHUNK, 1024);
+          const uint64_t bdesc_lo = smem_desc_sw128(sa + A_BYTES + 2 * C::PART_BYTES + kk * 2048, CHUNK, 1024);
+          const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
+          if (CG == 2) {
+            tc_mma_f16_pair(tmem, adesc, bdesc_hm, C::IDESC_HM, acc);
+            tc_mma_f16_pair(tmem + C::LO_COL, adesc, bdesc_lo, C::IDESC_LO, acc);
+          } else {
+            tc_mma_f16(tmem, adesc, bdesc_hm, C::IDESC_HM, acc);
+            tc_mma_f16(tmem + C::LO_COL, adesc, bdesc_lo, C::IDESC_LO, acc);
           }
+        }
         any = true;
         const uint32_t e = smem_addr(&tl.empty[stage]);
         if (CG == 2) {
@@ -253,11 +268,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
 #pragma unroll 1
       for (int c = 0; c < BN; c += 32) {
-        uint32_t v[32];
-        tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + c, v);
+        // experts c .. c+31 of the tile: CTA r of a pair staged experts 64r ..
+        // 64r+63, whose x*hi and x*mid sums are columns 128r + j and
+        // 128r + 64 + j of the hi|mid accumulator (j = expert mod 64); x*lo
+        // sums follow at LO_COL + expert
+        const uint32_t row = static_cast<uint32_t>(quad * 32) << 16;
+        const int hi_col = c + 64 * (c / 64);
+        uint32_t vh[32], vm[32], vl[32];
+        tmem_ld32(tmem + row + hi_col, vh);
+        tmem_ld32(tmem + row + hi_col + 64, vm);
+        tmem_ld32(tmem + row + C::LO_COL + c, vl);
         tmem_ld_wait();
+        // hi + (mid + lo): mid + lo is the exact product with the weight's low
+        // 16 bits whenever a logit is a single product, so that logit is the
+        // correctly rounded x * w
 #pragma unroll
-        for (int i = 0; i < 32; ++i) stg[lane * 33 + i] = __uint_as_float(v[i]);
+        for (int i = 0; i < 32; ++i)
+          stg[lane * 33 + i] =
+              __fadd_rn(__uint_as_float(vh[i]), __fadd_rn(__uint_as_float(vm[i]), __uint_as_float(vl[i])));
         __syncwarp();
         const int e = n0 + c + lane;
 #pragma unroll 4
