@@ -39,6 +39,7 @@
 #include <cuda_fp8.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdlib>
 #include <mutex>
 
@@ -87,6 +88,8 @@ struct MxParams {
   uint8_t* out8;             // SwiGLU: h codes [max_rows, n_out]
   uint8_t* out8_sf;          // SwiGLU: h scales (n_out / 32 per row)
   uint16_t* out16;           // plain: bf16 [max_rows, n_out]
+  uint64_t wait_ns;          // bound of the pipeline waits (those that also watch the abort flag);
+                             // the waits that drain copies and MMAs in flight keep kWaitLimitNs
   uint32_t* flags;
 };
 
@@ -244,7 +247,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int64_t sfb0_atom = (static_cast<int64_t>(tile.g) * NT + nt0) * KT;
         const int64_t sfb1_atom = (static_cast<int64_t>(tile.g) * NT + nt1) * KT;
         for (int kb = 0; kb < KT; ++kb) {
-          if (!mbar_wait(smem_addr(&tl.empty[stage]), phase ^ 1u, abort, p.flags, kFlagTimeout)) {
+          if (!mbar_wait(smem_addr(&tl.empty[stage]), phase ^ 1u, abort, p.flags, kFlagTimeout, p.wait_ns)) {
             ok = false;
             break;
           }
@@ -303,12 +306,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true, issued_any = false;
       for (int t = unit; ok && t < total; t += n_units, ++j) {
         // the previous tile's epilogue has read the columns this accumulator shares with it
-        if (j > 0 && !mbar_wait(smem_addr(&tl.drained), (j - 1) & 1u, abort, p.flags, kFlagTimeout)) break;
+        if (j > 0 && !mbar_wait(smem_addr(&tl.drained), (j - 1) & 1u, abort, p.flags, kFlagTimeout, p.wait_ns))
+          break;
         tc_fence_after();
         issued_any = true;
         const uint32_t d_tmem = tmem_base + (acc ? kAcc1Col : 0u);
         for (int kb = 0; kb < KT; ++kb) {
-          if (!mbar_wait(smem_addr(&tl.full[stage]), phase, abort, p.flags, kFlagTimeout)) {
+          if (!mbar_wait(smem_addr(&tl.full[stage]), phase, abort, p.flags, kFlagTimeout, p.wait_ns)) {
             ok = false;
             break;
           }
@@ -376,7 +380,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t acc = 0, acc_phase = 0;
     for (int t = unit; t < total; t += n_units) {
       const Tile tile = decode_tile(tl, G, BN, C::TILE_M, t);
-      if (!mbar_wait(smem_addr(&tl.tfull[acc]), acc_phase, abort, p.flags, kFlagTimeout)) break;
+      if (!mbar_wait(smem_addr(&tl.tfull[acc]), acc_phase, abort, p.flags, kFlagTimeout, p.wait_ns)) break;
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + (acc ? kAcc1Col : 0u);
       const int row = tile.m0 + r_in_tile;
@@ -551,6 +555,14 @@ cudaError_t launch_gemm(const CUtensorMap* maps, const MxParams& p, int64_t boun
 // the epilogue has read the 32 accumulator columns the two buffers share), not
 // the operand stream.  Single CTAs are the default; MOE_FFN_CTA_GROUP=1|2
 // forces one variant (tests run both).
+// Bound of the pipeline waits (moe_set_wait_limit_ns); 0 = kWaitLimitNs.
+std::atomic<uint64_t> g_mx_wait_ns{0};
+
+uint64_t mx_pipeline_wait_ns() {
+  const uint64_t v = g_mx_wait_ns.load(std::memory_order_relaxed);
+  return v == 0 ? kWaitLimitNs : v;
+}
+
 int choose_cta_group(const FfnMxArgs& a) {
   static int forced = [] {
     const char* v = std::getenv("MOE_FFN_CTA_GROUP");
@@ -570,6 +582,7 @@ cudaError_t launch_pair(const FfnMxArgs& a, const CUtensorMap& mA1, const CUtens
   p.G = a.G;
   p.max_rows = a.max_rows;
   p.flags = a.flags;
+  p.wait_ns = mx_pipeline_wait_ns();
   const int64_t m_bound = (a.max_rows + Cfg<CG>::TILE_M - 1) / Cfg<CG>::TILE_M + a.G;
   CUtensorMap maps[6];
   // GEMM1: K = d, n_out = f, h codes and scales out
@@ -611,6 +624,8 @@ cudaError_t launch_pair(const FfnMxArgs& a, const CUtensorMap& mA1, const CUtens
 }
 
 }  // namespace
+
+void set_mx_pipeline_wait_ns(uint64_t ns) { g_mx_wait_ns.store(ns, std::memory_order_relaxed); }
 
 cudaError_t launch_ffn_mx(const FfnMxArgs& a, cudaStream_t s) {
   if (a.max_rows <= 0 || a.G <= 0) return cudaSuccess;

@@ -156,3 +156,42 @@ def test_empty_layer():
     y, st, flags = gu.layer_fwd(dl)
     assert flags == 0 and y.shape == (0, 128)
     assert np.all(st["counts"] == 0) and np.all(st["kept"] == 0) and st["num_dropped"][0] == 0
+
+
+_OVERLAP_SCRIPT = r"""
+import sys
+sys.path.insert(0, {root!r})
+import numpy as np
+from expert_router_gemm_b200 import synth, moe
+from expert_router_gemm_b200.configs import Workload
+from tests import gpu_util as gu
+out = []
+for w in (Workload("ov-pairs", T=1536, d=512, N=8, k=2, f=384, f_shared=128, capacity_factor=1.1),
+          Workload("ov-single", T=1024, d=256, N=32, k=4, f=256, capacity_factor=1.25),
+          Workload("ov-f32", T=300, d=100, N=6, k=3, f=72, capacity_factor=1.25, dtype="f32")):
+    dl = moe.to_device(synth.make_inputs(w), moe.config_from_workload(w))
+    y, st, flags = gu.layer_fwd(dl)
+    assert flags == 0
+    out.append(y.view(np.uint8).tobytes())
+    out.append(b"".join(np.ascontiguousarray(st[k]).tobytes() for k in sorted(st)))
+import hashlib
+print("DIGEST", hashlib.sha256(b"".join(out)).hexdigest())
+"""
+
+
+def test_overlapped_launches_change_no_result():
+    """Kernels launched to overlap the end of their predecessor (the default)
+    give the same bytes as plain launches (MOE_PDL=0): layer outputs and every
+    statistic, for CTA-pair and single-CTA GEMMs and the fp32 layer."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    digests = []
+    for pdl in ("1", "0"):
+        env = dict(os.environ, MOE_PDL=pdl)
+        r = subprocess.run([sys.executable, "-c", _OVERLAP_SCRIPT.format(root=root)], env=env,
+                           capture_output=True, text=True, timeout=600)
+        assert r.returncode == 0, r.stdout + r.stderr
+        digests.append([l for l in r.stdout.splitlines() if l.startswith("DIGEST")][0])
+    assert digests[0] == digests[1]

@@ -54,3 +54,31 @@ def test_pipeline_wait_timeout_is_reported_and_the_next_call_is_correct(w):
     assert flags2 == 0 and staged["flags"] == 0
     np.testing.assert_array_equal(y2, staged["y"])
     compare_layer(inp, w, y2, staged["idx"], staged["row_map"], staged["logits"], tol=2e-2)
+
+
+def test_fp8_pipeline_wait_timeout_is_reported_and_the_next_call_is_correct():
+    """The same for the block-scaled FP8 grouped GEMM (single CTAs, the default
+    shape): a short bound makes its pipeline waits run out, the call returns
+    with MOE_FLAG_WAIT_TIMEOUT, and the next call with the default bound gives
+    the bytes the layer gave before."""
+    w = Workload("timeout-mx", T=2048, d=1024, N=8, k=2, f=1024, capacity_factor=1.25)
+    inp = synth.make_inputs(w)
+    cfg = moe.config_from_workload(w, gemm="mxfp8")
+    dl = moe.to_device(inp, cfg)
+    dl.quantize_mx()
+    before, _, f0 = gu.layer_fwd(dl)
+    assert f0 == 0
+    lb, _, _ = moe.moe_workspace_size(cfg)
+    ws = torch.empty(lb, dtype=torch.uint8, device="cuda")
+    y = torch.zeros((w.T, w.d), dtype=moe.act_dtype(cfg), device="cuda")
+    moe.moe_set_wait_limit_ns(SHORT_NS)
+    try:
+        moe.moe_layer_fwd(cfg, dl.weights(), dl.x, y, None, ws)
+        flags = moe.moe_read_flags(ws)
+    finally:
+        moe.moe_set_wait_limit_ns(0)
+    assert flags & moe.MOE_FLAG_WAIT_TIMEOUT, f"flags {flags:#x}"
+    assert torch.cuda.synchronize() is None
+    after, _, f1 = gu.layer_fwd(dl)
+    assert f1 == 0
+    np.testing.assert_array_equal(after, before)
