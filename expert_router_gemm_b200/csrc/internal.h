@@ -183,8 +183,9 @@ struct FfnMxArgs {
   uint32_t* flags;
 };
 cudaError_t launch_ffn_mx(const FfnMxArgs& a, cudaStream_t s);
-// The same bound for the block-scaled FP8 grouped GEMM.
+// The same bound for the block-scaled FP8 grouped GEMM, and for the router GEMM.
 void set_mx_pipeline_wait_ns(uint64_t ns);
+void set_router_wait_ns(uint64_t ns);
 
 // Quantize G weights [G][K][N] (bf16, N contiguous) to K-major FP8 codes
 // [G][N][K] and scale bytes [G][N/128][K/128][512]; K, N multiples of 128.

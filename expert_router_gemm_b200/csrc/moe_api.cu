@@ -882,6 +882,7 @@ moe_status_t moe_set_wait_limit_ns(uint64_t ns) {
   if (ns > 2000000000ull) return MOE_ERR_INVALID_ARG;
   set_pipeline_wait_ns(ns);
   set_mx_pipeline_wait_ns(ns);
+  set_router_wait_ns(ns);
   return MOE_OK;
 }
 

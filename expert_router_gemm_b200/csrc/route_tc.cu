@@ -35,6 +35,7 @@
 //           twice the MMA work.
 // Every mbarrier wait is bounded (MOE_FLAG_WAIT_TIMEOUT).
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "device_utils.cuh"
@@ -84,8 +85,13 @@ struct RtParams {
   int N, d;
   int kb_per_split;    // K slabs per split (blockIdx.z = split)
   float* partials;     // [splits][T, N]: split z writes partials + z * T * N
+  uint64_t wait_ns;    // bound of the pipeline waits (those that also watch the abort flag);
+                       // the waits that drain copies and MMAs in flight keep kWaitLimitNs
   uint32_t* flags;
 };
+
+// Bound of the pipeline waits (moe_set_wait_limit_ns); 0 = kWaitLimitNs.
+std::atomic<uint64_t> g_router_wait_ns{0};
 
 // W_r fp32 [d, N] -> three bf16 slabs [3][d][NP] (columns N..NP-1 zero).
 // Block (32, 8): threadIdx.y picks one of 8 rows, a thread splits 4 adjacent
@@ -169,7 +175,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       uint32_t stage = 0, phase = 0, issued = 0, last_par = 0;
       for (int kb = 0; kb < KB; ++kb) {
-        if (!mbar_wait(smem_addr(&tl.empty[stage]), phase ^ 1u, abort, p.flags, kFlagTimeout)) break;
+        if (!mbar_wait(smem_addr(&tl.empty[stage]), phase ^ 1u, abort, p.flags, kFlagTimeout, p.wait_ns)) break;
         const uint32_t fb_local = smem_addr(&tl.full[stage]);
         const uint32_t sa = smem_addr(base + stage * C::STAGE_BYTES);
         if (CG == 1) {
@@ -214,7 +220,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t stage = 0, phase = 0;
       bool ok = true, any = false;
       for (int kb = 0; kb < KB; ++kb) {
-        if (!mbar_wait(smem_addr(&tl.full[stage]), phase, abort, p.flags, kFlagTimeout)) {
+        if (!mbar_wait(smem_addr(&tl.full[stage]), phase, abort, p.flags, kFlagTimeout, p.wait_ns)) {
           ok = false;
           break;
         }
@@ -264,7 +270,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // has completed) so that the global stores are whole 128-byte row pieces.
     const int quad = warp & 3;
     float* stg = reinterpret_cast<float*>(base) + quad * 32 * 33;  // 32 x 33 words: conflict-free both ways
-    if (KB > 0 && mbar_wait(smem_addr(&tl.tfull), 0u, abort, p.flags, kFlagTimeout)) {
+    if (KB > 0 && mbar_wait(smem_addr(&tl.tfull), 0u, abort, p.flags, kFlagTimeout, p.wait_ns)) {
       tc_fence_after();
 #pragma unroll 1
       for (int c = 0; c < BN; c += 32) {
@@ -353,6 +359,8 @@ int split_width(int N) { return N > 64 ? (N + 127) / 128 * 128 : (N + 63) / 64 *
 
 int router_split_width(int N) { return split_width(N); }
 
+void set_router_wait_ns(uint64_t ns) { g_router_wait_ns.store(ns, std::memory_order_relaxed); }
+
 size_t router_split_bytes(int d, int N) { return 3ull * d * split_width(N) * sizeof(uint16_t); }
 
 cudaError_t launch_router_split(const float* w_router, int d, int N, void* split, cudaStream_t s) {
@@ -384,7 +392,8 @@ cudaError_t launch_router_tc(const RouteArgs& a, const void* split, bool make_sp
   const int kbs = (kb_total + splits - 1) / splits;
   splits = (kb_total + kbs - 1) / kbs;  // every split has at least one slab
   *n_partials = splits;
-  RtParams p{a.T, a.N, a.d, kbs, partials, a.flags};
+  const uint64_t w = g_router_wait_ns.load(std::memory_order_relaxed);
+  RtParams p{a.T, a.N, a.d, kbs, partials, w == 0 ? kWaitLimitNs : w, a.flags};
   if (pairs) return launch_tile<128, 2>(mx, mw, p, splits, s);
   return launch_tile<64, 1>(mx, mw, p, splits, s);
 }

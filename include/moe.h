@@ -428,9 +428,10 @@ moe_status_t moe_layer_bwd(const moe_config_t* cfg, const moe_weights_t* weights
 
 /*
  * moe_set_wait_limit_ns - failure handling (the pages define no such call):
- * the time bound of the grouped GEMMs' pipeline waits (bf16 and block-scaled
- * FP8: a stage's operands, a free stage, an accumulator) for kernels launched
- * after this call, process wide.  ns = 0 restores the default of 2 s, within which every legitimate wait
+ * the time bound of the pipeline waits of the tensor-core GEMMs (the bf16 and
+ * block-scaled FP8 grouped GEMMs and the router GEMM: a stage's operands, a
+ * free stage, an accumulator) for kernels launched after this call, process
+ * wide.  ns = 0 restores the default of 2 s, within which every legitimate wait
  * ends; a shorter bound makes those waits run out on purpose, which is how the
  * timeout path is tested: the kernel then raises MOE_FLAG_WAIT_TIMEOUT, still
  * waits (with the default bound) for the copies and MMAs it has in flight,

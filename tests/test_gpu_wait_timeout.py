@@ -82,3 +82,35 @@ def test_fp8_pipeline_wait_timeout_is_reported_and_the_next_call_is_correct():
     after, _, f1 = gu.layer_fwd(dl)
     assert f1 == 0
     np.testing.assert_array_equal(after, before)
+
+
+def test_router_pipeline_wait_timeout_is_reported_and_the_next_call_is_correct():
+    """The tensor-core router GEMM (CTA pairs, K split) under the short bound:
+    moe_route returns with MOE_FLAG_WAIT_TIMEOUT, and with the default bound
+    again it gives the routing it gave before, bit for bit."""
+    w = Workload("timeout-router", T=4096, d=2048, N=128, k=8, f=128, capacity_factor=1.0)
+    inp = synth.make_inputs(w, experts=False)
+    cfg = moe.config_from_workload(w)
+    x, wr = gu.cuda_tensor(inp.x), gu.cuda_tensor(inp.w_router)
+
+    def route():
+        idx = torch.full((w.T, w.k), -7, dtype=torch.int32, device="cuda")
+        wt = torch.full((w.T, w.k), float("nan"), dtype=torch.float32, device="cuda")
+        ws = gu.op_workspace(cfg)
+        moe.moe_route(cfg, x, wr, None, None, None, idx, wt, None, ws)
+        flags = moe.moe_read_flags(ws)
+        return gu.host(idx), gu.host(wt), flags
+
+    idx0, wt0, f0 = route()
+    assert f0 == 0
+    moe.moe_set_wait_limit_ns(SHORT_NS)
+    try:
+        _, _, flags = route()
+    finally:
+        moe.moe_set_wait_limit_ns(0)
+    assert flags & moe.MOE_FLAG_WAIT_TIMEOUT, f"flags {flags:#x}"
+    assert torch.cuda.synchronize() is None
+    idx1, wt1, f1 = route()
+    assert f1 == 0
+    np.testing.assert_array_equal(idx1, idx0)
+    np.testing.assert_array_equal(wt1, wt0)
