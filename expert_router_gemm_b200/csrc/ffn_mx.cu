@@ -549,12 +549,6 @@ cudaError_t launch_gemm(const CUtensorMap* maps, const MxParams& p, int64_t boun
   return cudaGetLastError();
 }
 
-// CTA pairs halve the B operand each SM stages, but measured no faster here
-// (Qwen3-shaped layer: 1.32 vs 1.23-1.32 ms; tensor pipe 52 % vs 58 % busy):
-// the limit is the hand-over between tiles (the next tile's MMA waits until
-// the epilogue has read the 32 accumulator columns the two buffers share), not
-// the operand stream.  Single CTAs are the default; MOE_FFN_CTA_GROUP=1|2
-// forces one variant (tests run both).
 // Bound of the pipeline waits (moe_set_wait_limit_ns); 0 = kWaitLimitNs.
 std::atomic<uint64_t> g_mx_wait_ns{0};
 
@@ -563,6 +557,12 @@ uint64_t mx_pipeline_wait_ns() {
   return v == 0 ? kWaitLimitNs : v;
 }
 
+// CTA pairs halve the B operand each SM stages, but measured no faster here
+// (Qwen3-shaped layer: 1.32 vs 1.23-1.32 ms; tensor pipe 52 % vs 58 % busy):
+// the limit is the hand-over between tiles (the next tile's MMA waits until
+// the epilogue has read the 32 accumulator columns the two buffers share), not
+// the operand stream.  Single CTAs are the default; MOE_FFN_CTA_GROUP=1|2
+// forces one variant (tests run both).
 int choose_cta_group(const FfnMxArgs& a) {
   static int forced = [] {
     const char* v = std::getenv("MOE_FFN_CTA_GROUP");
