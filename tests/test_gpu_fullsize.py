@@ -31,7 +31,19 @@ SAMPLE = 1024   # tokens of each full-size layer whose outputs the oracle recomp
 @pytest.mark.parametrize("name", ["tiny-fp32", "mixtral-8x7b-shaped", "qwen3-moe-shaped",
                                   "deepseek-v3-shaped", "skewed-stress"])
 def test_full_size_layer(name):
-    w = configs.get(name)
+    _check_full_size(configs.get(name))
+
+
+def test_large_batch_layer():
+    """The Qwen3-shaped layer at T = 65536: 0.52 M kept rows, so the permuted
+    rows (4.4 GB) and expert outputs lie beyond 32-bit byte offsets, and the
+    segment table, the tile lists and the combine run at eight times the bench
+    batch."""
+    _check_full_size(configs.QWEN3.scaled(65536))
+
+
+def _check_full_size(w):
+    name = w.name
     inp = synth.make_inputs(w)
     cfg = moe.config_from_workload(w)
     dl = moe.to_device(inp, cfg)
