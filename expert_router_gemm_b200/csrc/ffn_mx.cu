@@ -304,6 +304,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---------------------------------------------------------------- MMA issuer
       uint32_t stage = 0, phase = 0, acc = 0, j = 0, sfset = 0;
       bool ok = true, issued_any = false;
+      // Descriptors of stage 0 at K offset 0.  Their start-address field is the
+      // shared address / 16 (14 bits, no carry below 256 KB), so a stage or a
+      // 32-byte K step is a constant added to the descriptor: this thread's
+      // instruction stream per K stage stays short next to the MMAs it feeds.
+      const uint64_t adesc0 = smem_desc_sw128(smem_addr(sA), 16, 1024);
+      const uint64_t bdesc0 = smem_desc_sw128(smem_addr(sB), 16, 1024);
+      const uint64_t sfdesc0 = smem_desc_plain(smem_addr(sSF), 16, 128);
       for (int t = unit; ok && t < total; t += n_units, ++j) {
         // the previous tile's epilogue has read the columns this accumulator shares with it
         if (j > 0 && !mbar_wait(smem_addr(&tl.drained), (j - 1) & 1u, abort, p.flags, kFlagTimeout, p.wait_ns))
@@ -317,28 +324,29 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t a_addr = smem_addr(sA + stage * A_BYTES);
-          const uint32_t b_addr = smem_addr(sB + stage * C::B_BYTES);
-          const uint32_t sf_addr = smem_addr(sSF + stage * SF_BYTES);
+          const uint64_t adesc_s = adesc0 + stage * static_cast<uint32_t>(A_BYTES >> 4);
+          const uint64_t bdesc_s = bdesc0 + stage * static_cast<uint32_t>(C::B_BYTES >> 4);
+          const uint64_t sfdesc_s = sfdesc0 + stage * static_cast<uint32_t>(SF_BYTES >> 4);
           // scale atoms -> this stage's TMEM scale set (executed in order with
           // the MMAs issued around them)
           const uint32_t sfa_col = tmem_base + kSfaCol + sfset * kSfSet;
           const uint32_t sfb_col = tmem_base + kSfbCol + sfset * kSfSet;
           sfset ^= 1u;
+          constexpr uint32_t kAtom16 = SF_ATOM >> 4;
           if (CG == 2) {
-            tc_cp_32x128b_x4_pair(sfa_col, smem_desc_plain(sf_addr, 16, 128));
-            tc_cp_32x128b_x4_pair(sfb_col, smem_desc_plain(sf_addr + SF_ATOM, 16, 128));
-            tc_cp_32x128b_x4_pair(sfb_col + 4, smem_desc_plain(sf_addr + 2 * SF_ATOM, 16, 128));
+            tc_cp_32x128b_x4_pair(sfa_col, sfdesc_s);
+            tc_cp_32x128b_x4_pair(sfb_col, sfdesc_s + kAtom16);
+            tc_cp_32x128b_x4_pair(sfb_col + 4, sfdesc_s + 2 * kAtom16);
           } else {
-            tc_cp_32x128b_x4(sfa_col, smem_desc_plain(sf_addr, 16, 128));
-            tc_cp_32x128b_x4(sfb_col, smem_desc_plain(sf_addr + SF_ATOM, 16, 128));
-            tc_cp_32x128b_x4(sfb_col + 4, smem_desc_plain(sf_addr + 2 * SF_ATOM, 16, 128));
+            tc_cp_32x128b_x4(sfa_col, sfdesc_s);
+            tc_cp_32x128b_x4(sfb_col, sfdesc_s + kAtom16);
+            tc_cp_32x128b_x4(sfb_col + 4, sfdesc_s + 2 * kAtom16);
           }
 #pragma unroll
           for (int kk = 0; kk < BK / MMA_K; ++kk) {
             // A and B K-major: advance 32 values (32 bytes) inside the swizzle row
-            const uint64_t adesc = smem_desc_sw128(a_addr + kk * 32, 16, 1024);
-            const uint64_t bdesc = smem_desc_sw128(b_addr + kk * 32, 16, 1024);
+            const uint64_t adesc = adesc_s + static_cast<uint64_t>(kk * 2);
+            const uint64_t bdesc = bdesc_s + static_cast<uint64_t>(kk * 2);
             const uint32_t sel = static_cast<uint32_t>(kk) << 30;   // scale byte kk of each word
             const uint32_t idesc = idesc_mxf8(C::TILE_M, MMA_N, static_cast<uint32_t>(kk));
             if (CG == 2)
