@@ -422,6 +422,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---------------------------------------------------------------- MMA issuer
       uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
       bool ok = true, issued_any = false;
+      // Descriptors of stage 0 at K offset 0.  Their start-address field is the
+      // shared address / 16 (14 bits, no carry below 256 KB), so a stage or a K
+      // step is a constant added to the descriptor: this thread's instruction
+      // stream per K stage stays short next to the MMAs it feeds.
+      const uint64_t adesc0 = smem_desc_sw128(smem_addr(sA), 16, 1024);
+      const uint64_t bdesc0 = smem_desc_sw128(smem_addr(sB), B_CHUNK, 1024);
       for (int t = unit; ok && t < total; t += n_units) {
         if (!mbar_wait(smem_addr(&tl.tempty[acc]), acc_phase ^ 1u, abort, p.flags, kFlagTimeout, p.wait_ns)) break;
         tc_fence_after();
@@ -437,14 +443,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (lsu_a) fence_proxy_async_smem();   // cp.async (generic proxy) writes -> MMA operand reads
           tc_fence_after();
-          const uint32_t a_addr = smem_addr(sA + stage * A_BYTES);
-          const uint32_t b_addr = smem_addr(sB + stage * C::B_BYTES);
+          const uint64_t adesc_s = adesc0 + stage * static_cast<uint32_t>(A_BYTES >> 4);
+          const uint64_t bdesc_s = bdesc0 + stage * static_cast<uint32_t>(C::B_BYTES >> 4);
 #pragma unroll
           for (int kk = 0; kk < BK / MMA_K; ++kk) {
             // A: K-major, advance 16 elements (32 bytes) inside the swizzle row
-            const uint64_t adesc = smem_desc_sw128(a_addr + kk * 32, 16, 1024);
+            const uint64_t adesc = adesc_s + static_cast<uint64_t>(kk * (32 >> 4));
             // B: MN-major, advance 16 K rows = two 8-row swizzle atoms (2048 bytes)
-            const uint64_t bdesc = smem_desc_sw128(b_addr + kk * 2048, B_CHUNK, 1024);
+            const uint64_t bdesc = bdesc_s + static_cast<uint64_t>(kk * (2048 >> 4));
             if (CG == 2)
               tc_mma_f16_pair(d_tmem, adesc, bdesc, C::IDESC, (kb | kk) != 0 ? 1u : 0u);
             else
