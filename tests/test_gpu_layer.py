@@ -38,6 +38,8 @@ SMALL = [
     # generic slot loop), the latter with a shared expert
     Workload("top32-bf16", T=512, d=256, N=64, k=32, f=128, capacity_factor=1.25),
     Workload("top3-shared-bf16", T=600, d=192, N=12, k=3, f=192, f_shared=64, capacity_factor=1.0),
+    # the largest expert count with the largest top-k
+    Workload("n256-top32-bf16", T=256, d=128, N=256, k=32, f=64, capacity_factor=1.25),
 ]
 
 F32 = [
