@@ -552,7 +552,9 @@ def main():
 
         def staged(evs):
             evs[0].record(stream)
-            moe.moe_route(cfg, dl.x, dl.w_router, dl.bias, dl.selection_bias, None, idx, wt, stats, ws_op, stream)
+            # the layer's routing as moe_layer_fwd runs it: with the split made once
+            moe.moe_route_with_split(cfg, dl.x, dl.w_router, dl.router_split, dl.bias, dl.selection_bias, None,
+                                     idx, wt, stats, ws_op, stream)
             evs[1].record(stream)
             if mx:
                 moe.moe_dispatch_mx(cfg, dl.x, idx, row_map, seg_off, seg_count, x8, x8sf, stats, ws_op,

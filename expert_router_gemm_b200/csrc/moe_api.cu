@@ -524,6 +524,21 @@ moe_status_t moe_route(const moe_config_t* cfg, const void* x, const float* w_ro
                   reinterpret_cast<cudaStream_t>(stream));
 }
 
+moe_status_t moe_route_with_split(const moe_config_t* cfg, const void* x, const float* w_router,
+                                  const void* w_router_split, const float* router_bias, const float* selection_bias,
+                                  float* logits_out, int32_t* topk_idx, float* topk_w, moe_stats_t* stats, void* ws,
+                                  size_t ws_bytes, moe_stream_t stream) {
+  Dims D;
+  moe_status_t s = derive(cfg, &D);
+  if (s != MOE_OK) return s;
+  if (D.T > 0 && (x == nullptr || w_router == nullptr || topk_idx == nullptr || topk_w == nullptr))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_router_split)) return MOE_ERR_MISALIGNED;
+  if ((s = check_ws(ws, ws_bytes, layout(D).op_end)) != MOE_OK) return s;
+  return do_route(D, x, w_router, router_bias, selection_bias, nullptr, logits_out, topk_idx, topk_w, stats, ws,
+                  reinterpret_cast<cudaStream_t>(stream), D.bf16 ? w_router_split : nullptr);
+}
+
 moe_status_t moe_route_from_logits(const moe_config_t* cfg, const float* logits, const float* selection_bias,
                                    int32_t* topk_idx, float* topk_w, moe_stats_t* stats, void* ws,
                                    size_t ws_bytes, moe_stream_t stream) {

@@ -68,6 +68,8 @@ _PROTOS = {
                                           ctypes.POINTER(_SZ), ctypes.POINTER(ctypes.c_int64)]),
     "moe_route": (ctypes.c_int, [ctypes.POINTER(moe_config_t), _P, _P, _P, _P, _P, _P, _P,
                                  ctypes.POINTER(moe_stats_t), _P, _SZ, _P]),
+    "moe_route_with_split": (ctypes.c_int, [ctypes.POINTER(moe_config_t), _P, _P, _P, _P, _P, _P, _P, _P,
+                                            ctypes.POINTER(moe_stats_t), _P, _SZ, _P]),
     "moe_route_from_logits": (ctypes.c_int, [ctypes.POINTER(moe_config_t), _P, _P, _P, _P,
                                              ctypes.POINTER(moe_stats_t), _P, _SZ, _P]),
     "moe_bias_update": (ctypes.c_int, [ctypes.POINTER(moe_config_t), _P, _P, ctypes.c_float, _P]),
@@ -210,6 +212,15 @@ def moe_route(cfg, x, w_router, router_bias, selection_bias, logits_out, topk_id
            "moe_route")
 
 
+def moe_route_with_split(cfg, x, w_router, w_router_split, router_bias, selection_bias, logits_out, topk_idx,
+                         topk_w, stats, ws, stream=None):
+    _check(_lib.moe_route_with_split(ctypes.byref(cfg), _ptr(x), _ptr(w_router), _ptr(w_router_split),
+                                     _ptr(router_bias), _ptr(selection_bias), _ptr(logits_out),
+                                     _ptr(topk_idx), _ptr(topk_w), _stats_ref(stats), _ptr(ws),
+                                     ws.numel() if ws is not None else 0, _stream(stream)),
+           "moe_route_with_split")
+
+
 def moe_route_from_logits(cfg, logits, selection_bias, topk_idx, topk_w, stats, ws, stream=None):
     _check(_lib.moe_route_from_logits(ctypes.byref(cfg), _ptr(logits), _ptr(selection_bias),
                                       _ptr(topk_idx), _ptr(topk_w), _stats_ref(stats), _ptr(ws),
@@ -336,7 +347,8 @@ def moe_router_split(w_router, d: int, N: int, split, stream=None) -> None:
 
 
 def moe_set_wait_limit_ns(ns: int) -> None:
-    """Bound of the bf16 grouped GEMM's pipeline waits for later launches (0: the 2 s default)."""
+    """Bound of the pipeline waits of later launches of the tensor-core kernels
+    (bf16 and FP8 grouped GEMMs, router GEMM); 0: the 2 s default."""
     _check(_lib.moe_set_wait_limit_ns(int(ns)), "moe_set_wait_limit_ns")
 
 

@@ -194,6 +194,25 @@ moe_status_t moe_route(const moe_config_t* cfg, const void* x, const float* w_ro
                        size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * moe_route_with_split - moe_route with the bf16 split of the router weight
+ * made beforehand by moe_router_split (see there), as moe_layer_fwd takes it in
+ * moe_weights_t.w_router_split: the same computation ("MoE 训练加速实战" §2.2,
+ * g = x W_r with the router in fp32) and the same results, byte for byte,
+ * without the per-call split of W_r.
+ *   w_router_split  device, 16-byte aligned, the split of this w_router for
+ *                   cfg's d and N (moe_router_split_bytes); owned by the caller,
+ *                   read only.  NULL: moe_route exactly.  fp32 layers (no
+ *                   tensor-core router) ignore it.
+ * All other arguments and errors as moe_route; a misaligned split gives
+ * MOE_ERR_MISALIGNED.
+ */
+moe_status_t moe_route_with_split(const moe_config_t* cfg, const void* x, const float* w_router,
+                                  const void* w_router_split, const float* router_bias,
+                                  const float* selection_bias, float* logits_out, int32_t* topk_idx,
+                                  float* topk_w, moe_stats_t* stats, void* ws, size_t ws_bytes,
+                                  moe_stream_t stream);
+
+/*
  * moe_route_from_logits - the same softmax / top-k / weights / statistics as
  * moe_route, starting from caller-supplied fp32 logits [T, N] (no GEMM), with
  * an optional selection_bias [N] as in moe_route.  This is the entry point on

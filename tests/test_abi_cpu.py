@@ -124,6 +124,23 @@ def test_route_argument_validation():
     assert _route_status(bad, ws_bytes=1 << 20) == INVALID
 
 
+def test_route_with_split_argument_validation():
+    # the same checks as moe_route, plus the split's alignment (never dereferenced here)
+    cfg = moe.make_config(T=256, d=128, N=128, k=8, f=256, capacity_factor=1.0, dtype="bf16")
+    ob = moe.moe_workspace_size(cfg)[1]
+
+    def call(x=0x10000, split=0x60000, idx=0x30000, ws=0x50000, ws_bytes=ob):
+        return moe.raw_call("moe_route_with_split", ctypes.byref(cfg), x, 0x20000, split, None, None, None,
+                            idx, 0x40000, None, ws, ctypes.c_size_t(ws_bytes), None)
+
+    assert call(split=0x60008) == MISAL
+    assert call(x=None) == INVALID
+    assert call(idx=None) == INVALID
+    assert call(x=0x10008) == MISAL
+    assert call(ws_bytes=16) == WS
+    assert call(ws=None) == WS
+
+
 def test_bias_update_argument_validation():
     cfg = moe.make_config(T=256, d=128, N=8, k=2, f=256, capacity_factor=1.25)
     f = ctypes.c_float

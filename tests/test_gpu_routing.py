@@ -276,3 +276,48 @@ def test_layer_with_a_router_split_made_once_is_unchanged():
     np.testing.assert_array_equal(y0, y1)
     for key in st0:
         np.testing.assert_array_equal(st0[key], st1[key], err_msg=key)
+
+
+@pytest.mark.parametrize("T,d,N,k,bias,sel,dtype", [
+    (300, 256, 8, 2, True, False, "bf16"),       # 64-expert tiles, K split four ways
+    (8192, 4096, 128, 8, False, False, "bf16"),  # the Qwen3-shaped router: CTA pairs
+    (1000, 512, 100, 6, True, True, "bf16"),     # ragged N, selection bias
+    (640, 7168, 256, 8, True, False, "bf16"),    # N = 256: two 128-expert column tiles
+    (256, 128, 8, 2, True, False, "f32"),        # fp32 layer: no tensor-core router, split ignored
+])
+def test_route_with_split_matches_route(T, d, N, k, bias, sel, dtype):
+    """moe_route_with_split, given the split that moe_router_split made once,
+    writes the bytes that moe_route writes: logits, indices, weights and every
+    statistic."""
+    if dtype == "bf16":
+        x = synth.f32_to_bf16_bits(synth.normal_f32(12, 1, (T, d)))
+    else:
+        x = synth.normal_f32(12, 1, (T, d))
+    wr = synth.normal_f32(12, 2, (d, N)) * np.float32(1 / np.sqrt(d))
+    b = gu.cuda_tensor(synth.normal_f32(12, 3, (N,))) if bias else None
+    sb = gu.cuda_tensor(synth.make_selection_bias(12, N)) if sel else None
+    cfg = moe.make_config(T=T, d=d, N=N, k=k, f=64, capacity_factor=1.0, dtype=dtype)
+    xd, wrd = gu.cuda_tensor(x), gu.cuda_tensor(wr)
+    split = torch.empty(moe.moe_router_split_bytes(d, N), dtype=torch.uint8, device="cuda")
+    moe.moe_router_split(wrd, d, N, split)
+
+    def run(with_split):
+        logits = torch.full((T, N), float("nan"), device="cuda")
+        idx = torch.full((T, k), -1, dtype=torch.int32, device="cuda")
+        wt = torch.full((T, k), float("nan"), device="cuda")
+        ws = gu.op_workspace(cfg)
+        bufs, st = gu.new_stats(N)
+        if with_split:
+            moe.moe_route_with_split(cfg, xd, wrd, split, b, sb, logits, idx, wt, st, ws)
+        else:
+            moe.moe_route(cfg, xd, wrd, b, sb, logits, idx, wt, st, ws)
+        assert moe.moe_read_flags(ws) == 0
+        return gu.host(logits), gu.host(idx), gu.host(wt), gu.stats_host(bufs)
+
+    lg0, idx0, wt0, st0 = run(False)
+    lg1, idx1, wt1, st1 = run(True)
+    np.testing.assert_array_equal(lg1, lg0)
+    np.testing.assert_array_equal(idx1, idx0)
+    np.testing.assert_array_equal(wt1, wt0)
+    for key in ("y_frac", "z_mean", "l_aux_p3", "l_aux_switch", "counts", "z_loss", "load_std", "top2_ratio"):
+        np.testing.assert_array_equal(st1[key], st0[key], err_msg=key)
