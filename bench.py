@@ -49,20 +49,35 @@ FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
 # A timed region at least this long has run into the power limiter's steady
-# state; shorter regions run at the burst clock.
+# state; shorter regions run at the burst clock unless their clock record says
+# otherwise (below).
 SUSTAINED_REGION_S = 2.0
+# A region whose sampled SM clock has a median below this fraction of the
+# maximum, with the power cap active, ran in the limiter's steady state too.
+CAPPED_CLOCK_FRAC = 0.75
+MIN_CLOCK_SAMPLES = 5
 
 
-def choose_tensor_peak(peaks, region_s: float):
+def choose_tensor_peak(peaks, region_s: float, clocks=None):
     """The measured bf16 tensor-core peak that matches how a kernel was timed:
-    the burst figure (a cuBLAS GEMM timed alone) for a region shorter than
-    SUSTAINED_REGION_S seconds, the sustained figure (a seconds-long loop under
-    the power cap) for a longer one.  Returns (peak, key, reason)."""
+    the sustained figure (a seconds-long loop under the power cap) when the
+    region lasted SUSTAINED_REGION_S seconds or more, or when its clock record
+    (`clocks`, a ClockSampler summary: at least MIN_CLOCK_SAMPLES samples) shows
+    the power cap active with the median SM clock below CAPPED_CLOCK_FRAC of the
+    maximum; the burst figure (a cuBLAS GEMM timed alone) otherwise.
+    Returns (peak, key, reason)."""
     if region_s >= SUSTAINED_REGION_S:
         return (peaks["bf16_tflops_sustained"], "bf16_tflops_sustained",
                 f"timed region {region_s:.2f} s >= {SUSTAINED_REGION_S:.0f} s: sustained (power-capped) peak")
+    c = clocks or {}
+    mhz, max_mhz = c.get("sm_mhz"), c.get("sm_max_mhz")
+    if (mhz and max_mhz and c.get("samples", 0) >= MIN_CLOCK_SAMPLES and "sw_power_cap" in c.get("reasons", ())
+            and mhz < CAPPED_CLOCK_FRAC * max_mhz):
+        return (peaks["bf16_tflops_sustained"], "bf16_tflops_sustained",
+                f"timed region {region_s:.3f} s ran power-capped (median SM clock {mhz:.0f} of {max_mhz:.0f} MHz, "
+                f"sw_power_cap, {c['samples']} samples): sustained peak")
     return (peaks["bf16_tflops"], "bf16_tflops",
-            f"timed region {region_s:.3f} s < {SUSTAINED_REGION_S:.0f} s: burst peak")
+            f"timed region {region_s:.3f} s < {SUSTAINED_REGION_S:.0f} s at the burst clock: burst peak")
 
 
 def cpu_model() -> str:
@@ -601,8 +616,8 @@ def main():
 
         peaks, peak_src = load_peaks()
         hbm = peaks["hbm_gbs"]
-        # the stage times come from region B: its length decides burst vs sustained
-        tc_peak, tc_key, tc_reason = choose_tensor_peak(peaks, region_b_s)
+        # the stage times come from region B: its length and clocks decide burst vs sustained
+        tc_peak, tc_key, tc_reason = choose_tensor_peak(peaks, region_b_s, clocks_b)
         # the FP8 GEMM's peak: the measured bf16 figure times the nominal FP8 : bf16
         # dense ratio (4.5 : 2.25 PFLOP/s)
         gemm_peak = 2.0 * tc_peak if mx else tc_peak
@@ -819,14 +834,15 @@ def main():
         # and weight gradients (6 d f), plus the shared expert's 2 + 4 + 6 d fs per token
         gemm_fl = 18.0 * d * f * a_kept + (12.0 + 6.0) * T * d * fs
         peaks, peak_src = load_peaks()
-        b_peak, b_key, b_reason = choose_tensor_peak(peaks, bms * n_b / 1e3)
+        b_clocks = bsampler.summary()
+        b_peak, b_key, b_reason = choose_tensor_peak(peaks, bms * n_b / 1e3, b_clocks)
         line["backward"] = {
             "what": "moe_layer_bwd: forward recomputed from x, then dx and every weight gradient (fp32)",
             "steps": n_b, "ms_per_step": round(bms, 4), "tokens/s": round(world * T / (bms / 1e3), 1),
             "gemm_flops_per_step": gemm_fl, "gemm_TFLOP/s": round(gemm_fl / (bms / 1e3) / 1e12, 1),
             "frac_of_bf16_peak": round(gemm_fl / (bms / 1e3) / 1e12 / b_peak, 4),
             "peak_source": f"{peak_src} {b_key}; {b_reason}", "device_flags": bflags,
-            "clocks": bsampler.summary()}
+            "clocks": b_clocks}
 
     if args.calibrate and world == 1 and not mx and w.dtype == "bf16":
         line["calibration"] = calibrate(cfg, w, dl, weights, stream, local)

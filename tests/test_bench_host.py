@@ -111,7 +111,7 @@ def test_workload_config_names_the_workload_and_its_sizes():
     assert "model" not in c
 
 
-def test_tensor_peak_follows_the_length_of_the_timed_region():
+def test_tensor_peak_follows_the_length_and_clocks_of_the_timed_region():
     peaks = {"hbm_gbs": 6538.0, "bf16_tflops": 1674.7, "bf16_tflops_sustained": 1364.1}
     p, key, why = bench.choose_tensor_peak(peaks, 0.042)     # 20 layer steps: a burst
     assert (p, key) == (1674.7, "bf16_tflops") and "burst" in why
@@ -119,6 +119,14 @@ def test_tensor_peak_follows_the_length_of_the_timed_region():
     assert (p, key) == (1364.1, "bf16_tflops_sustained") and "sustained" in why
     p, key, _ = bench.choose_tensor_peak(peaks, 12.0)
     assert key == "bf16_tflops_sustained"
+    # a short region decides by its clock record: capped and slow -> sustained
+    capped = {"sm_mhz": 990.0, "sm_max_mhz": 1965, "reasons": ["sw_power_cap"], "samples": 106}
+    p, key, why = bench.choose_tensor_peak(peaks, 0.53, capped)
+    assert key == "bf16_tflops_sustained" and "990" in why
+    # at the burst clock, with too few samples, or without the cap: burst
+    for c in (dict(capped, sm_mhz=1965.0), dict(capped, samples=2), dict(capped, reasons=[]), None,
+              {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}):
+        assert bench.choose_tensor_peak(peaks, 0.53, c)[1] == "bf16_tflops", c
 
 
 def test_cpu_model_is_named():
