@@ -184,6 +184,16 @@ class ClockSampler:
                 "samples": len(mhz), "power_w_max": round(max(s[1] for s in self.samples), 1)}
 
 
+def wait_gpu(end_event) -> None:
+    """Wait for a timed region's end event by polling: the wait sleeps between
+    polls, so the clock sampler's thread keeps taking samples while the GPU
+    works through the queued region (a blocking synchronize can starve it)."""
+    import torch
+    while not end_event.query():
+        time.sleep(0.0002)
+    torch.cuda.synchronize()
+
+
 # ----------------------------------------------------------------- oracle timing (CPU)
 def oracle_threads() -> int:
     try:
@@ -378,7 +388,7 @@ def calibrate(cfg, w, dl, weights, stream, local, seconds=3.0):
             for _ in range(reps):
                 fn()
             e1.record(stream)
-            torch.cuda.synchronize()
+            wait_gpu(e1)
         ms = e0.elapsed_time(e1) / reps
         c = smp.summary()
         tf = flops / ms / 1e9
@@ -512,7 +522,7 @@ def main():
         for _ in range(args.steps):
             layer()
         ev1.record(stream)
-        torch.cuda.synchronize()
+        wait_gpu(ev1)
     barrier()
     ms = max_over_ranks(ev0.elapsed_time(ev1)) / args.steps
     value = replicas.job_throughput(w.T, world, ms / 1e3)
@@ -605,7 +615,7 @@ def main():
             for evs in all_evs:
                 staged(evs)
             rb1.record(stream)
-            torch.cuda.synchronize()
+            wait_gpu(rb1)
         region_b_s = max_over_ranks(rb0.elapsed_time(rb1)) / 1e3
         clocks_b = bsampler.summary()
         stage_ms = {n: 0.0 for n in names}
@@ -784,7 +794,7 @@ def main():
             for _ in range(reps):
                 layer()
             s1.record(stream)
-            torch.cuda.synchronize()
+            wait_gpu(s1)
         barrier()
         s_ms = max_over_ranks(s0.elapsed_time(s1)) / reps
         line["steady_state"] = {"steps": reps, "seconds": round(s_ms * reps / 1e3, 2),
@@ -827,7 +837,7 @@ def main():
             for _ in range(n_b):
                 bwd_step()
             e1.record(stream)
-            torch.cuda.synchronize()
+            wait_gpu(e1)
         barrier()
         bms = max_over_ranks(e0.elapsed_time(e1)) / n_b
         # GEMM work of one step: forward recompute (6 d f per kept row), dgrad (6 d f)
