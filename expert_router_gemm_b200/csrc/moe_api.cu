@@ -757,6 +757,7 @@ moe_status_t moe_layer_bwd(const moe_config_t* cfg, const moe_weights_t* weights
   if (D.fs > 0 && (!aligned16(weights->ws1) || !aligned16(weights->ws3) || !aligned16(weights->ws2) ||
                    !aligned16(grads->dws1) || !aligned16(grads->dws3) || !aligned16(grads->dws2)))
     return MOE_ERR_MISALIGNED;
+  if (!aligned16(weights->w_router_split)) return MOE_ERR_MISALIGNED;
   const BwdLayout B = bwd_layout(D);
   if ((s = check_ws(ws, ws_bytes, B.end)) != MOE_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -798,7 +799,7 @@ moe_status_t moe_layer_bwd(const moe_config_t* cfg, const moe_weights_t* weights
   moe_stats_t rs{};
   rs.counts = at<int32_t*>(ws, B.counts);
   if ((s = do_route(D, x, weights->w_router, weights->router_bias, weights->selection_bias, nullptr, logits, idx, w,
-                    &rs, ws, st)) != MOE_OK)
+                    &rs, ws, st, weights->w_router_split)) != MOE_OK)
     return s;
   if ((s = do_dispatch(D, x, idx, row_map, seg_off, seg_count, xp, nullptr, nullptr, ws, st)) != MOE_OK) return s;
   if ((s = do_ffn(D, xp, seg_off, seg_count, weights->w1, weights->w3, weights->w2, f, false, h, o, ws, st, g, u)) !=

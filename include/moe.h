@@ -421,7 +421,9 @@ moe_status_t moe_layer_fwd(const moe_config_t* cfg, const moe_weights_t* weights
  * gradient; P_i the mean softmax score) and z_loss the z_loss statistic.  The
  * routing decisions (top-k set, capacity drops) carry no gradient, nor does the
  * selection bias.  The call recomputes the forward pass from x (activation
- * recomputation) and needs nothing saved from it.  bf16 layers with
+ * recomputation) and needs nothing saved from it; a router split in
+ * weights->w_router_split (moe_router_split) is used there as in
+ * moe_layer_fwd, with the same result.  bf16 layers with
  * gemm_format MOE_GEMM_ACT and seg_align a multiple of 64 (MOE_ERR_UNSUPPORTED
  * otherwise).  Weight gradients are fp32 and overwrite their buffers; dx is
  * bf16.  Deterministic.

@@ -132,6 +132,21 @@ def test_layer_backward_deterministic_and_empty():
         assert not np.any(z0[key]), key
 
 
+def test_layer_backward_with_a_router_split_made_once_is_unchanged():
+    """moe_layer_bwd with the bf16 split of W_r passed in (moe_router_split, made
+    once) gives the gradients it gives when its forward recompute splits W_r
+    itself, byte for byte (the wide router: CTA pairs)."""
+    w, aux, z = CASES[3]
+    inp = synth.make_inputs(w)
+    dl = moe.to_device(inp, moe.config_from_workload(w))
+    dy = synth.f32_to_bf16_bits(synth.normal_f32(12, 78, (w.T, w.d)))
+    a = _gpu_backward(dl, dy, aux, z)
+    dl.split_router()
+    b = _gpu_backward(dl, dy, aux, z)
+    for key in a:
+        assert np.array_equal(a[key].view(np.uint8), b[key].view(np.uint8)), key
+
+
 EDGE = [
     # capacity 0: every slot dropped, only the router path carries gradient
     (Workload("bwd-cap0", T=128, d=128, N=4, k=2, f=128, capacity_factor=0.0), 0.05, 0.01, None),
