@@ -191,6 +191,21 @@ def test_other_entry_points_validate():
     assert moe.raw_call("moe_read_flags", None, sz(256), None, None) == INVALID
 
 
+def test_router_split_alignment_is_checked_by_the_layer_calls():
+    # a misaligned w_router_split is refused on the host, forward and backward alike
+    cfg = moe.make_config(T=64, d=128, N=128, k=8, f=128, capacity_factor=1.0, dtype="bf16")
+    lb, _, _ = moe.moe_workspace_size(cfg)
+    bb = moe.moe_backward_workspace_size(cfg)
+    c = ctypes.byref(cfg)
+    sz = ctypes.c_size_t
+    w = moe.make_weights(0x100, w1=0x1000, w3=0x2000, w2=0x3000, w_router_split=0x8008)
+    assert moe.raw_call("moe_layer_fwd", c, ctypes.byref(w), 0x1000, 0x2000, None, 0x7000,
+                        sz(lb), None) == MISAL
+    g = moe.make_grads(dx=0x9000, dw_router=0xa000, dw1=0xb000, dw3=0xc000, dw2=0xd000)
+    assert moe.raw_call("moe_layer_bwd", c, ctypes.byref(w), 0x1000, 0x2000, ctypes.c_float(0.01),
+                        ctypes.c_float(1e-3), ctypes.byref(g), 0x7000, sz(bb), None) == MISAL
+
+
 def test_header_documents_every_entry_point():
     text = open(moe.HEADER_PATH).read()
     for f in moe.header_functions():
