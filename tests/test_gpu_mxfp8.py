@@ -118,6 +118,29 @@ def _run_mx(w: Workload):
     return inp, cfg, dl, y, st
 
 
+@pytest.mark.slow
+def test_mx_layer_at_the_bench_expert_shapes():
+    """The FP8 layer at the Qwen3-shaped workload's per-expert shapes (d=4096,
+    f=1536, top-8, capacity 512 rows per expert, about 500 rows each) with 32
+    of its 128 experts and T=2048: GEMM1 accumulates over K=4096 and GEMM2
+    writes 16 column tiles per row block, as in the benchmark's FP8 launches.
+    256 sampled tokens against the FP8 oracle, within the same tolerance."""
+    from dataclasses import replace
+    from expert_router_gemm_b200 import configs
+    w = replace(configs.QWEN3, name="qwen3-shaped-N32-T2048", T=2048, N=32)
+    assert moe.moe_capacity(moe.config_from_workload(w)) == 512
+    inp, cfg, dl, y, st = _run_mx(w)
+    ws = gu.op_workspace(cfg)
+    logits = torch.empty((w.T, w.N), device="cuda")
+    idx = torch.empty((w.T, w.k), dtype=torch.int32, device="cuda")
+    wt = torch.empty((w.T, w.k), device="cuda")
+    moe.moe_route(cfg, dl.x, dl.w_router, dl.bias, None, logits, idx, wt, None, ws)
+    r = _dispatch_mx(cfg, dl.x, idx)
+    rel, n, flips = compare_layer(inp, w, y, gu.host(idx), gu.host(r["row_map"]), gu.host(logits),
+                                  tol=TOL_MX, sample=256, mxfp8=True)
+    print(f"{w.name}: rel_frob vs FP8 oracle {rel:.3e} ({n} tokens, {flips} flips)")
+
+
 @pytest.mark.parametrize("w", SMALL, ids=[w.name for w in SMALL])
 def test_mx_layer_vs_oracle(w):
     inp, cfg, dl, y, st = _run_mx(w)
