@@ -40,6 +40,11 @@ SMALL = [
     Workload("top3-shared-bf16", T=600, d=192, N=12, k=3, f=192, f_shared=64, capacity_factor=1.0),
     # the largest expert count with the largest top-k
     Workload("n256-top32-bf16", T=256, d=128, N=256, k=32, f=64, capacity_factor=1.25),
+    # degenerate shapes: one token (capacity 1), top-1 routing, one expert (a
+    # dense SwiGLU MLP with weight 1; the router's one column padded to 64)
+    Workload("one-token-bf16", T=1, d=128, N=8, k=2, f=128, capacity_factor=1.0),
+    Workload("top1-bf16", T=700, d=256, N=16, k=1, f=192, capacity_factor=1.0),
+    Workload("one-expert-bf16", T=300, d=128, N=1, k=1, f=128, capacity_factor=1.0),
 ]
 
 F32 = [
