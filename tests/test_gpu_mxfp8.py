@@ -105,6 +105,9 @@ SMALL = [
     Workload("mx-finegrained", T=1024, d=256, N=128, k=8, f=256, capacity_factor=1.0),
     Workload("mx-shared", T=520, d=256, N=16, k=4, f=128, f_shared=256, capacity_factor=1.25),
     Workload("mx-deep-k", T=512, d=2048, N=4, k=2, f=1024, capacity_factor=1.0),
+    # degenerate shapes: one token, top-1 routing over one expert
+    Workload("mx-one-token", T=1, d=256, N=8, k=2, f=128, capacity_factor=1.0),
+    Workload("mx-one-expert", T=300, d=128, N=1, k=1, f=256, capacity_factor=1.0),
 ]
 
 
