@@ -141,3 +141,39 @@ def test_cpu_baseline_covers_the_whole_small_layer():
     assert e["kind"] == "oracle" and e["extrapolated"] is False and e["value"] > 0
     assert e["cores"] >= 1 and e["cpu_model"] and "whole layer" in e["sample"]
     assert "tiny-fp32" in bench.FULL_LAYER_WORKLOADS and "qwen3-moe-shaped" in bench.FULL_LAYER_WORKLOADS
+
+
+def test_waiting_for_a_timed_region_polls_and_lets_other_threads_run(monkeypatch):
+    """wait_gpu polls the region's end event with short sleeps (a blocking
+    synchronize kept the clock sampler's thread from running), then
+    synchronises once the event has completed."""
+    import threading
+    import torch
+
+    calls = {"sync": 0}
+    monkeypatch.setattr(torch.cuda, "synchronize", lambda *a, **k: calls.__setitem__("sync", calls["sync"] + 1))
+
+    class Event:
+        def __init__(self):
+            self.n = 0
+
+        def query(self):
+            self.n += 1
+            return self.n >= 50
+
+    ticks = []
+    stop = threading.Event()
+
+    def sampler():
+        while not stop.is_set():
+            ticks.append(1)
+            stop.wait(0.0005)
+
+    t = threading.Thread(target=sampler)
+    t.start()
+    ev = Event()
+    bench.wait_gpu(ev)
+    stop.set()
+    t.join()
+    assert ev.n == 50 and calls["sync"] == 1
+    assert len(ticks) > 1          # the other thread ran while the wait polled
